@@ -1,0 +1,166 @@
+/*
+ * ssm_oracle.c -- plain fp64 CPU oracle for the selective state-space scan (S6).
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker, not the product: only the
+ * test suite, the smoke check and the benchmark's CPU-baseline leg may load it.
+ * It shares no code, header or constant with the CUDA library and must never be
+ * linked into it.
+ *
+ * What it computes, written out as the definition with no blocking, fusion or
+ * reordering (every index is spelled out so it can be checked by eye):
+ *
+ *   for every sequence b and channel d, starting from h = h0[b,d,:] (zero if absent):
+ *     for t = 0 .. L-1:
+ *       v      = delta[b,d,t] + bias[d]                      (bias optional)
+ *       Delta  = softplus(v) if the flag is set, else v
+ *       for n = 0 .. N-1:
+ *         Abar = exp(Delta * A[d,n])                         zero-order hold, decay factor
+ *         Bbar = Delta * B[b,t,n]                            Euler input gain (default)
+ *              = expm1(Delta*A[d,n]) / A[d,n] * B[b,t,n]     exact zero-order hold (mode 1)
+ *         h[n] = Abar * h[n] + Bbar * x[b,d,t]               the linear recurrence
+ *       y      = sum_n C[b,t,n] * h[n]  +  D[d] * x[b,d,t]   readout plus skip (D optional)
+ *       y     *= z * sigmoid(z)                              SiLU gate (z optional)
+ *     final_state[b,d,:] = h
+ *
+ * Sources (page title, section / equation):
+ *  - "Module 19: State-Space Models (Mamba)" (learnllm), "The Math: The State-Space
+ *    Recurrence": Abar = exp(Delta A), exact ZOH Bbar = A^-1 (exp(Delta A) - I) B,
+ *    its small-step (Euler) limit Bbar ~ Delta B, which the lesson names as the form
+ *    Mamba's own kernel uses, and the recurrence h_t = Abar h_{t-1} + Bbar x_t,
+ *    y_t = C h_t.
+ *  - "Beyond attention with Mamba..." (xmarva lesson 10), section 3 "Selectivity":
+ *    h_t = exp(Delta_t a) h_{t-1} + Delta_t b_t x_t, y_t = c_t^T h_t; section 4 "The
+ *    Mamba block": Delta = softplus(dt_proj(seed) + bias), the skip y + u*D, then the
+ *    gate y * SiLU(z), in that order; section 7: the same recurrence for one token.
+ *  - "State-space models (Mamba, S4, hybrids)" (askaiml), section 1: y_t = C h_t + D x_t.
+ *
+ * Readings where the pages are silent: h0 = 0 unless given (the learnllm lesson unrolls
+ * the recurrence starting at a zero state); softplus(v) is written in the overflow-free
+ * form max(v,0) + log1p(exp(-|v|)), which is the same function; the exact-ZOH gain at
+ * A = 0 takes its limit Delta * B.
+ *
+ * Build:  gcc -O2 -fopenmp -shared -fPIC ssm_oracle.c -o libssm_oracle.so -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double oracle_softplus(double v)
+{
+    /* softplus(v) = log(1 + e^v); the identity softplus(v) = v + softplus(-v) keeps
+     * exp() from overflowing for large v. */
+    return (v > 0.0 ? v : 0.0) + log1p(exp(-fabs(v)));
+}
+
+static double oracle_silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+/* One token of the recurrence for one (sequence, channel): updates h[0..N) in place and
+ * returns the gated output.  delta_t is the step after any bias / softplus. */
+static double oracle_token(double *h, int64_t N, double delta_t, double x_t,
+                           const double *A_d,  /* A[d, 0..N)        */
+                           const double *B_t,  /* B[b, t, 0..N)     */
+                           const double *C_t,  /* C[b, t, 0..N)     */
+                           int has_D, double D_d, int has_z, double z_t, int zoh_exact)
+{
+    double y = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+        double a = A_d[n];
+        double Abar = exp(delta_t * a);
+        double Bbar;
+        if (zoh_exact)
+            Bbar = (a == 0.0 ? delta_t : expm1(delta_t * a) / a) * B_t[n];
+        else
+            Bbar = delta_t * B_t[n];
+        h[n] = Abar * h[n] + Bbar * x_t;
+        y += C_t[n] * h[n];
+    }
+    if (has_D)
+        y += D_d * x_t;
+    if (has_z)
+        y *= oracle_silu(z_t);
+    return y;
+}
+
+/*
+ * Full-sequence scan.
+ *   x, delta, z, y : [batch][dim][seqlen]
+ *   B, C           : [batch][seqlen][dstate]
+ *   A              : [dim][dstate]
+ *   D, delta_bias  : [dim]                 (NULL = absent)
+ *   h0, final_state: [batch][dim][dstate]  (NULL = zero start / not wanted)
+ *   z              : NULL = no gate
+ * nthreads <= 0 uses the OpenMP default.  Returns the number of threads used, or -1
+ * for a size it cannot handle (dstate above 256, negative sizes).
+ */
+int oracle_scan(const double *x, const double *delta, const double *delta_bias,
+                int delta_softplus, const double *A, const double *B, const double *C,
+                const double *D, const double *z, const double *h0, int zoh_exact,
+                double *y, double *final_state,
+                int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int nthreads)
+{
+    int used = 1;
+    if (dstate < 0 || dstate > 256 || batch < 0 || dim < 0 || seqlen < 0)
+        return -1;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    const int64_t channels = batch * dim;
+#pragma omp parallel
+    {
+#ifdef _OPENMP
+#pragma omp single
+        used = omp_get_num_threads();
+#endif
+        double h[256];
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t ch = 0; ch < channels; ++ch) {
+            const int64_t b = ch / dim;
+            const int64_t d = ch % dim;
+            for (int64_t n = 0; n < dstate; ++n)
+                h[n] = h0 ? h0[(b * dim + d) * dstate + n] : 0.0;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                const int64_t i = (b * dim + d) * seqlen + t;
+                double v = delta[i] + (delta_bias ? delta_bias[d] : 0.0);
+                double dt = delta_softplus ? oracle_softplus(v) : v;
+                y[i] = oracle_token(h, dstate, dt, x[i], A + d * dstate,
+                                    B + (b * seqlen + t) * dstate,
+                                    C + (b * seqlen + t) * dstate,
+                                    D != NULL, D ? D[d] : 0.0,
+                                    z != NULL, z ? z[i] : 0.0, zoh_exact);
+            }
+            if (final_state)
+                for (int64_t n = 0; n < dstate; ++n)
+                    final_state[(b * dim + d) * dstate + n] = h[n];
+        }
+    }
+    return used;
+}
+
+/*
+ * One decode step (one token per sequence), state updated in place.
+ *   state          : [batch][dim][dstate]   in/out
+ *   x, delta, z, y : [batch][dim]           delta is the final step (already activated)
+ *   B, C           : [batch][dstate]
+ *   A              : [dim][dstate];  D: [dim] or NULL;  z: NULL = no gate
+ */
+void oracle_step(double *state, const double *x, const double *delta, const double *A,
+                 const double *B, const double *C, const double *D, const double *z,
+                 double *y, int64_t batch, int64_t dim, int64_t dstate)
+{
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t i = b * dim + d;
+            y[i] = oracle_token(state + i * dstate, dstate, delta[i], x[i], A + d * dstate,
+                                B + b * dstate, C + b * dstate, D != NULL, D ? D[d] : 0.0,
+                                z != NULL, z ? z[i] : 0.0, 0);
+        }
+}

@@ -1,0 +1,125 @@
+"""Seeded synthetic inputs for the selective scan and the decode step.
+
+This module only draws random numbers in the shapes and distributions of the
+workloads; it computes nothing of the scan itself, so the CUDA path and the fp64
+oracle can both be fed from it.
+
+Workloads (sizes follow the Mamba shapes the pages use: mamba-130m has
+d_inner = 1536 and N = 16, xmarva lesson 10 section 4; the 2.8b shape has
+d_inner = 5120; the million-token length follows the long-context claims in
+learnllm "Module 19" and askaiml section 4):
+
+=============  ======  =========  =======  ===  =====================================
+name           batch   L          d_inner  N    dtype of x, delta, z, B, C
+=============  ======  =========  =======  ===  =====================================
+tiny           1       64         8        4    fp32
+mamba130m      8       2048       1536     16   bf16 (A, D, bias, state fp32)
+mamba2p8b      4       4096       5120     16   bf16
+long1m         1       1048576    1536     16   bf16
+decode         256     1 x 64     5120     16   bf16 tokens, fp32 state
+=============  ======  =========  =======  ===  =====================================
+
+Draw order (one generator seeded once): x, delta_raw, z, B, C, D, dt.
+  x, z ~ N(0, 1);  delta_raw = 0.5 * N(0, 1);  B, C ~ N(0, 1) per (b, t, n);
+  D ~ N(0, 1);  dt ~ U[1e-3, 1e-1] per channel (log-uniform on that range for the
+  2.8b shape);  delta_bias = log(expm1(dt)), evaluated in fp64 and stored fp32, so
+  that softplus(delta_bias) = dt;  A[d, n] = -(n + 1).
+The decode workload draws an N(0, 1) fp32 state and, per token, a positive step
+delta = dt * exp(0.5 * N(0, 1)) (the step is an input of the decode call, already
+positive), with x, z, B, C as above.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+CONFIGS = {
+    "tiny": dict(batch=1, seqlen=64, dim=8, dstate=4, dtype=torch.float32, dt_dist="uniform"),
+    "mamba130m": dict(batch=8, seqlen=2048, dim=1536, dstate=16, dtype=torch.bfloat16,
+                      dt_dist="uniform"),
+    "mamba2p8b": dict(batch=4, seqlen=4096, dim=5120, dstate=16, dtype=torch.bfloat16,
+                      dt_dist="loguniform"),
+    "long1m": dict(batch=1, seqlen=1 << 20, dim=1536, dstate=16, dtype=torch.bfloat16,
+                   dt_dist="uniform"),
+    "decode": dict(batch=256, steps=64, dim=5120, dstate=16, dtype=torch.bfloat16,
+                   dt_dist="uniform"),
+}
+
+DT_MIN, DT_MAX = 1e-3, 1e-1
+
+
+def _generator(device, seed):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _draw_dt(n, dist, g, device):
+    u = torch.rand(n, generator=g, device=device, dtype=torch.float64)
+    if dist == "uniform":
+        return DT_MIN + (DT_MAX - DT_MIN) * u
+    if dist == "loguniform":
+        return torch.exp(math.log(DT_MIN) + (math.log(DT_MAX) - math.log(DT_MIN)) * u)
+    raise ValueError("unknown dt distribution %r" % (dist,))
+
+
+def make_scan_inputs(batch, dim, seqlen, dstate, dtype=torch.float32, device="cpu", seed=0,
+                     dt_dist="uniform"):
+    """Inputs of one selective-scan call, as a dict of tensors on ``device``.
+
+    Keys: x, delta, z ([batch, dim, seqlen], ``dtype``); B, C ([batch, seqlen, dstate],
+    ``dtype``); A ([dim, dstate] fp32); D, delta_bias ([dim] fp32).  ``delta`` is the raw
+    step: the scan adds ``delta_bias`` and applies softplus.
+    """
+    g = _generator(device, seed)
+    f32 = torch.float32
+
+    def normal(*shape, scale=1.0):
+        t = torch.randn(*shape, generator=g, device=device, dtype=f32)
+        if scale != 1.0:
+            t.mul_(scale)
+        return t.to(dtype)
+
+    x = normal(batch, dim, seqlen)
+    delta = normal(batch, dim, seqlen, scale=0.5)
+    z = normal(batch, dim, seqlen)
+    B = normal(batch, seqlen, dstate)
+    C = normal(batch, seqlen, dstate)
+    D = torch.randn(dim, generator=g, device=device, dtype=f32)
+    dt = _draw_dt(dim, dt_dist, g, device)
+    delta_bias = torch.log(torch.expm1(dt)).to(f32)
+    A = -torch.arange(1, dstate + 1, device=device, dtype=f32).repeat(dim, 1).contiguous()
+    return dict(x=x, delta=delta, z=z, B=B, C=C, A=A, D=D, delta_bias=delta_bias)
+
+
+def make_config_inputs(name, device="cpu", seed=0):
+    c = CONFIGS[name]
+    if name == "decode":
+        return make_decode_inputs(c["batch"], c["dim"], c["dstate"], c["steps"], c["dtype"],
+                                  device=device, seed=seed)
+    return make_scan_inputs(c["batch"], c["dim"], c["seqlen"], c["dstate"], c["dtype"],
+                            device=device, seed=seed, dt_dist=c["dt_dist"])
+
+
+def make_decode_inputs(batch, dim, dstate, steps, dtype=torch.bfloat16, device="cpu", seed=0,
+                       dt_dist="uniform"):
+    """Inputs of ``steps`` chained decode calls.
+
+    Keys: state ([batch, dim, dstate] fp32, N(0,1)); x, delta, z ([steps, batch, dim],
+    ``dtype``; delta positive); B, C ([steps, batch, dstate], ``dtype``); A ([dim, dstate]
+    fp32); D ([dim] fp32).
+    """
+    g = _generator(device, seed)
+    f32 = torch.float32
+    state = torch.randn(batch, dim, dstate, generator=g, device=device, dtype=f32)
+    x = torch.randn(steps, batch, dim, generator=g, device=device, dtype=f32).to(dtype)
+    noise = torch.randn(steps, batch, dim, generator=g, device=device, dtype=f32)
+    z = torch.randn(steps, batch, dim, generator=g, device=device, dtype=f32).to(dtype)
+    B = torch.randn(steps, batch, dstate, generator=g, device=device, dtype=f32).to(dtype)
+    C = torch.randn(steps, batch, dstate, generator=g, device=device, dtype=f32).to(dtype)
+    D = torch.randn(dim, generator=g, device=device, dtype=f32)
+    dt = _draw_dt(dim, dt_dist, g, device).to(f32)
+    delta = (dt[None, None, :] * torch.exp(0.5 * noise)).to(dtype)
+    A = -torch.arange(1, dstate + 1, device=device, dtype=f32).repeat(dim, 1).contiguous()
+    return dict(state=state, x=x, delta=delta, z=z, B=B, C=C, A=A, D=D)

@@ -1,0 +1,287 @@
+"""Pins of the fp64 oracle against facts the pages print and the mathematics fixes.
+
+Each test drives the oracle's sequential scan (or decode step) through a worked example
+whose answer does not come from the oracle: the printed numbers of the pages (fixtures
+under tests/golden/, each with its citation), closed forms, and independent
+implementations (a Hillis-Steele scan over affine pairs, the O(L^2) convolution of a
+time-invariant SSM).  The set is chosen so that a dropped term, a wrong sign, a wrong
+index or a transposed operand in the oracle fails at least one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from tests.conftest import load_golden
+
+
+def _printed(value, decimals):
+    """Tolerance of a number printed with ``decimals`` digits after the point."""
+    return 0.5 * 10.0 ** (-decimals) + 1e-12
+
+
+def _one_state(abar_list, gain_list, x_list, c=1.0, h0=None, zoh=False):
+    """Run the oracle scan on one channel with one state.
+
+    The decay Abar_t and the Euler gain Bbar_t are planted through Delta_t and B_t:
+    A = -1, Delta_t = -ln(Abar_t), B_t = Bbar_t / Delta_t (so Delta_t B_t = Bbar_t).
+    """
+    abar = np.asarray(abar_list, dtype=np.float64)
+    L = len(x_list)
+    delta = -np.log(abar) * np.ones(L)
+    B = (np.asarray(gain_list, dtype=np.float64) * np.ones(L)) / delta
+    y, hN = oracle.scan(
+        x=np.asarray(x_list, dtype=np.float64).reshape(1, 1, L),
+        delta=delta.reshape(1, 1, L),
+        A=np.array([[-1.0]]),
+        B=B.reshape(1, L, 1),
+        C=(c * np.ones(L)).reshape(1, L, 1),
+        h0=None if h0 is None else np.array(h0, dtype=np.float64).reshape(1, 1, 1),
+        zoh_exact=zoh,
+    )
+    return y[0, 0], hN[0, 0]
+
+
+def test_toy_recurrence_printed_states():
+    g = load_golden("toy_recurrence.json")
+    y, _ = _one_state([g["Abar"]] * 4, [g["Bbar"]] * 4, g["x"])
+    tol = _printed(None, g["printed_decimals"])
+    np.testing.assert_allclose(y, g["h_printed"], atol=tol, rtol=0)
+    # the last state, unrounded: 0.8^3 * 1 + 0.2 * 10
+    assert abs(y[3] - 2.512) < 1e-12
+
+
+def test_impulse_response_halves():
+    g = load_golden("impulse_response.json")
+    y, _ = _one_state([g["Abar"]] * 5, [g["Bbar"]] * 5, g["x"], c=g["C"])
+    np.testing.assert_allclose(y, g["y_printed"], atol=_printed(None, g["printed_decimals"]))
+    np.testing.assert_allclose(y, [0.5 ** t for t in range(5)], rtol=1e-13)
+
+
+def test_zoh_decay_percentages():
+    g = load_golden("zoh_decay.json")
+    for case in g["cases"]:
+        # state 1, no input: one step leaves Abar = exp(Delta * A) of it
+        y, hN = oracle.scan(x=np.zeros((1, 1, 1)), delta=np.full((1, 1, 1), case["delta"]),
+                            A=np.array([[g["A"]]]), B=np.ones((1, 1, 1)), C=np.ones((1, 1, 1)),
+                            h0=np.ones((1, 1, 1)))
+        kept = 100.0 * hN[0, 0, 0]
+        assert abs(kept - case["kept_percent_printed"]) <= 0.5, (case, kept)
+        # the sign of A matters: exp(+Delta) would keep more than everything
+        assert hN[0, 0, 0] < 1.0
+
+
+def test_discretize_exact_zoh_printed():
+    g = load_golden("discretize_zoh.json")
+    N = len(g["A"])
+    A = np.array(g["A"]).reshape(1, N)
+    tol = _printed(None, g["printed_decimals"])
+    # Abar: start from h = 1 with no input, one step
+    _, hA = oracle.scan(x=np.zeros((1, 1, 1)), delta=np.full((1, 1, 1), g["delta"]), A=A,
+                        B=np.array(g["B"]).reshape(1, 1, N), C=np.zeros((1, 1, N)),
+                        h0=np.ones((1, 1, N)), zoh_exact=True)
+    np.testing.assert_allclose(hA[0, 0], g["Abar_printed"], atol=tol)
+    # Bbar: start from h = 0, input x = 1, one step (exact-ZOH gain mode)
+    _, hB = oracle.scan(x=np.ones((1, 1, 1)), delta=np.full((1, 1, 1), g["delta"]), A=A,
+                        B=np.array(g["B"]).reshape(1, 1, N), C=np.zeros((1, 1, N)),
+                        zoh_exact=True)
+    np.testing.assert_allclose(hB[0, 0], g["Bbar_printed"], atol=tol)
+
+
+def test_exact_over_euler_ratio_table():
+    g = load_golden("euler_ratio.json")
+    tol = _printed(None, g["printed_decimals"])
+    for p, printed in zip(g["p"], g["ratio_printed"]):
+        kw = dict(x=np.ones((1, 1, 1)), delta=np.full((1, 1, 1), p), A=np.array([[-1.0]]),
+                  B=np.ones((1, 1, 1)), C=np.ones((1, 1, 1)))
+        _, h_exact = oracle.scan(zoh_exact=True, **kw)
+        _, h_euler = oracle.scan(zoh_exact=False, **kw)
+        assert abs(h_euler[0, 0, 0] - p) < 1e-15          # Euler gain is Delta * B
+        ratio = h_exact[0, 0, 0] / h_euler[0, 0, 0]
+        assert abs(ratio - printed) <= tol, (p, ratio, printed)
+
+
+def test_affine_scan_printed_by_all_three_routes():
+    g = load_golden("affine_scan.json")
+    tol = _printed(None, g["printed_decimals"])
+    loop = oracle.affine_scan_loop(g["a"], g["b"])
+    par = oracle.affine_scan_hillis_steele(g["a"], g["b"])
+    np.testing.assert_allclose(loop, g["h_printed"], atol=tol)
+    np.testing.assert_allclose(par, g["h_printed"], atol=tol)
+    # the C loop, with a_t planted as the decay and b_t as the Euler gain at x = 1
+    y, _ = _one_state(g["a"], g["b"], [1.0] * len(g["a"]))
+    np.testing.assert_allclose(y, loop, rtol=1e-13, atol=1e-15)
+
+
+def test_selectivity_toy_percentages():
+    g = load_golden("selectivity_toy.json")
+    A = np.array([[g["A"]]])
+
+    def survives(deltas):
+        # key value 1 at t = 0, fillers carry no input; the last state is what is left of it
+        L = len(deltas)
+        x = np.zeros((1, 1, L))
+        x[0, 0, 0] = 1.0
+        _, hN = oracle.scan(x=x, delta=np.array(deltas).reshape(1, 1, L), A=A,
+                            B=np.ones((1, L, 1)), C=np.ones((1, L, 1)), zoh_exact=True)
+        return 100.0 * hN[0, 0, 0]
+
+    s = g["selective"]
+    sel = survives([s["key_delta"]] + [s["filler_delta"]] * s["fillers"])
+    assert abs(sel - s["survives_percent_printed"]) <= 0.5, sel
+    f = g["fixed"]
+    fixed = survives([f["delta"]] * (1 + f["fillers"]))
+    assert abs(fixed - f["survives_percent_printed"]) <= 0.05, fixed
+
+
+def test_lti_kernel_taps_torch_seed0_soft_pin():
+    torch = pytest.importorskip("torch")
+    g = load_golden("lti_taps.json")
+    torch.manual_seed(g["seed"])
+    abar = (torch.rand(4) * 0.9 + 0.05).double().numpy()
+    bbar = torch.randn(4).double().numpy()
+    c = torch.randn(4).double().numpy()
+    taps = oracle.lti_kernel(abar, bbar, c, 4)
+    np.testing.assert_allclose(taps, g["taps_printed"], atol=_printed(None, g["printed_decimals"]))
+
+
+def test_recurrence_equals_causal_convolution_when_time_invariant():
+    # Delta, B, C fixed over t: the scan is the convolution with K = (C Bbar, C Abar Bbar, ...)
+    rng = np.random.default_rng(1)
+    N, L = 5, 23
+    A = -rng.uniform(0.2, 3.0, size=(1, N))
+    delta0 = 0.37
+    Bv = rng.normal(size=N)
+    Cv = rng.normal(size=N)
+    x = rng.normal(size=L)
+    y, _ = oracle.scan(x=x.reshape(1, 1, L), delta=np.full((1, 1, L), delta0), A=A,
+                       B=np.tile(Bv, (L, 1)).reshape(1, L, N), C=np.tile(Cv, (L, 1)).reshape(1, L, N))
+    y_conv = oracle.lti_conv(np.exp(delta0 * A[0]), delta0 * Bv, Cv, x)
+    np.testing.assert_allclose(y[0, 0], y_conv, rtol=1e-11, atol=1e-12)
+
+
+def _random_case(rng, batch=2, dim=3, L=37, N=4):
+    return dict(
+        x=rng.normal(size=(batch, dim, L)),
+        delta=0.5 * rng.normal(size=(batch, dim, L)),
+        z=rng.normal(size=(batch, dim, L)),
+        B=rng.normal(size=(batch, L, N)),
+        C=rng.normal(size=(batch, L, N)),
+        A=-rng.uniform(0.5, 4.0, size=(dim, N)),
+        D=rng.normal(size=dim),
+        delta_bias=np.log(np.expm1(rng.uniform(1e-3, 1e-1, size=dim))),
+    )
+
+
+@pytest.mark.parametrize("shape", [(1, 3, 37, 4), (2, 3, 16, 5), (3, 2, 9, 16)])
+def test_loop_equals_bruteforce_parallel_scan(shape):
+    batch, dim, L, N = shape
+    case = _random_case(np.random.default_rng(sum(shape)), batch, dim, L, N)
+    y, hN = oracle.scan(delta_softplus=True, **case)
+    y2, h2 = oracle.scan_parallel_reference(delta_softplus=True, **case)
+    np.testing.assert_allclose(y, y2, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(hN, h2, rtol=1e-10, atol=1e-12)
+    # the distinguishing power of this pin: a transposed B ([b, n, t]) must not agree
+    if L != N:
+        bad = dict(case)
+        bad["B"] = np.ascontiguousarray(case["B"].reshape(batch, N, L).transpose(0, 2, 1))
+        yb, _ = oracle.scan(delta_softplus=True, **bad)
+        assert np.max(np.abs(yb - y2)) > 1e-3
+
+
+def test_causality_outputs_before_edit_are_identical():
+    rng = np.random.default_rng(7)
+    case = _random_case(rng, 2, 3, 40, 4)
+    y, _ = oracle.scan(delta_softplus=True, **case)
+    t0 = 17
+    edited = {k: v.copy() for k, v in case.items()}
+    edited["x"][..., t0] += 4.0
+    edited["delta"][..., t0] -= 1.0
+    edited["z"][..., t0] += 2.0
+    edited["B"][:, t0, :] *= -3.0
+    edited["C"][:, t0, :] += 1.0
+    y2, _ = oracle.scan(delta_softplus=True, **edited)
+    assert np.array_equal(y[..., :t0], y2[..., :t0])
+    assert not np.array_equal(y[..., t0], y2[..., t0])
+
+
+def test_skip_and_gate_closed_form():
+    # With C = 0 the state contributes nothing: y = D x SiLU(z).  sigmoid(0) = 1/2,
+    # sigmoid(ln 3) = 3/4, sigmoid(-ln 3) = 1/4.
+    zs = np.array([0.0, math.log(3.0), -math.log(3.0)])
+    x = np.array([2.0, 2.0, 2.0])
+    L = 3
+    y, _ = oracle.scan(x=x.reshape(1, 1, L), delta=np.full((1, 1, L), 0.3), A=np.array([[-1.0]]),
+                       B=np.ones((1, L, 1)), C=np.zeros((1, L, 1)), D=np.array([1.5]),
+                       z=zs.reshape(1, 1, L))
+    expect = 1.5 * x * zs * np.array([0.5, 0.75, 0.25])
+    np.testing.assert_allclose(y[0, 0], expect, rtol=1e-14, atol=1e-15)
+    # with no gate and no skip the output is the bare readout C h
+    y2, h2 = oracle.scan(x=x.reshape(1, 1, L), delta=np.full((1, 1, L), 0.3), A=np.array([[-1.0]]),
+                         B=np.ones((1, L, 1)), C=np.full((1, L, 1), 2.0))
+    assert abs(y2[0, 0, -1] - 2.0 * h2[0, 0, 0]) < 1e-15
+
+
+def test_softplus_and_bias_special_values():
+    # softplus(0) = ln 2, so with A = -1 one step keeps exp(-ln 2) = 1/2 of the state;
+    # softplus(ln 3) = ln 4 keeps 1/4; bias = log(expm1(dt)) gives back Delta = dt.
+    def kept(raw, bias):
+        _, hN = oracle.scan(x=np.zeros((1, 1, 1)), delta=np.full((1, 1, 1), raw),
+                            A=np.array([[-1.0]]), B=np.ones((1, 1, 1)), C=np.ones((1, 1, 1)),
+                            delta_bias=np.array([bias]), delta_softplus=True, h0=np.ones((1, 1, 1)))
+        return hN[0, 0, 0]
+
+    assert abs(kept(0.0, 0.0) - 0.5) < 1e-15
+    assert abs(kept(math.log(3.0), 0.0) - 0.25) < 1e-15
+    assert abs(kept(0.25, math.log(3.0) - 0.25) - 0.25) < 1e-14   # bias is added before softplus
+    dt = 0.0375
+    assert abs(kept(0.0, math.log(math.expm1(dt))) - math.exp(-dt)) < 1e-14
+    assert abs(kept(800.0, 0.0)) == 0.0                              # no overflow for large steps
+
+
+def test_small_step_holds_large_step_resets():
+    # Delta -> 0 keeps the state and writes nothing; a large Delta forgets it and
+    # writes Bbar x = Delta B x (Euler gain).
+    _, h_small = oracle.scan(x=np.full((1, 1, 1), 5.0), delta=np.full((1, 1, 1), 1e-9),
+                             A=np.array([[-1.0]]), B=np.ones((1, 1, 1)), C=np.ones((1, 1, 1)),
+                             h0=np.full((1, 1, 1), 3.0))
+    assert abs(h_small[0, 0, 0] - 3.0) < 1e-8
+    _, h_big = oracle.scan(x=np.full((1, 1, 1), 5.0), delta=np.full((1, 1, 1), 60.0),
+                           A=np.array([[-1.0]]), B=np.ones((1, 1, 1)), C=np.ones((1, 1, 1)),
+                           h0=np.full((1, 1, 1), 3.0))
+    assert abs(h_big[0, 0, 0] - 300.0) < 1e-9
+
+
+def test_decode_step_chaining_equals_scan_from_same_state():
+    rng = np.random.default_rng(11)
+    batch, dim, L, N = 3, 4, 12, 6
+    case = _random_case(rng, batch, dim, L, N)
+    h0 = rng.normal(size=(batch, dim, N))
+    # the step takes the final Delta: feed the scan the same steps with no bias/softplus
+    steps = np.log1p(np.exp(case["delta"] + case["delta_bias"][None, :, None]))
+    y, hN = oracle.scan(x=case["x"], delta=steps, A=case["A"], B=case["B"], C=case["C"],
+                        D=case["D"], z=case["z"], h0=h0)
+    st = h0
+    for t in range(L):
+        yt, st = oracle.step(st, case["x"][..., t], steps[..., t], case["A"], case["B"][:, t],
+                             case["C"][:, t], D=case["D"], z=case["z"][..., t])
+        np.testing.assert_allclose(yt, y[..., t], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(st, hN, rtol=1e-13, atol=1e-14)
+
+
+def test_decode_step_hand_example():
+    # one state: h = exp(-0.5 * 2) * 1 + 0.5 * 3 * 2 = e^-1 + 3; y = 0.5 h + 4 * 2 (no gate)
+    y, st = oracle.step(np.ones((1, 1, 1)), np.full((1, 1), 2.0), np.full((1, 1), 0.5),
+                        np.array([[-2.0]]), np.full((1, 1), 3.0), np.full((1, 1), 0.5),
+                        D=np.array([4.0]))
+    h = math.exp(-1.0) + 3.0
+    assert abs(st[0, 0, 0] - h) < 1e-15
+    assert abs(y[0, 0] - (0.5 * h + 8.0)) < 1e-14
+
+
+def test_empty_sequence_keeps_initial_state():
+    y, hN = oracle.scan(x=np.zeros((2, 3, 0)), delta=np.zeros((2, 3, 0)), A=-np.ones((3, 4)),
+                        B=np.zeros((2, 0, 4)), C=np.zeros((2, 0, 4)))
+    assert y.shape == (2, 3, 0)
+    assert np.all(hN == 0.0)
