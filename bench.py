@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 selective scan (S6) and decode step.
+
+One JSON line on rank 0.  A step is one pass of the whole hot path over one batch:
+for the scan workloads one ``ssm_selective_scan_fwd`` call (discretise, recurrence,
+readout, skip, gate, final state), for the decode workload one ``ssm_state_step`` call.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mamba130m]
+  python bench.py --impl reference ...        # the fp64 CPU oracle, timed on host cores
+
+Workloads (selective_state_space_45_b200.inputs.CONFIGS): mamba130m (default: batch 8,
+L 2048, d_inner 1536, N 16, bf16 in/out, fp32 state), mamba2p8b, long1m, decode.
+Multi-GPU: every rank runs its own replica (channels are independent; the path has no
+exchange step), timing is the max over ranks, value counts all ranks' work.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "selective-scan GB/s & tokens·channels/s (1 B200), % of HBM/MUFU roofline"
+UNIT = "tokens*channels/s"
+N_SM = 148
+MUFU_EX2_PER_CLK_PER_SM = 16        # SFU ex2 throughput per SM per clock
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_SM_MHZ = 1965.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mamba130m",
+                    choices=["mamba130m", "mamba2p8b", "long1m", "decode", "tiny"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0,
+                    help="CPU seconds the oracle baseline may spend")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_dist(world, backend, timeout_s=120):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist if world > 1 else None
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(dist, value, device="cpu"):
+    """Max of a float over all ranks (identity on one rank)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(dist, value, device="cpu"):
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ peaks, clocks, traffic
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), sm_max_mhz=float(p.get("sm_max_mhz", FALLBACK_SM_MHZ)),
+                    source="measured (MEASURED_PEAKS.json)")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=FALLBACK_HBM_GBS, sm_max_mhz=FALLBACK_SM_MHZ, source="fallback")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_45_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if taken on these sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f).get("%s %s" % (kernel, workload))
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return float(rec["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return dict(sm_mhz=statistics.median(sm) if sm else None,
+                    sm_max_mhz=float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                    reasons=reasons, samples=len(rows))
+
+
+# ------------------------------------------------------------------ workloads
+
+def scan_counts(batch, dim, L, N, in_size, out_size):
+    """Algorithmic bytes (each input read once, each output written once) and work."""
+    streams = batch * dim * L * (3 * in_size + out_size)          # x, delta, z in; y out
+    bc = 2 * batch * L * N * in_size                               # B, C in
+    params = dim * N * 4 + 2 * dim * 4                             # A; D and delta_bias
+    state = batch * dim * N * 4                                    # final state out
+    return dict(bytes=streams + bc + params + state, exps=batch * L * dim * N,
+                tokch=batch * L * dim)
+
+
+def step_counts(batch, dim, N, in_size, out_size):
+    state = 2 * batch * dim * N * 4                                # read + write in place
+    streams = batch * dim * (3 * in_size + out_size)               # x, delta, z in; y out
+    bc = 2 * batch * N * in_size
+    params = dim * N * 4 + dim * 4
+    return dict(bytes=state + streams + bc + params, exps=batch * dim * N, tokch=batch * dim)
+
+
+class Workload:
+    """Device-resident inputs of one workload, rotated over enough copies that the
+    bytes touched between two uses of the same copy exceed the L2 cache."""
+
+    def __init__(self, name, device, seed=0):
+        import torch
+        from selective_state_space_45_b200 import inputs
+        self.name, self.device = name, device
+        self.cfg = dict(inputs.CONFIGS[name])
+        self.kind = "decode" if name == "decode" else "scan"
+        c = self.cfg
+        dt = c["dtype"]
+        esz = torch.tensor([], dtype=dt).element_size()
+        if self.kind == "scan":
+            self.counts = scan_counts(c["batch"], c["dim"], c["seqlen"], c["dstate"], esz, esz)
+        else:
+            self.counts = step_counts(c["batch"], c["dim"], c["dstate"], esz, esz)
+        per_set = self.counts["bytes"]
+        self.nsets = max(1, min(4, -(-int(2.5 * L2_BYTES) // per_set)))
+        self.sets = []
+        for s in range(self.nsets):
+            inp = inputs.make_config_inputs(name, device=device, seed=seed + s)
+            if self.kind == "scan":
+                inp["y"] = torch.empty(inp["x"].shape, device=device, dtype=dt)
+                inp["fs"] = torch.empty(c["batch"], c["dim"], c["dstate"], device=device)
+            else:
+                inp["y"] = torch.empty(c["batch"], c["dim"], device=device, dtype=dt)
+            self.sets.append(inp)
+
+    def launch(self, i, stream=None):
+        import selective_state_space_45_b200 as ssm
+        s = self.sets[i % self.nsets]
+        if self.kind == "scan":
+            ssm.ssm_selective_scan_fwd(s["x"], s["delta"], s["delta_bias"], True, s["A"], s["B"],
+                                       s["C"], s["D"], s["z"], s["y"], s["fs"], stream)
+        else:
+            t = (i // self.nsets) % s["x"].shape[0]
+            ssm.ssm_state_step(s["state"], s["x"][t], s["delta"][t], s["A"], s["B"][t], s["C"][t],
+                               s["D"], s["z"][t], s["y"], stream)
+
+    def description(self):
+        c = self.cfg
+        if self.kind == "scan":
+            return ("%s-shaped selective scan: batch %d, L %d, d_inner %d, N %d, %s x/delta/z/B/C "
+                    "and y, fp32 A/D/bias/state" % (self.name, c["batch"], c["seqlen"], c["dim"],
+                                                     c["dstate"], str(c["dtype"]).split(".")[-1]))
+        return ("decode state step: batch %d, d_inner %d, N %d, fp32 state in place, one %s token "
+                "per sequence" % (c["batch"], c["dim"], c["dstate"], str(c["dtype"]).split(".")[-1]))
+
+
+def kernel_name(kind):
+    return "scan_fwd_kernel" if kind == "scan" else "state_step_kernel"
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def host_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_sample(name, n_target_tokch, seed=0):
+    """Inputs of a channel sample of workload ``name`` (CPU tensors widened to fp64 by the
+    oracle): all sequences, the first k channels, k chosen for ~n_target_tokch units."""
+    import torch
+    from selective_state_space_45_b200 import inputs
+    c = inputs.CONFIGS[name]
+    if name == "decode":
+        k = int(max(1, min(c["dim"], n_target_tokch // c["batch"])))
+        inp = inputs.make_decode_inputs(c["batch"], k, c["dstate"], 1, c["dtype"], device="cpu",
+                                        seed=seed)
+        sample = dict(state=inp["state"], x=inp["x"][0], delta=inp["delta"][0], A=inp["A"],
+                      B=inp["B"][0], C=inp["C"][0], D=inp["D"], z=inp["z"][0])
+        return "decode", sample, c["batch"] * k, "%d sequences x %d of %d channels, one token" % (
+            c["batch"], k, c["dim"])
+    per_channel = c["batch"] * c["seqlen"]
+    k = int(max(1, min(c["dim"], n_target_tokch // per_channel)))
+    L = c["seqlen"]
+    if k == 1 and n_target_tokch < per_channel:  # one channel of one sequence, shortened
+        L = int(max(64, min(L, n_target_tokch)))
+        inp = inputs.make_scan_inputs(1, 1, L, c["dstate"], c["dtype"], device="cpu", seed=seed,
+                                      dt_dist=c["dt_dist"])
+        return "scan", inp, L, "1 channel of 1 sequence, first %d of %d tokens" % (L, c["seqlen"])
+    inp = inputs.make_scan_inputs(c["batch"], k, L, c["dstate"], c["dtype"], device="cpu", seed=seed,
+                                  dt_dist=c["dt_dist"])
+    return "scan", inp, per_channel * k, "%d sequences x %d of %d channels, all %d tokens" % (
+        c["batch"], k, c["dim"], L)
+
+
+def _oracle_call(kind, inp, threads):
+    import oracle
+    if kind == "scan":
+        oracle.scan(x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], D=inp["D"],
+                    z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True, nthreads=threads)
+    else:
+        oracle.step(inp["state"], inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                    z=inp["z"])
+
+
+def oracle_rate(name, threads, budget_s):
+    """Time the oracle as it stands on a bounded sample sized to about ``budget_s`` seconds."""
+    kind, inp, units, what = _oracle_sample(name, 2048 * 16)
+    t0 = time.perf_counter()
+    _oracle_call(kind, inp, threads)
+    probe = max(time.perf_counter() - t0, 1e-4)
+    rate = units / probe
+    kind, inp, units, what = _oracle_sample(name, int(rate * budget_s))
+    t0 = time.perf_counter()
+    _oracle_call(kind, inp, threads)
+    wall = time.perf_counter() - t0
+    return dict(value=units / wall, unit=UNIT, cores=threads if kind == "scan" else 1, kind="oracle",
+                sample=what, seconds=round(wall, 3))
+
+
+def run_reference(args):
+    """The fp64 oracle timed on the host cores, step by step, on bounded samples."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    threads = host_threads()
+    # size each step so that warm-up + timed steps take about two minutes in total
+    per_step_s = max(0.02, min(30.0, 120.0 / max(1, args.steps + args.warmup)))
+    kind, inp, units, what = _oracle_sample(args.workload, 2048 * 16)
+    t0 = time.perf_counter()
+    _oracle_call(kind, inp, threads)
+    rate = units / max(time.perf_counter() - t0, 1e-4)
+    kind, inp, units, what = _oracle_sample(args.workload, int(rate * per_step_s))
+    for _ in range(args.warmup):
+        _oracle_call(kind, inp, threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_call(kind, inp, threads)
+    wall = time.perf_counter() - t0
+    value = units * args.steps / wall
+    cores = threads if kind == "scan" else 1
+    line = dict(metric=METRIC, value=value, unit=UNIT, impl="reference", n_gpus=args.gpus,
+                steps=args.steps, warmup=args.warmup, ms_per_step=1e3 * wall / args.steps,
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                data="synthetic", config=dict(workload=args.workload, sample=what),
+                cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle", sample=what),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def time_e2e(wl, steps, stream):
+    """The same metric through the public API with HOST buffers: every step copies its
+    inputs from pinned host memory, runs the call and reads the outputs back."""
+    import torch
+    import selective_state_space_45_b200 as ssm
+    dev = wl.sets[0]
+    names_in = (["x", "delta", "z", "B", "C", "A", "D", "delta_bias"] if wl.kind == "scan"
+                else ["state", "x", "delta", "z", "B", "C", "A", "D"])
+    names_out = ["y", "fs"] if wl.kind == "scan" else ["y", "state"]
+    host = {}
+    for n in names_in:
+        src = dev[n][0] if (wl.kind == "decode" and n in ("x", "delta", "z", "B", "C")) else dev[n]
+        host[n] = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
+        host[n].copy_(src)
+    outs = {n: torch.empty(dev[n].shape, dtype=dev[n].dtype, pin_memory=True) for n in names_out}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+
+    def one():
+        for n in names_in:
+            dst = dev[n][0] if (wl.kind == "decode" and n in ("x", "delta", "z", "B", "C")) else dev[n]
+            dst.copy_(host[n], non_blocking=True)
+        if wl.kind == "scan":
+            ssm.ssm_selective_scan_fwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"],
+                                       dev["B"], dev["C"], dev["D"], dev["z"], dev["y"], dev["fs"])
+        else:
+            ssm.ssm_state_step(dev["state"], dev["x"][0], dev["delta"][0], dev["A"], dev["B"][0],
+                               dev["C"][0], dev["D"], dev["z"][0], dev["y"])
+        for n in names_out:
+            outs[n].copy_(dev[n], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) / 1e3
+    return dict(value=wl.counts["tokch"] * steps / sec, unit=UNIT, h2d_bytes_per_step=h2d,
+                d2h_bytes_per_step=d2h, ms_per_step=1e3 * sec / steps)
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    import selective_state_space_45_b200 as ssm
+    ssm.load_library()
+
+    wl = Workload(args.workload, device, seed=rank)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            wl.launch(i, stream)
+    torch.cuda.synchronize()
+    barrier(dist, device)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local).start()
+    time.sleep(0.3)                       # let the sampler take its first reading
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    with torch.cuda.stream(stream):
+        t_begin.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            wl.launch(args.warmup + i, stream)
+            ends[i].record(stream)
+        t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    clocks = sampler.stop()
+
+    local_sec = t_begin.elapsed_time(t_end) / 1e3
+    kern_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    sec = max_over_ranks(dist, local_sec, device)
+    kern_ms = max_over_ranks(dist, kern_ms, device)
+    total_units = sum_over_ranks(dist, wl.counts["tokch"] * args.steps, device)
+
+    e2e = time_e2e(wl, args.e2e_steps, stream)
+    e2e_val = sum_over_ranks(dist, e2e["value"], device)
+
+    peaks = load_peaks()
+    kern_s = kern_ms / 1e3
+    gbs = wl.counts["bytes"] / kern_s / 1e9
+    if wl.kind == "scan":
+        peak_gexp = N_SM * MUFU_EX2_PER_CLK_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e9
+        achieved = wl.counts["exps"] / kern_s / 1e9
+        roof = dict(bound="alu", achieved=achieved, peak=peak_gexp, unit="Gexp/s",
+                    frac=achieved / peak_gexp,
+                    traffic=recorded_traffic(kernel_name(wl.kind), wl.name),
+                    kernel=kernel_name(wl.kind), kernel_ms=kern_ms,
+                    peak_basis="148 SMs x 16 ex2/clk/SM x %.0f MHz max SM clock" % peaks["sm_max_mhz"],
+                    hbm=dict(achieved_gbs=gbs, peak_gbs=peaks["hbm_gbs"], frac=gbs / peaks["hbm_gbs"],
+                             peak_source=peaks["source"]))
+    else:
+        roof = dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                    frac=gbs / peaks["hbm_gbs"],
+                    traffic=recorded_traffic(kernel_name(wl.kind), wl.name),
+                    kernel=kernel_name(wl.kind), kernel_ms=kern_ms,
+                    peak_basis="measured copy bandwidth, burst (%s)" % peaks["source"])
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_rate(args.workload, host_threads(), args.cpu_budget_s)
+
+    if rank == 0:
+        c = wl.cfg
+        config = dict(workload=wl.description(), batch=c["batch"], d_inner=c["dim"], dstate=c["dstate"],
+                      parallelism="replicas x%d" % world,
+                      l2=("%d rotating input sets of %.0f MB (%.0f MB touched per cycle) > 126 MB L2"
+                          % (wl.nsets, wl.counts["bytes"] / 1e6, wl.nsets * wl.counts["bytes"] / 1e6)))
+        if wl.kind == "scan":
+            config.update(seqlen=c["seqlen"], global_batch=c["batch"] * world)
+        line = dict(metric=METRIC, value=total_units / sec, unit=UNIT, n_gpus=world, steps=args.steps,
+                    warmup=args.warmup, ms_per_step=1e3 * sec / args.steps, higher_is_better=True,
+                    scaling="weak", vs_baseline=None, dtype="f32",
+                    io_dtype=str(c["dtype"]).split(".")[-1], data="synthetic", config=config,
+                    gb_per_s=gbs * world, roofline=roof, cpu_baseline=cpu,
+                    e2e=dict(value=e2e_val, unit=UNIT, h2d_bytes_per_step=e2e["h2d_bytes_per_step"],
+                             d2h_bytes_per_step=e2e["d2h_bytes_per_step"]),
+                    gpu_launches=args.steps, clocks=clocks, impl="ours")
+        print(json.dumps(line), flush=True)
+    barrier(dist, device)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

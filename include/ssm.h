@@ -1,0 +1,103 @@
+/*
+ * ssm.h -- C ABI of the B200 selective state-space scan library (libssm.so).
+ *
+ * Two operations:
+ *   ssm_selective_scan_fwd  the selective scan (S6) over a whole sequence;
+ *   ssm_state_step          one decode token on a carried state, updated in place.
+ *
+ * Both compute, per sequence b and channel d, with an N-wide fp32 state h:
+ *     Delta_t = softplus(delta[b,d,t] + delta_bias[d])   (bias and softplus optional)
+ *     h_n    <- exp(Delta_t * A[d,n]) * h_n + Delta_t * B[b,t,n] * x[b,d,t]
+ *     y[b,d,t] = (sum_n C[b,t,n] * h_n + D[d] * x[b,d,t]) * SiLU(z[b,d,t])
+ * Sources: zero-order-hold decay Abar = exp(Delta A) and its Euler input gain
+ * Bbar ~ Delta B ("Module 19: State-Space Models (Mamba)", learnllm, section "The Math:
+ * The State-Space Recurrence"); input-dependent Delta, B, C ("Beyond attention with
+ * Mamba, state space models and hybrids", xmarva lesson 10, section 3 "Selectivity");
+ * softplus step with bias, the skip D*x and then the SiLU(z) gate (same lesson,
+ * section 4 "The Mamba block"); the one-token update (section 7 "Generation with a
+ * state of fixed size").
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no memory and keeps no state between calls.
+ *  - Every pointer must be 16-byte aligned (SSM_ERR_ALIGNMENT otherwise).
+ *  - The call is asynchronous on `cuda_stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and never synchronises.  Argument errors are returned before
+ *    anything is launched; a launch failure returns SSM_ERR_CUDA.  Faults inside a
+ *    kernel surface, as usual for CUDA, at the caller's next synchronisation.
+ *  - dtype codes: SSM_F32 (fp32) or SSM_BF16 (bf16).  A, D, delta_bias and the state
+ *    are always fp32; the state arithmetic is fp32 whatever the input dtype.
+ *  - dstate (N) must be in 1..16 (SSM_ERR_UNSUPPORTED above 16).
+ */
+#ifndef SSM_H_
+#define SSM_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSM_F32 = 0,
+    SSM_BF16 = 1
+} ssm_dtype;
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1,   /* null required pointer, negative size, bad dtype code   */
+    SSM_ERR_UNSUPPORTED = 2,   /* dstate outside 1..16, sizes beyond the int32 index range */
+    SSM_ERR_ALIGNMENT = 3,     /* a pointer not 16-byte aligned                            */
+    SSM_ERR_CUDA = 4           /* the CUDA runtime reported an error at launch             */
+} ssm_status;
+
+/*
+ * Selective scan forward over whole sequences, starting from a zero state.
+ *
+ *   x, delta, z : [batch][dim][seqlen], in_dtype, contiguous ("channels first").
+ *                 delta is the raw step; z may be NULL (no gate).
+ *   delta_bias  : [dim] fp32, or NULL (no bias).  Added to delta before the softplus.
+ *   delta_softplus : nonzero -> Delta = softplus(delta + bias); zero -> Delta = delta + bias.
+ *   A           : [dim][dstate] fp32 (Mamba keeps it negative; any value is accepted).
+ *   B, C        : [batch][seqlen][dstate], in_dtype, shared by all channels of a sequence.
+ *   D           : [dim] fp32, or NULL (no skip term).
+ *   y           : [batch][dim][seqlen], out_dtype, written.
+ *   final_state : [batch][dim][dstate] fp32, or NULL; receives h after the last token
+ *                 (all zeros when seqlen == 0).
+ * Sizes: batch, dim, seqlen >= 0 (a zero size launches nothing except the zero final
+ * state); 1 <= dstate <= 16; batch*dim*seqlen and batch*seqlen*dstate must be below 2^62
+ * and seqlen below 2^31.
+ * The N-wide state never leaves the chip: only y and final_state are written.
+ */
+int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_bias,
+                           int delta_softplus, const float *A, const void *B, const void *C,
+                           const float *D, const void *z, void *y, float *final_state,
+                           int batch, int dim, int seqlen, int dstate,
+                           int in_dtype, int out_dtype, void *cuda_stream);
+
+/*
+ * One decode step: every (b, d) channel takes one token and its state is updated in place.
+ *
+ *   state       : [batch][dim][dstate] fp32, read and overwritten.
+ *   x, delta, z : [batch][dim], in_dtype.  delta is the final step Delta (already
+ *                 positive: no bias, no softplus is applied here).  z may be NULL.
+ *   A           : [dim][dstate] fp32.   D: [dim] fp32 or NULL.
+ *   B, C        : [batch][dstate], in_dtype.
+ *   y           : [batch][dim], out_dtype, written.
+ * Chaining L calls from a state h0 gives the same y and state as the scan over those L
+ * tokens started from h0.
+ */
+int ssm_state_step(float *state, const void *x, const void *delta, const float *A,
+                   const void *B, const void *C, const float *D, const void *z, void *y,
+                   int batch, int dim, int dstate, int in_dtype, int out_dtype,
+                   void *cuda_stream);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char *ssm_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int ssm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_H_ */

@@ -1,0 +1,22 @@
+"""B200 (sm_100a) selective state-space scan (S6): forward scan and decode step.
+
+The computation lives in ``libssm.so`` (C ABI in ``include/ssm.h``); this package only
+loads it and marshals torch tensors into it.
+"""
+from ._lib import (  # noqa: F401
+    LIB_PATH,
+    SSM_BF16,
+    SSM_ERR_ALIGNMENT,
+    SSM_ERR_CUDA,
+    SSM_ERR_INVALID_ARG,
+    SSM_ERR_UNSUPPORTED,
+    SSM_F32,
+    SSM_OK,
+    SsmError,
+    load_library,
+    selective_scan,
+    ssm_selective_scan_fwd,
+    ssm_state_step,
+    ssm_status_string,
+    ssm_version,
+)

@@ -1,0 +1,121 @@
+"""ctypes binding of libssm.so (include/ssm.h): argument marshalling only.
+
+Every step of the computation runs in the CUDA kernels behind the C ABI.  There is no
+fallback: if the library is missing or was built for another architecture the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm.so")
+
+SSM_F32, SSM_BF16 = 0, 1
+SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_ALIGNMENT, SSM_ERR_CUDA = range(5)
+
+_DTYPE_CODE = {torch.float32: SSM_F32, torch.bfloat16: SSM_BF16}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class SsmError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__("%s (status %d)" % (msg, status))
+        self.status = status
+
+
+def load_library(path: str | None = None):
+    """Load libssm.so once (raises if it is absent: build it with
+    ``python -m selective_state_space_45_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError("libssm.so not found at %s; build it first "
+                               "(python -m selective_state_space_45_b200.build)" % p)
+        lib = ctypes.CDLL(p)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        lib.ssm_selective_scan_fwd.restype = i
+        lib.ssm_selective_scan_fwd.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp,
+                                               i, i, i, i, i, i, vp]
+        lib.ssm_state_step.restype = i
+        lib.ssm_state_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+        lib.ssm_status_string.restype = ctypes.c_char_p
+        lib.ssm_status_string.argtypes = [i]
+        lib.ssm_version.restype = i
+        lib.ssm_version.argtypes = []
+        _lib = lib
+        return lib
+
+
+def ssm_status_string(status: int) -> str:
+    return load_library().ssm_status_string(int(status)).decode()
+
+
+def ssm_version() -> int:
+    return int(load_library().ssm_version())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libssm must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream, *tensors):
+    if stream is None:
+        dev = next((t.device for t in tensors if isinstance(t, torch.Tensor) and t.is_cuda), None)
+        if dev is None:
+            return None
+        return torch.cuda.current_stream(dev).cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status):
+    if status != SSM_OK:
+        raise SsmError(status, ssm_status_string(status))
+
+
+def ssm_selective_scan_fwd(x, delta, delta_bias, delta_softplus, A, B, C, D, z, y, final_state,
+                           stream=None):
+    """Selective scan forward (see include/ssm.h).  Tensors are CUDA tensors in the
+    layouts of the header: x, delta, z, y [batch, dim, L]; B, C [batch, L, N]; A [dim, N];
+    D, delta_bias [dim]; final_state [batch, dim, N].  Writes y and final_state in place."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    _check(load_library().ssm_selective_scan_fwd(
+        _ptr(x), _ptr(delta), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(A), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), _ptr(y), _ptr(final_state), batch, dim, L, N,
+        _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, x, y)))
+
+
+def ssm_state_step(state, x, delta, A, B, C, D, z, y, stream=None):
+    """One decode step (see include/ssm.h): state [batch, dim, N] fp32 updated in place;
+    x, delta, z, y [batch, dim]; B, C [batch, N]."""
+    batch, dim, N = state.shape
+    _check(load_library().ssm_state_step(
+        _ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(y),
+        batch, dim, N, _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, state, y)))
+
+
+def selective_scan(x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
+                   out_dtype=None, return_final_state=True, stream=None):
+    """Allocate y (and the final state) with torch and run ``ssm_selective_scan_fwd``."""
+    batch, dim, L = x.shape
+    y = torch.empty((batch, dim, L), device=x.device, dtype=out_dtype or x.dtype)
+    fs = (torch.empty((batch, dim, A.shape[1]), device=x.device, dtype=torch.float32)
+          if return_final_state else None)
+    ssm_selective_scan_fwd(x, delta, delta_bias, delta_softplus, A, B, C, D, z, y, fs, stream)
+    return (y, fs) if return_final_state else y

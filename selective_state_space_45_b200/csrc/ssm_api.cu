@@ -1,0 +1,179 @@
+// ssm_api.cu -- the C ABI of libssm.so: argument checks, kernel choice, launch.
+//
+// Every entry point checks its arguments on the host before touching the GPU; a
+// rejected call launches nothing.  Kernels run on the caller's stream, asynchronously.
+#include <climits>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include "../../include/ssm.h"
+#include "scan_fwd.cuh"
+#include "state_step.cuh"
+
+namespace {
+
+constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(int t) { return t == SSM_F32 || t == SSM_BF16; }
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA; }
+
+// Time sub-chunks per tile: 1 keeps each channel's scan in one warp; 4 splits every
+// tile over four warps and stitches them, which fills the GPU when there are few
+// channels (long single sequences).  SSM_SCAN_SPLIT=1|4 forces one for measurement.
+int choose_split(long long channels) {
+    if (const char *e = std::getenv("SSM_SCAN_SPLIT")) {
+        const int v = std::atoi(e);
+        if (v == 1 || v == 4) return v;
+    }
+    return channels >= 8192 ? 1 : 4;
+}
+
+template <class Cfg>
+int launch_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
+    ssm::ScanArgs a = a0;
+    const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
+    const long long blocks = groups * (long long)a.batch;
+    if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    a.groups_per_seq = int(groups);
+    const size_t smem = Cfg::SMEM_BYTES;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return SSM_ERR_CUDA;
+    }
+    ssm::scan_fwd_kernel<Cfg><<<unsigned(blocks), Cfg::NTHREADS, smem, stream>>>(a);
+    return status_of(cudaGetLastError());
+}
+
+// NP (padded states) x split -> tile shape.  K = 1: one warp per channel group, 32-token
+// tiles, 4 channel groups per CTA.  K = 4: four 8-token sub-chunks per 32-token tile,
+// 2 channel groups per CTA.
+template <int NP, typename Tin, typename Tout, bool VEC>
+int dispatch_split(const ssm::ScanArgs &a, int split, cudaStream_t s) {
+    constexpr int CG1 = (NP == 16) ? 4 : (NP == 8 ? 2 : 1);
+    constexpr int CG4 = (NP == 16) ? 2 : 1;
+    if (split == 1) return launch_scan<ssm::ScanCfg<NP, 1, 32, CG1, 3, Tin, Tout, VEC>>(a, s);
+    return launch_scan<ssm::ScanCfg<NP, 4, 8, CG4, 3, Tin, Tout, VEC>>(a, s);
+}
+
+template <typename Tin, typename Tout>
+int dispatch_np(const ssm::ScanArgs &a, int split, bool vec, cudaStream_t s) {
+    const int N = a.dstate;
+    if (N <= 4)
+        return vec ? dispatch_split<4, Tin, Tout, true>(a, split, s)
+                   : dispatch_split<4, Tin, Tout, false>(a, split, s);
+    if (N <= 8)
+        return vec ? dispatch_split<8, Tin, Tout, true>(a, split, s)
+                   : dispatch_split<8, Tin, Tout, false>(a, split, s);
+    return vec ? dispatch_split<16, Tin, Tout, true>(a, split, s)
+               : dispatch_split<16, Tin, Tout, false>(a, split, s);
+}
+
+template <int NP, typename Tin, typename Tout>
+int launch_step_np(const ssm::StepArgs &a, cudaStream_t s) {
+    constexpr int G = NP / 4;
+    const long long threads = (long long)a.batch * a.dim * G;
+    const long long blocks = (threads + 255) / 256;
+    if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    if (a.dstate % 4 == 0)
+        ssm::state_step_kernel<NP, Tin, Tout, true><<<unsigned(blocks), 256, 0, s>>>(a);
+    else
+        ssm::state_step_kernel<NP, Tin, Tout, false><<<unsigned(blocks), 256, 0, s>>>(a);
+    return status_of(cudaGetLastError());
+}
+
+template <typename Tin, typename Tout>
+int launch_step(const ssm::StepArgs &a, cudaStream_t s) {
+    if (a.dstate <= 4) return launch_step_np<4, Tin, Tout>(a, s);
+    if (a.dstate <= 8) return launch_step_np<8, Tin, Tout>(a, s);
+    return launch_step_np<16, Tin, Tout>(a, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_version(void) { return kVersion; }
+
+const char *ssm_status_string(int status) {
+    switch (status) {
+    case SSM_OK: return "ok";
+    case SSM_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or bad dtype)";
+    case SSM_ERR_UNSUPPORTED: return "unsupported size (dstate must be 1..16; grid too large)";
+    case SSM_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case SSM_ERR_CUDA: return "CUDA runtime error at launch";
+    default: return "unknown status";
+    }
+}
+
+int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_bias,
+                           int delta_softplus, const float *A, const void *B, const void *C,
+                           const float *D, const void *z, void *y, float *final_state,
+                           int batch, int dim, int seqlen, int dstate,
+                           int in_dtype, int out_dtype, void *cuda_stream) {
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return SSM_ERR_INVALID_ARG;
+    if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1) return SSM_ERR_INVALID_ARG;
+    if (dstate > 16) return SSM_ERR_UNSUPPORTED;
+    const long long channels = (long long)batch * dim;
+    const bool work = channels > 0 && seqlen > 0;
+    if (work && (!x || !delta || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, delta, delta_bias, A, B, C, D, z, y, final_state};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSM_ERR_ALIGNMENT;
+    if (channels == 0) return SSM_OK;
+    if (!work && !final_state) return SSM_OK;
+
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (!work)   // empty sequences: the final state is the zero start state
+        return status_of(cudaMemsetAsync(final_state, 0, size_t(channels) * dstate * sizeof(float), stream));
+
+    ssm::ScanArgs a{};
+    a.x = x; a.delta = delta; a.delta_bias = delta_bias; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.z = z; a.y = y; a.final_state = final_state;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = dstate;
+    a.softplus = delta_softplus ? 1 : 0;
+
+    // 16-byte staging needs every row of x/delta/z/y and every sequence's B/C block to
+    // start on a 16-byte boundary: seqlen a multiple of the 16-byte element count.
+    const int ein = in_dtype == SSM_F32 ? 4 : 8;
+    const int eout = out_dtype == SSM_F32 ? 4 : 8;
+    const bool vec = (seqlen % ein == 0) && (seqlen % eout == 0);
+    const int split = choose_split(channels);
+
+    if (in_dtype == SSM_F32 && out_dtype == SSM_F32) return dispatch_np<float, float>(a, split, vec, stream);
+    if (in_dtype == SSM_BF16 && out_dtype == SSM_BF16)
+        return dispatch_np<__nv_bfloat16, __nv_bfloat16>(a, split, vec, stream);
+    if (in_dtype == SSM_BF16) return dispatch_np<__nv_bfloat16, float>(a, split, vec, stream);
+    return dispatch_np<float, __nv_bfloat16>(a, split, vec, stream);
+}
+
+int ssm_state_step(float *state, const void *x, const void *delta, const float *A,
+                   const void *B, const void *C, const float *D, const void *z, void *y,
+                   int batch, int dim, int dstate, int in_dtype, int out_dtype,
+                   void *cuda_stream) {
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return SSM_ERR_INVALID_ARG;
+    if (batch < 0 || dim < 0 || dstate < 1) return SSM_ERR_INVALID_ARG;
+    if (dstate > 16) return SSM_ERR_UNSUPPORTED;
+    const long long channels = (long long)batch * dim;
+    if (channels > 0 && (!state || !x || !delta || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {state, x, delta, A, B, C, D, z, y};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSM_ERR_ALIGNMENT;
+    if (channels == 0) return SSM_OK;
+
+    ssm::StepArgs a{};
+    a.state = state; a.x = x; a.delta = delta; a.A = A; a.B = B; a.C = C; a.D = D; a.z = z;
+    a.y = y; a.batch = batch; a.dim = dim; a.dstate = dstate;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (in_dtype == SSM_F32 && out_dtype == SSM_F32) return launch_step<float, float>(a, stream);
+    if (in_dtype == SSM_BF16 && out_dtype == SSM_BF16)
+        return launch_step<__nv_bfloat16, __nv_bfloat16>(a, stream);
+    if (in_dtype == SSM_BF16) return launch_step<__nv_bfloat16, float>(a, stream);
+    return launch_step<float, __nv_bfloat16>(a, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI: the library loads, exports what include/ssm.h declares,
+and rejects bad arguments before touching the GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import selective_state_space_45_b200 as ssm
+from selective_state_space_45_b200 import build as ssm_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm.h")
+
+# fake, 16-byte aligned "device" addresses: validation returns before any is dereferenced
+P = 0x7F0000001000
+MIS = 0x7F0000001004
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssm_build.build()
+    return ssm.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w \*]*?\b(ssm_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for expected in ("ssm_selective_scan_fwd", "ssm_state_step", "ssm_status_string", "ssm_version"):
+        assert expected in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert getattr(lib, name) is not None
+
+
+def test_status_strings_and_version(lib):
+    assert ssm.ssm_status_string(ssm.SSM_OK) == "ok"
+    for code in range(1, 5):
+        s = ssm.ssm_status_string(code)
+        assert s and s != "unknown status"
+    assert ssm.ssm_status_string(99) == "unknown status"
+    assert ssm.ssm_version() >= 10000
+
+
+def scan(lib, **kw):
+    args = dict(x=P, delta=P, bias=None, sp=1, A=P, B=P, C=P, D=P, z=P, y=P, fs=P,
+                batch=2, dim=3, L=8, N=16, din=ssm.SSM_BF16, dout=ssm.SSM_BF16)
+    args.update(kw)
+    return lib.ssm_selective_scan_fwd(args["x"], args["delta"], args["bias"], args["sp"], args["A"],
+                                      args["B"], args["C"], args["D"], args["z"], args["y"],
+                                      args["fs"], args["batch"], args["dim"], args["L"], args["N"],
+                                      args["din"], args["dout"], None)
+
+
+def step(lib, **kw):
+    args = dict(state=P, x=P, delta=P, A=P, B=P, C=P, D=P, z=P, y=P, batch=2, dim=3, N=16,
+                din=ssm.SSM_BF16, dout=ssm.SSM_BF16)
+    args.update(kw)
+    return lib.ssm_state_step(args["state"], args["x"], args["delta"], args["A"], args["B"], args["C"],
+                              args["D"], args["z"], args["y"], args["batch"], args["dim"], args["N"],
+                              args["din"], args["dout"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(delta=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(A=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(B=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(C=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(y=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(batch=-1), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dim=-5), ssm.SSM_ERR_INVALID_ARG),
+    (dict(L=-1), ssm.SSM_ERR_INVALID_ARG),
+    (dict(N=0), ssm.SSM_ERR_INVALID_ARG),
+    (dict(N=17), ssm.SSM_ERR_UNSUPPORTED),
+    (dict(N=64), ssm.SSM_ERR_UNSUPPORTED),
+    (dict(din=2), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dout=-1), ssm.SSM_ERR_INVALID_ARG),
+    (dict(x=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(B=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(y=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(fs=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(bias=MIS), ssm.SSM_ERR_ALIGNMENT),
+    # nothing to do: accepted without a launch, optional pointers may be absent
+    (dict(batch=0), ssm.SSM_OK),
+    (dict(dim=0, x=None, y=None), ssm.SSM_OK),
+    (dict(L=0, fs=None), ssm.SSM_OK),
+])
+def test_scan_argument_checks(lib, kw, status):
+    assert scan(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(state=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(x=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(delta=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(y=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(batch=-2), ssm.SSM_ERR_INVALID_ARG),
+    (dict(N=0), ssm.SSM_ERR_INVALID_ARG),
+    (dict(N=17), ssm.SSM_ERR_UNSUPPORTED),
+    (dict(din=7), ssm.SSM_ERR_INVALID_ARG),
+    (dict(state=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(A=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(batch=0), ssm.SSM_OK),
+])
+def test_step_argument_checks(lib, kw, status):
+    assert step(lib, **kw) == status
+
+
+def test_python_binding_raises_on_error(lib):
+    with pytest.raises(ssm.SsmError) as e:
+        ssm._lib._check(ssm.SSM_ERR_UNSUPPORTED)
+    assert e.value.status == ssm.SSM_ERR_UNSUPPORTED
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises((RuntimeError, OSError)):
+        ctypes_path = str(tmp_path / "nope.so")
+        saved = ssm._lib._lib
+        ssm._lib._lib = None
+        try:
+            ssm.load_library(ctypes_path)
+        finally:
+            ssm._lib._lib = saved

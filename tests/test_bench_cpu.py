@@ -1,0 +1,94 @@
+"""bench.py host logic on CPU: multi-rank timing reduction over 2 gloo ranks, the
+algorithmic byte / work counts, and the CPU-baseline leg."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w, local = bench.dist_env()
+    dist = bench.init_dist(w, "gloo", timeout_s=30)
+    bench.barrier(dist)
+    # rank 1 is the slow rank; the job time is the slowest rank's
+    mx = bench.max_over_ranks(dist, 1.5 + r)
+    total = bench.sum_over_ranks(dist, 1000 * (r + 1))
+    bench.barrier(dist)
+    dist.destroy_process_group()
+    out.put((r, w, local, mx, total))
+
+
+def test_two_gloo_ranks_reduce_time_and_work():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [x[0] for x in res] == [0, 1]
+    for r, w, local, mx, total in res:
+        assert w == 2 and local == r
+        assert mx == 2.5            # max over ranks
+        assert total == 3000.0      # work of all ranks
+
+
+def test_single_rank_reductions_are_identity():
+    assert bench.max_over_ranks(None, 3.25) == 3.25
+    assert bench.sum_over_ranks(None, 7.0) == 7.0
+
+
+def test_scan_counts_mamba130m():
+    c = bench.scan_counts(8, 1536, 2048, 16, 2, 2)
+    assert c["tokch"] == 8 * 2048 * 1536
+    assert c["exps"] == 8 * 2048 * 1536 * 16
+    # x, delta, z in and y out (2 B each) + B, C + A, D, bias + final state
+    expect = 8 * 1536 * 2048 * 8 + 2 * 8 * 2048 * 16 * 2 + 1536 * 16 * 4 + 2 * 1536 * 4 + 8 * 1536 * 16 * 4
+    assert c["bytes"] == expect
+    assert abs(c["bytes"] / 1e6 - 203.2) < 0.1
+
+
+def test_step_counts_decode():
+    c = bench.step_counts(256, 5120, 16, 2, 2)
+    assert c["tokch"] == 256 * 5120
+    assert abs(c["bytes"] / 1e6 - 178.6) < 0.5
+
+
+def test_oracle_rate_is_bounded_and_reports_cores():
+    r = bench.oracle_rate("tiny", threads=2, budget_s=0.2)
+    assert r["kind"] == "oracle" and r["cores"] == 2 and r["value"] > 0
+    assert r["seconds"] < 5.0
+
+
+def test_reference_arm_prints_one_line(capsys):
+    rc = bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"])
+    assert rc == 0
+    import json
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["unit"] == bench.UNIT and d["higher_is_better"] is True
+
+
+@pytest.mark.parametrize("world", [1])
+def test_dist_env_defaults(world, monkeypatch):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.dist_env() == (0, 1, 0)
