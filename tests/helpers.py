@@ -1,7 +1,9 @@
 """Shared test helpers: tolerances of the parity bar and channel sampling.
 
 Tolerances (one reading of the parity bar, applied per output tensor):
-  * fp32 inputs:  normwise relative error  max|gpu - ref| / max|ref|  <= 1e-4.
+  * fp32 inputs:  normwise relative error  max|gpu - ref| / max|ref|  <= 1e-4; when the
+    output is written as bf16, each element may also carry its bf16 rounding
+    (at most 2^-8 of its magnitude): |gpu - ref| <= 1e-4 max|ref| + 2^-8 |ref|.
   * bf16 inputs, fp32 state:  relative L2 error <= 5e-3, and max-abs <= 2e-2 on every
     fp32 output (final state; y when it is written in fp32).  A bf16 y is rounded to
     bf16 on the way out, so there the max-abs bound is applied as |gpu - ref| <=
@@ -14,6 +16,7 @@ FP32_REL = 1e-4
 BF16_MAXABS = 2e-2
 BF16_RELL2 = 5e-3
 BF16_ULP = 2.0 ** -7
+BF16_HALF_ULP = 2.0 ** -8
 
 
 def to64(t):
@@ -33,7 +36,11 @@ def assert_parity(gpu, ref, in_dtype, out_dtype=None, what="y"):
     stats = dict(max_abs=float(err.max()), norm_rel=float(err.max()) / scale,
                  rel_l2=float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)))
     if in_dtype == torch.float32:
-        assert stats["norm_rel"] <= FP32_REL, (what, stats)
+        if out_dtype == torch.bfloat16:
+            bad = err > FP32_REL * scale + BF16_HALF_ULP * np.abs(r)
+            assert not bad.any(), (what, stats, int(bad.sum()))
+        else:
+            assert stats["norm_rel"] <= FP32_REL, (what, stats)
     else:
         assert stats["rel_l2"] <= BF16_RELL2, (what, stats)
         if out_dtype == torch.bfloat16:
