@@ -9,6 +9,8 @@ namespace ssm {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+__device__ __forceinline__ int tid_x() { return static_cast<int>(threadIdx.x); }
+
 // Hardware base-2 exponential (the SFU's ex2), flush-to-zero.  Used for the per-(t, n)
 // decay exp(Delta * a) = 2^(Delta * a * log2 e), with a * log2 e folded in once per state.
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -24,9 +26,25 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
-// softplus(v) = log(1 + e^v), in the overflow-free form max(v, 0) + log1p(e^-|v|).
+// log1p(u) for u in [0, 1], as u * p(u) with p a degree-7 polynomial fitted to log1p(u)/u
+// (least squares at Chebyshev nodes, relative weighting).  Evaluated in fp32 Horner form
+// its relative error is below 3.3e-7 on the whole interval.
+__device__ __forceinline__ float log1p_unit(float u) {
+    float p = -0.008336497470736504f;
+    p = fmaf(p, u, 0.04337085038423538f);
+    p = fmaf(p, u, -0.10667790472507477f);
+    p = fmaf(p, u, 0.1767549365758896f);
+    p = fmaf(p, u, -0.2447046935558319f);
+    p = fmaf(p, u, 0.3327118754386902f);
+    p = fmaf(p, u, -0.49997127056121826f);
+    p = fmaf(p, u, 0.9999997615814209f);
+    return u * p;
+}
+
+// softplus(v) = log(1 + e^v), in the overflow-free form max(v, 0) + log1p(e^-|v|):
+// one SFU exponential, the logarithm on the FMA pipe.
 __device__ __forceinline__ float softplus_f(float v) {
-    return fmaxf(v, 0.f) + log1pf(ex2_approx(-fabsf(v) * kLog2e));
+    return fmaxf(v, 0.f) + log1p_unit(ex2_approx(-fabsf(v) * kLog2e));
 }
 
 // SiLU(z) = z * sigmoid(z) = z / (1 + e^-z).

@@ -48,7 +48,8 @@ struct ScanArgs {
     int groups_per_seq;  // ceil(dim / CH)
 };
 
-template <int NP_, int K_, int TS_, int CG_, int NSTAGE_, typename Tin_, typename Tout_, bool VEC_>
+template <int NP_, int K_, int TS_, int CG_, int NSTAGE_, typename Tin_, typename Tout_, bool VEC_,
+          int MINB_ = 1>
 struct ScanCfg {
     using Tin = Tin_;
     using Tout = Tout_;
@@ -58,6 +59,7 @@ struct ScanCfg {
     static constexpr int CG = CG_;            // channel groups (of CPW channels) per CTA
     static constexpr int NSTAGE = NSTAGE_;    // cp.async ring depth (tiles)
     static constexpr bool VEC = VEC_;
+    static constexpr int MINB = MINB_;        // resident CTAs per SM the register budget targets
     static constexpr int G = NP / 4;          // lanes per channel
     static constexpr int CPW = 32 / G;        // channels per warp
     static constexpr int CH = CG * CPW;       // channels per CTA
@@ -70,6 +72,7 @@ struct ScanCfg {
     static constexpr int Y_ROW = T + EOUT;          // spread channels over banks
     static constexpr int PREP_ROW = T + 1;          // float2 elements
     static_assert(TS % G == 0, "sub-chunk must be a multiple of the lane group");
+    static_assert(K > 1 || TS % 4 == 0, "the register-carried scan works in 4-token blocks");
     static_assert((T * sizeof(Tin)) % 16 == 0 && (T * sizeof(Tout)) % 16 == 0, "tile rows");
 
     // shared-memory layout (byte offsets, 16-byte aligned pieces)
@@ -168,7 +171,7 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(Cfg::NTHREADS)
+__global__ void __launch_bounds__(Cfg::NTHREADS, Cfg::MINB)
 scan_fwd_kernel(const ScanArgs p) {
     using Tin = typename Cfg::Tin;
     using Tout = typename Cfg::Tout;
@@ -259,24 +262,60 @@ scan_fwd_kernel(const ScanArgs p) {
         __syncthreads();
 
         // ---- scan of this warp's sub-chunk ----
-        float yp[TS];
+        // yout[m]: the channel's full readout for token j*TS + m*G + r, once summed
+        // over the G lanes of the channel.
+        float yout[TS / G];
         const float2 *prow = prep + c * Cfg::PREP_ROW + j * TS;
         if constexpr (K == 1) {
+            // Blocks of 4 tokens.  The decays exp(Delta*a) and writes Delta*x*B of the
+            // NEXT block are computed before the recurrence of the current one, so the
+            // 16 independent SFU operations of a block overlap the short FFMA chain.
+            constexpr int TB = 4;
+            constexpr int NB = TS / TB;
+            float ac[TB][4], wc[TB][4];
+            auto decay_write = [&](int i0, float (&a)[TB][4], float (&w)[TB][4]) {
 #pragma unroll
-            for (int i = 0; i < TS; ++i) {
-                const float2 dd = prow[i];
-                const float4 bq = *reinterpret_cast<const float4 *>(Bf + i * NP + 4 * r);
-                const float4 cq = *reinterpret_cast<const float4 *>(Cf + i * NP + 4 * r);
-                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-                const float cc4[4] = {cq.x, cq.y, cq.z, cq.w};
-                float acc = 0.f;
+                for (int u = 0; u < TB; ++u) {
+                    const float2 dd = prow[i0 + u];
+                    const float4 bq = *reinterpret_cast<const float4 *>(Bf + (i0 + u) * NP + 4 * r);
+                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const float a = ex2_approx(dd.x * A2[s]);
-                    h[s] = fmaf(a, h[s], dd.y * bb[s]);
-                    acc = fmaf(cc4[s], h[s], acc);
+                    for (int s = 0; s < 4; ++s) {
+                        a[u][s] = ex2_approx(dd.x * A2[s]);
+                        w[u][s] = dd.y * bb[s];
+                    }
                 }
-                yp[i] = acc;
+            };
+            decay_write(0, ac, wc);
+#pragma unroll
+            for (int blk = 0; blk < NB; ++blk) {
+                float an[TB][4], wn[TB][4];
+                if (blk + 1 < NB) decay_write((blk + 1) * TB, an, wn);
+                float yp[TB];
+#pragma unroll
+                for (int u = 0; u < TB; ++u) {
+                    const float4 cq = *reinterpret_cast<const float4 *>(Cf + (blk * TB + u) * NP + 4 * r);
+                    const float cc4[4] = {cq.x, cq.y, cq.z, cq.w};
+                    float acc = 0.f;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        h[s] = fmaf(ac[u][s], h[s], wc[u][s]);
+                        acc = fmaf(cc4[s], h[s], acc);
+                    }
+                    yp[u] = acc;
+                }
+#pragma unroll
+                for (int g = 0; g < TB / G; ++g)
+                    yout[blk * (TB / G) + g] = GroupReduceScatter<G>::run(yp + g * G, r);
+                if (blk + 1 < NB) {
+#pragma unroll
+                    for (int u = 0; u < TB; ++u)
+#pragma unroll
+                        for (int s = 0; s < 4; ++s) {
+                            ac[u][s] = an[u][s];
+                            wc[u][s] = wn[u][s];
+                        }
+                }
             }
         } else {
             float hl[TS][4], Pl[TS][4];
@@ -322,6 +361,7 @@ scan_fwd_kernel(const ScanArgs p) {
                     make_float4(h[0], h[1], h[2], h[3]);
             }
             cur ^= 1;
+            float yp[TS];
 #pragma unroll
             for (int i = 0; i < TS; ++i) {
                 const int tt = j * TS + i;
@@ -332,12 +372,14 @@ scan_fwd_kernel(const ScanArgs p) {
                 for (int s = 0; s < 4; ++s) acc = fmaf(cc4[s], fmaf(Pl[i][s], hin[s], hl[i][s]), acc);
                 yp[i] = acc;
             }
+#pragma unroll
+            for (int m = 0; m < TS / G; ++m) yout[m] = GroupReduceScatter<G>::run(yp + m * G, r);
         }
 
-        // ---- sum over the channel's lanes, skip, gate; stage y ----
+        // ---- skip, gate; stage y ----
 #pragma unroll
         for (int m = 0; m < TS / G; ++m) {
-            const float ysum = GroupReduceScatter<G>::run(yp + m * G, r);
+            const float ysum = yout[m];
             const int tt = j * TS + m * G + r;
             const float xv = to_f32(sv.xs[c * Cfg::RAW_ROW + tt]);
             float yv = fmaf(Dd, xv, ysum);

@@ -1,0 +1,432 @@
+// scan_lanes.cuh -- selective scan forward, one channel per lane (many-channel inputs).
+//
+// Same computation as scan_fwd.cuh (sources there): per sequence b, channel d, state n,
+//   Delta = softplus(delta + bias[d]), h_n <- exp(Delta*A[d,n]) h_n + Delta*B[b,t,n]*x,
+//   y = (sum_n C[b,t,n] h_n + D[d] x) * SiLU(z),
+// with the state carried in registers from the first token to the last.
+//
+// Layout of the work
+//   * A CTA owns CH = 32*CG channels of one sequence and walks L in T-token tiles.
+//   * Warp (cg, q) holds states 4q..4q+3 of the 32 channels of channel group cg, one
+//     channel per lane.  B_t and C_t of a state quad are the same for every lane, so
+//     each is one broadcast shared-memory load per token; the state quads of a channel
+//     live in different warps and their readouts are summed once per (t, d) after the
+//     tile, through a shared buffer, instead of by shuffles inside the recurrence.
+//   * The softplus step and Delta*x (prep) and the skip, gate and output conversion
+//     (epilogue) are computed once per (t, d) by "chunk tasks" of 8 tokens of one
+//     channel, with 16-byte shared accesses laid out to be free of bank conflicts.
+//   * x, delta, z, B, C are staged through a cp.async ring of NSTAGE tiles (16-byte
+//     copies) when every row is 16-byte aligned; otherwise by guarded scalar loads.
+#pragma once
+
+#include "common.cuh"
+#include "scan_fwd.cuh"   // ScanArgs
+
+namespace ssm {
+
+template <int NP_, int CG_, int T_, int NSTAGE_, typename Tin_, typename Tout_, bool VEC_, int MINB_,
+          bool PIPE_ = false>
+struct LaneCfg {
+    using Tin = Tin_;
+    using Tout = Tout_;
+    static constexpr int NP = NP_;          // padded state width (multiple of 4)
+    static constexpr int Q = NP / 4;        // state quads = warps per channel group
+    static constexpr int CG = CG_;          // channel groups of 32 per CTA
+    static constexpr int CH = 32 * CG;      // channels per CTA
+    static constexpr int T = T_;            // tokens per tile
+    static constexpr int NSTAGE = NSTAGE_;
+    static constexpr bool VEC = VEC_;
+    static constexpr int MINB = MINB_;
+    static constexpr bool PIPE = PIPE_;     // decays of the next 4 tokens before the current recurrence
+    static constexpr int NWARP = Q * CG;
+    static constexpr int NTHREADS = 32 * NWARP;
+    static constexpr int EIN = 16 / sizeof(Tin);
+    static constexpr int EOUT = 16 / sizeof(Tout);
+    static constexpr int T8 = T / 8;                  // 8-token chunks per tile row
+    static constexpr int NTASK = CH * T8;             // chunk tasks per tile
+    static constexpr int TASKS_PER_THREAD = (NTASK + NTHREADS - 1) / NTHREADS;
+    static constexpr int RAW_ROW = T + EIN;           // row stride 16 B past a multiple of
+    static constexpr int Y_ROW = T + EOUT;            // 16 B: conflict-free 16 B column reads
+    static constexpr int YP_ROW = T + 4;              // floats; 36 words for T = 32
+    static_assert(T % 8 == 0 && T % 4 == 0, "tile must hold whole 8-token chunks");
+    static_assert(NTASK % NTHREADS == 0, "chunk tasks must divide evenly");
+
+    static constexpr size_t al(size_t v) { return (v + 15) & ~size_t(15); }
+    static constexpr size_t RAW_ARR = al(size_t(CH) * RAW_ROW * sizeof(Tin));
+    static constexpr size_t RAW_BC = al(size_t(T) * NP * sizeof(Tin));
+    static constexpr size_t STAGE_BYTES = 3 * RAW_ARR + 2 * RAW_BC;
+    static constexpr size_t OFF_RAW = 0;
+    // prep: float4 [T/2][CH] = (Delta_t, Delta_t x_t, Delta_t+1, Delta_t+1 x_t+1)
+    static constexpr size_t OFF_PREP = OFF_RAW + NSTAGE * STAGE_BYTES;
+    static constexpr size_t OFF_BF = OFF_PREP + al(size_t(T / 2) * CH * sizeof(float4));
+    static constexpr size_t OFF_CF = OFF_BF + al(size_t(T) * NP * sizeof(float));
+    static constexpr size_t OFF_YP = OFF_CF + al(size_t(T) * NP * sizeof(float));
+    static constexpr size_t OFF_Y = OFF_YP + al(size_t(Q) * CH * YP_ROW * sizeof(float));
+    static constexpr size_t OFF_BIAS = OFF_Y + al(size_t(CH) * Y_ROW * sizeof(Tout));
+    static constexpr size_t SMEM_BYTES = OFF_BIAS + al(size_t(CH) * sizeof(float));
+};
+
+// 8 consecutive values of a staged row as fp32 (the row start is 16-byte aligned).
+template <typename T> __device__ __forceinline__ void load8(const T *src, float (&v)[8]);
+template <> __device__ __forceinline__ void load8<float>(const float *src, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(src);
+    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <> __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *src, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(src);
+    const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {            // bf16 -> fp32 is a 16-bit left shift
+        v[2 * k] = __uint_as_float(w[k] << 16);
+        v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+}
+
+// 8 fp32 values stored as 8 values of T (16-byte aligned destination).
+template <typename T> __device__ __forceinline__ void store8(T *dst, const float (&v)[8]);
+template <> __device__ __forceinline__ void store8<float>(float *dst, const float (&v)[8]) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <> __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16 *dst, const float (&v)[8]) {
+    unsigned w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<const unsigned *>(&p);
+    }
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Stage tile [t0, t0 + T) of x, delta, z (rows of nch channels) and of B, C into ring stage
+// st, with every index split by compile-time divisors.  VEC: 16-byte cp.async chunks, each
+// wholly inside or wholly outside [0, L) because L is a multiple of the chunk width.
+template <class Cfg>
+__device__ __forceinline__ void load_tile_lanes(const ScanArgs &p, unsigned char *smem, int st, int t0,
+                                                size_t row0, size_t bc0, int nch) {
+    using Tin = typename Cfg::Tin;
+    constexpr int CH = Cfg::CH, T = Cfg::T, NT = Cfg::NTHREADS, EIN = Cfg::EIN, NP = Cfg::NP;
+    Stage<Cfg> s(smem, st);
+    const int L = p.seqlen, N = p.dstate;
+    const Tin *gx = static_cast<const Tin *>(p.x) + row0;
+    const Tin *gd = static_cast<const Tin *>(p.delta) + row0;
+    const Tin *gz = p.z ? static_cast<const Tin *>(p.z) + row0 : gx;
+    const int narr = p.z ? 3 : 2;
+    const Tin *gb = static_cast<const Tin *>(p.B) + bc0 + size_t(t0) * N;
+    const Tin *gc = static_cast<const Tin *>(p.C) + bc0 + size_t(t0) * N;
+    if constexpr (Cfg::VEC) {
+        constexpr int CPR = T / EIN;                 // 16-byte chunks per row
+        constexpr int ROWC = 3 * CH * CPR;
+#pragma unroll
+        for (int k = 0; k < (ROWC + NT - 1) / NT; ++k) {
+            const int i = tid_x() + k * NT;
+            const int a = i / (CH * CPR);
+            const int rem = i % (CH * CPR);
+            const int cc = rem / CPR, q = rem % CPR;
+            if (i < ROWC && a < narr && cc < nch && t0 + q * EIN < L) {
+                const Tin *src = (a == 0 ? gx : a == 1 ? gd : gz) + size_t(cc) * L + t0 + q * EIN;
+                Tin *dst = (a == 0 ? s.xs : a == 1 ? s.ds : s.zs) + cc * Cfg::RAW_ROW + q * EIN;
+                cp_async_16(dst, src);
+            }
+        }
+        if (N == NP) {                               // dense B, C rows: T * NP values each
+            constexpr int BCC = T * NP / EIN;        // chunks per array
+            constexpr int TOK_PER_CHUNK_NUM = EIN;   // a chunk holds EIN / NP tokens' values
+#pragma unroll
+            for (int k = 0; k < (2 * BCC + NT - 1) / NT; ++k) {
+                const int i = tid_x() + k * NT;
+                const int which = i / BCC, q = i % BCC;
+                if (i < 2 * BCC && t0 + (q * TOK_PER_CHUNK_NUM) / NP < L)
+                    cp_async_16((which ? s.cs : s.bs) + q * EIN, (which ? gc : gb) + q * EIN);
+            }
+        } else {
+            const int valid_t = min(T, L - t0);
+            const int bc_chunks = (valid_t * N * int(sizeof(Tin))) / 16;
+            for (int i = tid_x(); i < 2 * bc_chunks; i += NT) {
+                const int which = i >= bc_chunks;
+                const int q = i - which * bc_chunks;
+                cp_async_16((which ? s.cs : s.bs) + q * EIN, (which ? gc : gb) + q * EIN);
+            }
+        }
+    } else {
+        constexpr int NEL = 3 * CH * T;
+#pragma unroll 4
+        for (int k = 0; k < (NEL + NT - 1) / NT; ++k) {
+            const int i = tid_x() + k * NT;
+            const int a = i / (CH * T);
+            const int rem = i % (CH * T);
+            const int cc = rem / T, tt = rem % T;
+            if (i < NEL && a < narr && cc < nch && t0 + tt < L) {
+                const Tin *src = (a == 0 ? gx : a == 1 ? gd : gz) + size_t(cc) * L + t0 + tt;
+                Tin *dst = (a == 0 ? s.xs : a == 1 ? s.ds : s.zs) + cc * Cfg::RAW_ROW + tt;
+                *dst = *src;
+            }
+        }
+        const int nbc = min(T, L - t0) * N;
+        for (int i = tid_x(); i < 2 * nbc; i += NT) {
+            const int which = i >= nbc;
+            const int q = i - which * nbc;
+            (which ? s.cs : s.bs)[q] = (which ? gc : gb)[q];
+        }
+    }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::NTHREADS, Cfg::MINB)
+scan_lanes_kernel(const ScanArgs p) {
+    using Tin = typename Cfg::Tin;
+    using Tout = typename Cfg::Tout;
+    constexpr int NP = Cfg::NP, Q = Cfg::Q, CH = Cfg::CH, T = Cfg::T, NT = Cfg::NTHREADS;
+    extern __shared__ __align__(16) unsigned char smem[];
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int cg = warp / Q;            // channel group of this warp
+    const int q = warp - cg * Q;        // state quad of this warp
+    const int c = cg * 32 + lane;       // channel within the CTA
+    const int b = blockIdx.x / p.groups_per_seq;
+    const int d0 = (blockIdx.x - b * p.groups_per_seq) * CH;
+    const int L = p.seqlen, N = p.dstate, dim = p.dim;
+    const int nch = min(CH, dim - d0);
+    const bool dvalid = c < nch;
+
+    float4 *prep = reinterpret_cast<float4 *>(smem + Cfg::OFF_PREP);
+    float *Bf = reinterpret_cast<float *>(smem + Cfg::OFF_BF);
+    float *Cf = reinterpret_cast<float *>(smem + Cfg::OFF_CF);
+    float *yp = reinterpret_cast<float *>(smem + Cfg::OFF_YP);
+    Tout *ys = reinterpret_cast<Tout *>(smem + Cfg::OFF_Y);
+
+    // this lane's 4 states: A * log2(e)
+    float A2[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const int n = 4 * q + s;
+        A2[s] = (dvalid && n < N) ? p.A[size_t(d0 + c) * N + n] * kLog2e : 0.f;
+    }
+    // per chunk task: its channel is the same in every tile, so bias and D live in registers
+    float tbias[Cfg::TASKS_PER_THREAD], tD[Cfg::TASKS_PER_THREAD];
+#pragma unroll
+    for (int k = 0; k < Cfg::TASKS_PER_THREAD; ++k) {
+        const int cc = (tid + k * NT) % CH;
+        tbias[k] = (p.delta_bias != nullptr && cc < nch) ? p.delta_bias[d0 + cc] : 0.f;
+        tD[k] = (p.D != nullptr && cc < nch) ? p.D[d0 + cc] : 0.f;
+    }
+
+    const size_t row0 = (size_t(b) * dim + d0) * size_t(L);
+    const size_t bc0 = size_t(b) * L * size_t(N);
+    const int ntiles = (L + T - 1) / T;
+
+#pragma unroll
+    for (int s = 0; s < Cfg::NSTAGE - 1; ++s) {
+        if (s < ntiles) load_tile_lanes<Cfg>(p, smem, s, s * T, row0, bc0, nch);
+        cp_async_commit();
+    }
+
+    float h[4] = {0.f, 0.f, 0.f, 0.f};
+
+    for (int tile = 0; tile < ntiles; ++tile) {
+        const int st = tile % Cfg::NSTAGE;
+        const int t0 = tile * T;
+        cp_async_wait<Cfg::NSTAGE - 2>();
+        __syncthreads();
+        {
+            const int nt = tile + Cfg::NSTAGE - 1;
+            if (nt < ntiles) load_tile_lanes<Cfg>(p, smem, nt % Cfg::NSTAGE, nt * T, row0, bc0, nch);
+            cp_async_commit();
+        }
+        Stage<Cfg> sv(smem, st);
+
+        // ---- prep: Delta and Delta*x once per (t, d); task = (channel, 8-token chunk),
+        //      lanes run over channels so the 16-byte row reads and writes are conflict free
+#pragma unroll
+        for (int k = 0; k < Cfg::TASKS_PER_THREAD; ++k) {
+            const int task = tid + k * NT;
+            const int cc = task % CH, t8 = task / CH;
+            float dr[8], xr[8];
+            load8<Tin>(sv.ds + cc * Cfg::RAW_ROW + 8 * t8, dr);
+            load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+            const float bias = tbias[k];
+            float o[16];
+            if (cc < nch && t0 + 8 * t8 + 8 <= L) {          // whole chunk inside the data
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    float dl = dr[u] + bias;
+                    if (p.softplus) dl = softplus_f(dl);
+                    o[2 * u] = dl;
+                    o[2 * u + 1] = dl * xr[u];
+                }
+            } else {
+                const bool cok = cc < nch;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    float dl = dr[u] + bias;
+                    if (p.softplus) dl = softplus_f(dl);
+                    const bool ok = cok && (t0 + 8 * t8 + u < L);   // past L / dim: no-op token
+                    o[2 * u] = ok ? dl : 0.f;
+                    o[2 * u + 1] = ok ? dl * xr[u] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int u2 = 0; u2 < 4; ++u2)
+                prep[(4 * t8 + u2) * CH + cc] = make_float4(o[4 * u2], o[4 * u2 + 1], o[4 * u2 + 2], o[4 * u2 + 3]);
+        }
+        // B, C of the tile widened to fp32, zero past dstate / past L
+        if (N == NP && t0 + T <= L) {                       // dense rows: 8 values at a time
+            constexpr int NV = T * NP / 8;
+#pragma unroll
+            for (int k = 0; k < (2 * NV + NT - 1) / NT; ++k) {
+                const int i = tid + k * NT;
+                if (i < 2 * NV) {
+                    const int which = i >= NV;
+                    const int v = i - which * NV;
+                    float f[8];
+                    load8<Tin>((which ? sv.cs : sv.bs) + 8 * v, f);
+                    store8<float>((which ? Cf : Bf) + 8 * v, f);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < (T * NP + NT - 1) / NT; ++k) {
+                const int i = tid + k * NT;
+                if (i < T * NP) {
+                    const int tt = i / NP, n = i % NP;
+                    const bool ok = n < N && t0 + tt < L;
+                    Bf[i] = ok ? to_f32(sv.bs[tt * N + n]) : 0.f;
+                    Cf[i] = ok ? to_f32(sv.cs[tt * N + n]) : 0.f;
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- the recurrence: 4 states of one channel per lane, carried across tiles ----
+        {
+            const float4 *pp = prep + c;
+            float *ypr = yp + (q * CH + c) * Cfg::YP_ROW;
+            // decays a = exp(Delta*A) and writes w = Delta*x*B of the 4 tokens of group g
+            auto decay_write = [&](int g, float (&a)[4][4], float (&w)[4][4]) {
+                const float4 d01 = pp[(2 * g) * CH];   // (Delta, Delta*x) of tokens 4g, 4g+1
+                const float4 d23 = pp[(2 * g + 1) * CH];
+                const float dl[4] = {d01.x, d01.z, d23.x, d23.z};
+                const float dx[4] = {d01.y, d01.w, d23.y, d23.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 bq = *reinterpret_cast<const float4 *>(Bf + (4 * g + u) * NP + 4 * q);
+                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        a[u][s] = ex2_approx(dl[u] * A2[s]);
+                        w[u][s] = dx[u] * bb[s];
+                    }
+                }
+            };
+            auto recur_read = [&](int g, const float (&a)[4][4], const float (&w)[4][4]) {
+                float out[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 cq = *reinterpret_cast<const float4 *>(Cf + (4 * g + u) * NP + 4 * q);
+                    const float cc4[4] = {cq.x, cq.y, cq.z, cq.w};
+                    float acc = 0.f;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        h[s] = fmaf(a[u][s], h[s], w[u][s]);
+                        acc = fmaf(cc4[s], h[s], acc);
+                    }
+                    out[u] = acc;
+                }
+                *reinterpret_cast<float4 *>(ypr + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
+            };
+            if constexpr (Cfg::PIPE) {
+                float a0[4][4], w0[4][4];
+                decay_write(0, a0, w0);
+#pragma unroll
+                for (int g = 0; g < T / 4; ++g) {
+                    float a1[4][4], w1[4][4];
+                    if (g + 1 < T / 4) decay_write(g + 1, a1, w1);
+                    recur_read(g, a0, w0);
+                    if (g + 1 < T / 4) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+#pragma unroll
+                            for (int s = 0; s < 4; ++s) { a0[u][s] = a1[u][s]; w0[u][s] = w1[u][s]; }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int g = 0; g < T / 4; ++g) {
+                    float a0[4][4], w0[4][4];
+                    decay_write(g, a0, w0);
+                    recur_read(g, a0, w0);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- epilogue: sum the quads, skip, gate, convert; stage y rows ----
+#pragma unroll
+        for (int k = 0; k < Cfg::TASKS_PER_THREAD; ++k) {
+            const int task = tid + k * NT;
+            const int cc = task % CH, t8 = task / CH;
+            float acc[8];
+            {
+                const float *src = yp + cc * Cfg::YP_ROW + 8 * t8;
+                const float4 a0 = *reinterpret_cast<const float4 *>(src);
+                const float4 a1 = *reinterpret_cast<const float4 *>(src + 4);
+                acc[0] = a0.x; acc[1] = a0.y; acc[2] = a0.z; acc[3] = a0.w;
+                acc[4] = a1.x; acc[5] = a1.y; acc[6] = a1.z; acc[7] = a1.w;
+            }
+#pragma unroll
+            for (int qq = 1; qq < Q; ++qq) {
+                const float *src = yp + (qq * CH + cc) * Cfg::YP_ROW + 8 * t8;
+                const float4 a0 = *reinterpret_cast<const float4 *>(src);
+                const float4 a1 = *reinterpret_cast<const float4 *>(src + 4);
+                acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
+                acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
+            }
+            float xr[8];
+            load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+            const float Dd = tD[k];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = fmaf(Dd, xr[u], acc[u]);
+            if (p.z != nullptr) {
+                float zr[8];
+                load8<Tin>(sv.zs + cc * Cfg::RAW_ROW + 8 * t8, zr);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[u] *= silu_f(zr[u]);
+            }
+            store8<Tout>(ys + cc * Cfg::Y_ROW + 8 * t8, acc);
+        }
+        __syncthreads();
+
+        // ---- write y rows back (coalesced) ----
+        Tout *gy = static_cast<Tout *>(p.y) + row0;
+        if constexpr (Cfg::VEC) {
+            constexpr int CPR = T / Cfg::EOUT;
+#pragma unroll
+            for (int k = 0; k < (CH * CPR + NT - 1) / NT; ++k) {
+                const int i = tid + k * NT;
+                const int cc = i / CPR, qq = i % CPR;
+                const int tg = t0 + qq * Cfg::EOUT;
+                if (i < CH * CPR && cc < nch && tg < L)
+                    *reinterpret_cast<uint4 *>(gy + size_t(cc) * L + tg) =
+                        *reinterpret_cast<const uint4 *>(ys + cc * Cfg::Y_ROW + qq * Cfg::EOUT);
+            }
+        } else {
+            for (int i = tid; i < nch * T; i += NT) {
+                const int cc = i / T, tt = i % T;
+                if (t0 + tt < L) gy[size_t(cc) * L + t0 + tt] = ys[cc * Cfg::Y_ROW + tt];
+            }
+        }
+    }
+    cp_async_wait<0>();
+
+    if (p.final_state != nullptr && dvalid) {
+        float *fs = p.final_state + (size_t(b) * dim + d0 + c) * N;
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            if (4 * q + s < N) fs[4 * q + s] = h[s];
+    }
+}
+
+}  // namespace ssm

@@ -9,6 +9,9 @@
 
 #include "../../include/ssm.h"
 #include "scan_fwd.cuh"
+#include "scan_lanes.cuh"
+#include "scan_ws.cuh"
+#include "scan_fused.cuh"
 #include "state_step.cuh"
 
 namespace {
@@ -32,8 +35,8 @@ int choose_split(long long channels) {
     return channels >= 8192 ? 1 : 4;
 }
 
-template <class Cfg>
-int launch_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
+template <class Cfg, class Kernel>
+int launch_cfg(Kernel kernel, const ssm::ScanArgs &a0, cudaStream_t stream) {
     ssm::ScanArgs a = a0;
     const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
     const long long blocks = groups * (long long)a.batch;
@@ -41,23 +44,51 @@ int launch_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     a.groups_per_seq = int(groups);
     const size_t smem = Cfg::SMEM_BYTES;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return SSM_ERR_CUDA;
     }
-    ssm::scan_fwd_kernel<Cfg><<<unsigned(blocks), Cfg::NTHREADS, smem, stream>>>(a);
+    kernel<<<unsigned(blocks), Cfg::NTHREADS, smem, stream>>>(a);
     return status_of(cudaGetLastError());
 }
 
-// NP (padded states) x split -> tile shape.  K = 1: one warp per channel group, 32-token
-// tiles, 4 channel groups per CTA.  K = 4: four 8-token sub-chunks per 32-token tile,
-// 2 channel groups per CTA.
+template <class Cfg> int launch_scan(const ssm::ScanArgs &a, cudaStream_t s) {
+    return launch_cfg<Cfg>(ssm::scan_fwd_kernel<Cfg>, a, s);
+}
+
+template <class Cfg> int launch_lanes(const ssm::ScanArgs &a, cudaStream_t s) {
+    return launch_cfg<Cfg>(ssm::scan_lanes_kernel<Cfg>, a, s);
+}
+
+template <class Cfg> int launch_ws(const ssm::ScanArgs &a, cudaStream_t s) {
+    return launch_cfg<Cfg>(ssm::scan_ws_kernel<Cfg>, a, s);
+}
+
+template <class Cfg> int launch_fused(const ssm::ScanArgs &a, cudaStream_t s) {
+    return launch_cfg<Cfg>(ssm::scan_fused_kernel<Cfg>, a, s);
+}
+
+// split 1: one channel per lane, state carried in registers over the whole sequence
+// (warp-specialised kernel; SSM_SCAN_IMPL=lanes selects the single-role variant for
+// measurement when the state is 16 wide).
+// split 4: four stitched 8-token sub-chunks per 32-token tile (few channels, long L).
 template <int NP, typename Tin, typename Tout, bool VEC>
 int dispatch_split(const ssm::ScanArgs &a, int split, cudaStream_t s) {
-    constexpr int CG1 = (NP == 16) ? 4 : (NP == 8 ? 2 : 1);
+    if (split == 1) {
+        const char *impl = std::getenv("SSM_SCAN_IMPL");
+        if constexpr (NP == 16) {
+            if (impl && std::strcmp(impl, "lanes") == 0)
+                return launch_lanes<ssm::LaneCfg<16, 1, 32, 3, Tin, Tout, VEC, 4, true>>(a, s);
+            if (impl && std::strcmp(impl, "ws") == 0)
+                return launch_ws<ssm::WsCfg<16, 4, 16, Tin, Tout, VEC, 3>>(a, s);
+            return launch_fused<ssm::FusedCfg<16, 16, Tin, Tout, VEC, 4>>(a, s);
+        } else if constexpr (NP == 8) {
+            return launch_fused<ssm::FusedCfg<8, 16, Tin, Tout, VEC, 5>>(a, s);
+        } else {
+            return launch_fused<ssm::FusedCfg<4, 16, Tin, Tout, VEC, 8>>(a, s);
+        }
+    }
     constexpr int CG4 = (NP == 16) ? 2 : 1;
-    if (split == 1) return launch_scan<ssm::ScanCfg<NP, 1, 32, CG1, 3, Tin, Tout, VEC>>(a, s);
-    return launch_scan<ssm::ScanCfg<NP, 4, 8, CG4, 3, Tin, Tout, VEC>>(a, s);
+    return launch_scan<ssm::ScanCfg<NP, 4, 8, CG4, 3, Tin, Tout, VEC, 1>>(a, s);
 }
 
 template <typename Tin, typename Tout>
@@ -73,17 +104,25 @@ int dispatch_np(const ssm::ScanArgs &a, int split, bool vec, cudaStream_t s) {
                : dispatch_split<16, Tin, Tout, false>(a, split, s);
 }
 
-template <int NP, typename Tin, typename Tout>
-int launch_step_np(const ssm::StepArgs &a, cudaStream_t s) {
+template <int NP, int J, typename Tin, typename Tout>
+int launch_step_j(const ssm::StepArgs &a, cudaStream_t s) {
     constexpr int G = NP / 4;
-    const long long threads = (long long)a.batch * a.dim * G;
-    const long long blocks = (threads + 255) / 256;
+    const long long quads = (long long)a.batch * a.dim * G;
+    const long long blocks = (quads + 256LL * J - 1) / (256LL * J);
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
     if (a.dstate % 4 == 0)
-        ssm::state_step_kernel<NP, Tin, Tout, true><<<unsigned(blocks), 256, 0, s>>>(a);
+        ssm::state_step_kernel<NP, Tin, Tout, true, J><<<unsigned(blocks), 256, 0, s>>>(a);
     else
-        ssm::state_step_kernel<NP, Tin, Tout, false><<<unsigned(blocks), 256, 0, s>>>(a);
+        ssm::state_step_kernel<NP, Tin, Tout, false, J><<<unsigned(blocks), 256, 0, s>>>(a);
     return status_of(cudaGetLastError());
+}
+
+// Channel-quads per thread of the decode step; SSM_STEP_J=1|4 overrides (measurement only).
+template <int NP, typename Tin, typename Tout>
+int launch_step_np(const ssm::StepArgs &a, cudaStream_t s) {
+    const char *e = std::getenv("SSM_STEP_J");
+    if (e && e[0] == '4') return launch_step_j<NP, 4, Tin, Tout>(a, s);
+    return launch_step_j<NP, 1, Tin, Tout>(a, s);
 }
 
 template <typename Tin, typename Tout>

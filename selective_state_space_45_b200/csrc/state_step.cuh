@@ -29,74 +29,103 @@ struct StepArgs {
     int batch, dim, dstate;
 };
 
-template <int NP, typename Tin, typename Tout, bool VEC4>
+// 4 consecutive input values (8 or 16 bytes, aligned) as fp32.
+template <typename T> __device__ __forceinline__ void load4_nc(const T *src, float (&v)[4]);
+template <> __device__ __forceinline__ void load4_nc<float>(const float *src, float (&v)[4]) {
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(src));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <> __device__ __forceinline__ void load4_nc<__nv_bfloat16>(const __nv_bfloat16 *src, float (&v)[4]) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(src));
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+
+// One thread = J channel-quads (4 states each).  Quad j of a thread is global quad
+// gq = (blockIdx.x * J + j) * blockDim.x + threadIdx.x, so each of the J accesses of a
+// warp covers 32 consecutive quads (512 contiguous bytes of state at N = 16).  Every load
+// of all J quads is issued before the first store (the state is written in place, so a
+// store could otherwise hold back the next quad's loads), keeping J * 16 bytes of state
+// in flight per thread.
+template <int NP, typename Tin, typename Tout, bool VEC4, int J>
 __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
     constexpr int G = NP / 4;
-    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long nchan = (long long)p.batch * p.dim;
-    const long long chl = gid / G;
-    const int r = int(gid - chl * G);
-    const bool active = chl < nchan;
-    const long long ch = active ? chl : 0;   // inactive lanes still join the shuffles
+    const long long nquad = (long long)p.batch * p.dim * G;
     const int N = p.dstate;
-    const int b = int(ch / p.dim);
-    const int d = int(ch - (long long)b * p.dim);
-
-    const float dl = to_f32(static_cast<const Tin *>(p.delta)[ch]);
-    const float xv = to_f32(static_cast<const Tin *>(p.x)[ch]);
-    const float dx = dl * xv;
-    const Tin *Bb = static_cast<const Tin *>(p.B) + (size_t)b * N;
-    const Tin *Cb = static_cast<const Tin *>(p.C) + (size_t)b * N;
-    float *hp = p.state + (size_t)ch * N;
-    const float *Ap = p.A + (size_t)d * N;
-    const int n0 = 4 * r;
-
-    float h[4], a4[4], bb[4], cc[4];
-    if constexpr (VEC4) {   // N % 4 == 0: whole 16-byte quads
-        const bool q = active && n0 < N;
-        float4 hv = q ? *reinterpret_cast<const float4 *>(hp + n0) : make_float4(0.f, 0.f, 0.f, 0.f);
-        float4 av = q ? __ldg(reinterpret_cast<const float4 *>(Ap + n0)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        h[0] = hv.x; h[1] = hv.y; h[2] = hv.z; h[3] = hv.w;
-        a4[0] = av.x; a4[1] = av.y; a4[2] = av.z; a4[3] = av.w;
+    long long chs[J];
+    int rs[J], ds[J];
+    bool act[J];
+    float h[J][4], a4[J][4], bb[J][4], cc[J][4], dl[J], xv[J], zv[J], Dv[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const long long g = ((long long)blockIdx.x * J + j) * blockDim.x + threadIdx.x;
+        act[j] = g < nquad;
+        const long long q = act[j] ? g : 0;          // inactive lanes still join the shuffles
+        const long long ch = q / G;
+        const int r = int(q - ch * G);
+        const int b = int(ch / p.dim);
+        const int d = int(ch - (long long)b * p.dim);
+        chs[j] = ch; rs[j] = r; ds[j] = d;
+        const int n0 = 4 * r;
+        const float *hp = p.state + (size_t)ch * N + n0;
+        const float *Ap = p.A + (size_t)d * N + n0;
+        const Tin *Bb = static_cast<const Tin *>(p.B) + (size_t)b * N + n0;
+        const Tin *Cb = static_cast<const Tin *>(p.C) + (size_t)b * N + n0;
+        if constexpr (VEC4) {   // N % 4 == 0: whole 16-byte quads
+            if (act[j] && n0 < N) {
+                const float4 hv = *reinterpret_cast<const float4 *>(hp);
+                const float4 av = __ldg(reinterpret_cast<const float4 *>(Ap));
+                h[j][0] = hv.x; h[j][1] = hv.y; h[j][2] = hv.z; h[j][3] = hv.w;
+                a4[j][0] = av.x; a4[j][1] = av.y; a4[j][2] = av.z; a4[j][3] = av.w;
+                load4_nc<Tin>(Bb, bb[j]);
+                load4_nc<Tin>(Cb, cc[j]);
+            } else {
+#pragma unroll
+                for (int s = 0; s < 4; ++s) h[j][s] = a4[j][s] = bb[j][s] = cc[j][s] = 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const bool ok = act[j] && n0 + s < N;
+                h[j][s] = ok ? hp[s] : 0.f;
+                a4[j][s] = ok ? Ap[s] : 0.f;
+                bb[j][s] = ok ? to_f32(Bb[s]) : 0.f;
+                cc[j][s] = ok ? to_f32(Cb[s]) : 0.f;
+            }
+        }
+        dl[j] = to_f32(static_cast<const Tin *>(p.delta)[ch]);
+        xv[j] = to_f32(static_cast<const Tin *>(p.x)[ch]);
+        zv[j] = p.z != nullptr ? to_f32(static_cast<const Tin *>(p.z)[ch]) : 0.f;
+        Dv[j] = p.D != nullptr ? p.D[d] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const float dx = dl[j] * xv[j];
+        float acc = 0.f;
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-            bb[s] = q ? to_f32(Bb[n0 + s]) : 0.f;
-            cc[s] = q ? to_f32(Cb[n0 + s]) : 0.f;
+            h[j][s] = fmaf(ex2_approx(dl[j] * a4[j][s] * kLog2e), h[j][s], dx * bb[j][s]);
+            acc = fmaf(cc[j][s], h[j][s], acc);
         }
-    } else {
+        const int n0 = 4 * rs[j];
+        float *hp = p.state + (size_t)chs[j] * N + n0;
+        if constexpr (VEC4) {
+            if (act[j] && n0 < N)
+                *reinterpret_cast<float4 *>(hp) = make_float4(h[j][0], h[j][1], h[j][2], h[j][3]);
+        } else {
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const bool q = active && n0 + s < N;
-            h[s] = q ? hp[n0 + s] : 0.f;
-            a4[s] = q ? Ap[n0 + s] : 0.f;
-            bb[s] = q ? to_f32(Bb[n0 + s]) : 0.f;
-            cc[s] = q ? to_f32(Cb[n0 + s]) : 0.f;
+            for (int s = 0; s < 4; ++s)
+                if (act[j] && n0 + s < N) hp[s] = h[j][s];
         }
-    }
-
-    float acc = 0.f;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        h[s] = fmaf(ex2_approx(dl * a4[s] * kLog2e), h[s], dx * bb[s]);
-        acc = fmaf(cc[s], h[s], acc);
-    }
-
-    if constexpr (VEC4) {
-        if (active && n0 < N)
-            *reinterpret_cast<float4 *>(hp + n0) = make_float4(h[0], h[1], h[2], h[3]);
-    } else {
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-            if (active && n0 + s < N) hp[n0 + s] = h[s];
-    }
-
-#pragma unroll
-    for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-
-    if (active && r == 0) {
-        float yv = fmaf(p.D != nullptr ? p.D[d] : 0.f, xv, acc);
-        if (p.z != nullptr) yv *= silu_f(to_f32(static_cast<const Tin *>(p.z)[ch]));
-        static_cast<Tout *>(p.y)[ch] = from_f32<Tout>(yv);
+        for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (act[j] && rs[j] == 0) {
+            float yv = fmaf(Dv[j], xv[j], acc);
+            if (p.z != nullptr) yv *= silu_f(zv[j]);
+            static_cast<Tout *>(p.y)[chs[j]] = from_f32<Tout>(yv);
+        }
     }
 }
 
