@@ -72,7 +72,7 @@ struct ScanCfg {
     static constexpr int Y_ROW = T + EOUT;          // spread channels over banks
     static constexpr int PREP_ROW = T + 1;          // float2 elements
     static_assert(TS % G == 0, "sub-chunk must be a multiple of the lane group");
-    static_assert(K > 1 || TS % 4 == 0, "the register-carried scan works in 4-token blocks");
+    static_assert(K > 1, "the stitched kernel splits every tile over several warps");
     static_assert((T * sizeof(Tin)) % 16 == 0 && (T * sizeof(Tout)) % 16 == 0, "tile rows");
 
     // shared-memory layout (byte offsets, 16-byte aligned pieces)
@@ -227,7 +227,7 @@ scan_fwd_kernel(const ScanArgs p) {
         cp_async_commit();
     }
 
-    float h[4] = {0.f, 0.f, 0.f, 0.f};       // K == 1: carried state; K > 1: last carry (warp K-1)
+    float h[4] = {0.f, 0.f, 0.f, 0.f};       // carry after the last tile (kept by warp K-1)
     int cur = 0;                               // carry double-buffer index (K > 1)
 
     for (int tile = 0; tile < ntiles; ++tile) {
@@ -266,58 +266,7 @@ scan_fwd_kernel(const ScanArgs p) {
         // over the G lanes of the channel.
         float yout[TS / G];
         const float2 *prow = prep + c * Cfg::PREP_ROW + j * TS;
-        if constexpr (K == 1) {
-            // Blocks of 4 tokens.  The decays exp(Delta*a) and writes Delta*x*B of the
-            // NEXT block are computed before the recurrence of the current one, so the
-            // 16 independent SFU operations of a block overlap the short FFMA chain.
-            constexpr int TB = 4;
-            constexpr int NB = TS / TB;
-            float ac[TB][4], wc[TB][4];
-            auto decay_write = [&](int i0, float (&a)[TB][4], float (&w)[TB][4]) {
-#pragma unroll
-                for (int u = 0; u < TB; ++u) {
-                    const float2 dd = prow[i0 + u];
-                    const float4 bq = *reinterpret_cast<const float4 *>(Bf + (i0 + u) * NP + 4 * r);
-                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        a[u][s] = ex2_approx(dd.x * A2[s]);
-                        w[u][s] = dd.y * bb[s];
-                    }
-                }
-            };
-            decay_write(0, ac, wc);
-#pragma unroll
-            for (int blk = 0; blk < NB; ++blk) {
-                float an[TB][4], wn[TB][4];
-                if (blk + 1 < NB) decay_write((blk + 1) * TB, an, wn);
-                float yp[TB];
-#pragma unroll
-                for (int u = 0; u < TB; ++u) {
-                    const float4 cq = *reinterpret_cast<const float4 *>(Cf + (blk * TB + u) * NP + 4 * r);
-                    const float cc4[4] = {cq.x, cq.y, cq.z, cq.w};
-                    float acc = 0.f;
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        h[s] = fmaf(ac[u][s], h[s], wc[u][s]);
-                        acc = fmaf(cc4[s], h[s], acc);
-                    }
-                    yp[u] = acc;
-                }
-#pragma unroll
-                for (int g = 0; g < TB / G; ++g)
-                    yout[blk * (TB / G) + g] = GroupReduceScatter<G>::run(yp + g * G, r);
-                if (blk + 1 < NB) {
-#pragma unroll
-                    for (int u = 0; u < TB; ++u)
-#pragma unroll
-                        for (int s = 0; s < 4; ++s) {
-                            ac[u][s] = an[u][s];
-                            wc[u][s] = wn[u][s];
-                        }
-                }
-            }
-        } else {
+        {
             float hl[TS][4], Pl[TS][4];
             float hs[4] = {0.f, 0.f, 0.f, 0.f}, P[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
@@ -408,8 +357,8 @@ scan_fwd_kernel(const ScanArgs p) {
     }
     cp_async_wait<0>();
 
-    // ---- final state: held by every lane (K == 1) or by the last sub-chunk's warp ----
-    if (p.final_state != nullptr && dvalid && (K == 1 || j == K - 1)) {
+    // ---- final state: held by the last sub-chunk's warp ----
+    if (p.final_state != nullptr && dvalid && j == K - 1) {
         float *fs = p.final_state + (size_t(b) * dim + d) * N;
 #pragma unroll
         for (int s = 0; s < 4; ++s)

@@ -20,12 +20,11 @@
 #pragma once
 
 #include "common.cuh"
-#include "scan_fwd.cuh"   // ScanArgs
+#include "scan_fwd.cuh"   // ScanArgs, Stage
 
 namespace ssm {
 
-template <int NP_, int CG_, int T_, int NSTAGE_, typename Tin_, typename Tout_, bool VEC_, int MINB_,
-          bool PIPE_ = false>
+template <int NP_, int CG_, int T_, int NSTAGE_, typename Tin_, typename Tout_, bool VEC_, int MINB_>
 struct LaneCfg {
     using Tin = Tin_;
     using Tout = Tout_;
@@ -37,7 +36,6 @@ struct LaneCfg {
     static constexpr int NSTAGE = NSTAGE_;
     static constexpr bool VEC = VEC_;
     static constexpr int MINB = MINB_;
-    static constexpr bool PIPE = PIPE_;     // decays of the next 4 tokens before the current recurrence
     static constexpr int NWARP = Q * CG;
     static constexpr int NTHREADS = 32 * NWARP;
     static constexpr int EIN = 16 / sizeof(Tin);
@@ -337,27 +335,20 @@ scan_lanes_kernel(const ScanArgs p) {
                 }
                 *reinterpret_cast<float4 *>(ypr + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
             };
-            if constexpr (Cfg::PIPE) {
-                float a0[4][4], w0[4][4];
-                decay_write(0, a0, w0);
+            // decays and writes of the next 4 tokens are computed before the recurrence
+            // of the current 4, so the SFU work overlaps the FFMA chain
+            float a0[4][4], w0[4][4];
+            decay_write(0, a0, w0);
 #pragma unroll
-                for (int g = 0; g < T / 4; ++g) {
-                    float a1[4][4], w1[4][4];
-                    if (g + 1 < T / 4) decay_write(g + 1, a1, w1);
-                    recur_read(g, a0, w0);
-                    if (g + 1 < T / 4) {
+            for (int g = 0; g < T / 4; ++g) {
+                float a1[4][4], w1[4][4];
+                if (g + 1 < T / 4) decay_write(g + 1, a1, w1);
+                recur_read(g, a0, w0);
+                if (g + 1 < T / 4) {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
+                    for (int u = 0; u < 4; ++u)
 #pragma unroll
-                            for (int s = 0; s < 4; ++s) { a0[u][s] = a1[u][s]; w0[u][s] = w1[u][s]; }
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int g = 0; g < T / 4; ++g) {
-                    float a0[4][4], w0[4][4];
-                    decay_write(g, a0, w0);
-                    recur_read(g, a0, w0);
+                        for (int s = 0; s < 4; ++s) { a0[u][s] = a1[u][s]; w0[u][s] = w1[u][s]; }
                 }
             }
         }

@@ -10,8 +10,6 @@
 #include "../../include/ssm.h"
 #include "scan_fwd.cuh"
 #include "scan_lanes.cuh"
-#include "scan_ws.cuh"
-#include "scan_fused.cuh"
 #include "state_step.cuh"
 
 namespace {
@@ -59,33 +57,14 @@ template <class Cfg> int launch_lanes(const ssm::ScanArgs &a, cudaStream_t s) {
     return launch_cfg<Cfg>(ssm::scan_lanes_kernel<Cfg>, a, s);
 }
 
-template <class Cfg> int launch_ws(const ssm::ScanArgs &a, cudaStream_t s) {
-    return launch_cfg<Cfg>(ssm::scan_ws_kernel<Cfg>, a, s);
-}
-
-template <class Cfg> int launch_fused(const ssm::ScanArgs &a, cudaStream_t s) {
-    return launch_cfg<Cfg>(ssm::scan_fused_kernel<Cfg>, a, s);
-}
-
-// split 1: one channel per lane, state carried in registers over the whole sequence
-// (warp-specialised kernel; SSM_SCAN_IMPL=lanes selects the single-role variant for
-// measurement when the state is 16 wide).
+// split 1: one channel per lane, state carried in registers over the whole sequence.
 // split 4: four stitched 8-token sub-chunks per 32-token tile (few channels, long L).
 template <int NP, typename Tin, typename Tout, bool VEC>
 int dispatch_split(const ssm::ScanArgs &a, int split, cudaStream_t s) {
     if (split == 1) {
-        const char *impl = std::getenv("SSM_SCAN_IMPL");
-        if constexpr (NP == 16) {
-            if (impl && std::strcmp(impl, "lanes") == 0)
-                return launch_lanes<ssm::LaneCfg<16, 1, 32, 3, Tin, Tout, VEC, 4, true>>(a, s);
-            if (impl && std::strcmp(impl, "ws") == 0)
-                return launch_ws<ssm::WsCfg<16, 4, 16, Tin, Tout, VEC, 3>>(a, s);
-            return launch_fused<ssm::FusedCfg<16, 16, Tin, Tout, VEC, 4>>(a, s);
-        } else if constexpr (NP == 8) {
-            return launch_fused<ssm::FusedCfg<8, 16, Tin, Tout, VEC, 5>>(a, s);
-        } else {
-            return launch_fused<ssm::FusedCfg<4, 16, Tin, Tout, VEC, 8>>(a, s);
-        }
+        if constexpr (NP == 16) return launch_lanes<ssm::LaneCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>>(a, s);
+        else if constexpr (NP == 8) return launch_lanes<ssm::LaneCfg<8, 1, 32, 3, Tin, Tout, VEC, 8>>(a, s);
+        else return launch_lanes<ssm::LaneCfg<4, 2, 32, 3, Tin, Tout, VEC, 8>>(a, s);
     }
     constexpr int CG4 = (NP == 16) ? 2 : 1;
     return launch_scan<ssm::ScanCfg<NP, 4, 8, CG4, 3, Tin, Tout, VEC, 1>>(a, s);
@@ -117,11 +96,10 @@ int launch_step_j(const ssm::StepArgs &a, cudaStream_t s) {
     return status_of(cudaGetLastError());
 }
 
-// Channel-quads per thread of the decode step; SSM_STEP_J=1|4 overrides (measurement only).
+// One channel-quad per thread: at 32 registers the SM holds 2048 threads, each with its
+// 16-byte state load in flight, which measured faster than several quads per thread.
 template <int NP, typename Tin, typename Tout>
 int launch_step_np(const ssm::StepArgs &a, cudaStream_t s) {
-    const char *e = std::getenv("SSM_STEP_J");
-    if (e && e[0] == '4') return launch_step_j<NP, 4, Tin, Tout>(a, s);
     return launch_step_j<NP, 1, Tin, Tout>(a, s);
 }
 
