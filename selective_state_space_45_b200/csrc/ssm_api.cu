@@ -2,6 +2,7 @@
 //
 // Every entry point checks its arguments on the host before touching the GPU; a
 // rejected call launches nothing.  Kernels run on the caller's stream, asynchronously.
+#include <algorithm>
 #include <climits>
 #include <cstdint>
 #include <cstdlib>
@@ -9,7 +10,6 @@
 
 #include "../../include/ssm.h"
 #include "scan_fwd.cuh"
-#include "scan_lanes.cuh"
 #include "state_step.cuh"
 
 namespace {
@@ -22,65 +22,89 @@ bool valid_dtype(int t) { return t == SSM_F32 || t == SSM_BF16; }
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA; }
 
-// Time sub-chunks per tile: 1 keeps each channel's scan in one warp; 4 splits every
-// tile over four warps and stitches them, which fills the GPU when there are few
-// channels (long single sequences).  SSM_SCAN_SPLIT=1|4 forces one for measurement.
-int choose_split(long long channels) {
-    if (const char *e = std::getenv("SSM_SCAN_SPLIT")) {
+constexpr int kSmCount = 148;          // B200
+constexpr int kMinSegTokens = 4096;     // shortest segment worth a carry correction
+
+// Segments per sequence: 1 while the channel groups alone fill the GPU; otherwise enough
+// segments for about three CTAs per SM, each at least kMinSegTokens long.
+// SSM_SCAN_SEGMENTS=k forces k (used by the tests to reach the two-pass path).
+int choose_segments(long long channel_groups, int seqlen) {
+    if (const char *e = std::getenv("SSM_SCAN_SEGMENTS")) {
         const int v = std::atoi(e);
-        if (v == 1 || v == 4) return v;
+        if (v >= 1) return v;
     }
-    return channels >= 8192 ? 1 : 4;
+    if (channel_groups >= 2LL * kSmCount) return 1;
+    const long long want = (3LL * kSmCount + channel_groups - 1) / channel_groups;
+    const long long room = seqlen / kMinSegTokens;
+    return int(std::max(1LL, std::min(want, room)));
 }
 
-template <class Cfg, class Kernel>
-int launch_cfg(Kernel kernel, const ssm::ScanArgs &a0, cudaStream_t stream) {
-    ssm::ScanArgs a = a0;
-    const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
-    const long long blocks = groups * (long long)a.batch;
+template <class Cfg, bool SEG>
+int launch_scan_kernel(const ssm::ScanArgs &a, long long blocks, cudaStream_t stream) {
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
-    a.groups_per_seq = int(groups);
+    if (blocks == 0) return SSM_OK;
     const size_t smem = Cfg::SMEM_BYTES;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        cudaError_t e = cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, SEG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return SSM_ERR_CUDA;
     }
-    kernel<<<unsigned(blocks), Cfg::NTHREADS, smem, stream>>>(a);
+    ssm::scan_fwd_kernel<Cfg, SEG><<<unsigned(blocks), Cfg::NTHREADS, smem, stream>>>(a);
     return status_of(cudaGetLastError());
 }
 
-template <class Cfg> int launch_scan(const ssm::ScanArgs &a, cudaStream_t s) {
-    return launch_cfg<Cfg>(ssm::scan_fwd_kernel<Cfg>, a, s);
-}
-
-template <class Cfg> int launch_lanes(const ssm::ScanArgs &a, cudaStream_t s) {
-    return launch_cfg<Cfg>(ssm::scan_lanes_kernel<Cfg>, a, s);
-}
-
-// split 1: one channel per lane, state carried in registers over the whole sequence.
-// split 4: four stitched 8-token sub-chunks per 32-token tile (few channels, long L).
-template <int NP, typename Tin, typename Tout, bool VEC>
-int dispatch_split(const ssm::ScanArgs &a, int split, cudaStream_t s) {
-    if (split == 1) {
-        if constexpr (NP == 16) return launch_lanes<ssm::LaneCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>>(a, s);
-        else if constexpr (NP == 8) return launch_lanes<ssm::LaneCfg<8, 1, 32, 3, Tin, Tout, VEC, 8>>(a, s);
-        else return launch_lanes<ssm::LaneCfg<4, 2, 32, 3, Tin, Tout, VEC, 8>>(a, s);
+// One scan: a single pass when the sequence fits one CTA per channel group, else the two
+// segment passes with a stream-ordered scratch buffer of batch*dim*nseg*(NP+1) floats.
+template <class Cfg>
+int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
+    ssm::ScanArgs a = a0;
+    const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
+    if (groups > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    a.groups_per_seq = int(groups);
+    const long long cgroups = groups * a.batch;
+    int nseg = choose_segments(cgroups, a.seqlen);
+    long long seg_len = (a.seqlen + nseg - 1) / nseg;
+    seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
+    nseg = int((a.seqlen + seg_len - 1) / seg_len);
+    if (nseg <= 1) {
+        a.pass = 0;
+        a.nseg = 1;
+        a.seg_len = a.seqlen;
+        return launch_scan_kernel<Cfg, false>(a, cgroups, stream);
     }
-    constexpr int CG4 = (NP == 16) ? 2 : 1;
-    return launch_scan<ssm::ScanCfg<NP, 4, 8, CG4, 3, Tin, Tout, VEC, 1>>(a, s);
+    const size_t rows = size_t(a.batch) * a.dim * nseg;
+    const size_t bytes = rows * Cfg::NP * sizeof(float) + rows * sizeof(float);
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, bytes, stream) != cudaSuccess) return SSM_ERR_CUDA;
+    a.nseg = nseg;
+    a.seg_len = int(seg_len);
+    a.seg_h = static_cast<float *>(ws);
+    a.seg_s = a.seg_h + rows * Cfg::NP;
+    a.pass = 1;
+    int st = launch_scan_kernel<Cfg, true>(a, cgroups * nseg, stream);
+    if (st == SSM_OK) {
+        a.pass = 2;
+        st = launch_scan_kernel<Cfg, true>(a, cgroups * (nseg - 1), stream);
+    }
+    const cudaError_t fe = cudaFreeAsync(ws, stream);
+    if (st == SSM_OK && fe != cudaSuccess) st = SSM_ERR_CUDA;
+    return st;
+}
+
+// Tile shape per padded state width: 32-token tiles; 32 channels per CTA (64 at N <= 4).
+template <int NP, typename Tin, typename Tout, bool VEC>
+int dispatch_cfg(const ssm::ScanArgs &a, cudaStream_t s) {
+    if constexpr (NP == 16) return run_scan<ssm::ScanCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>>(a, s);
+    else if constexpr (NP == 8) return run_scan<ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>>(a, s);
+    else return run_scan<ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>>(a, s);
 }
 
 template <typename Tin, typename Tout>
-int dispatch_np(const ssm::ScanArgs &a, int split, bool vec, cudaStream_t s) {
+int dispatch_np(const ssm::ScanArgs &a, bool vec, cudaStream_t s) {
     const int N = a.dstate;
-    if (N <= 4)
-        return vec ? dispatch_split<4, Tin, Tout, true>(a, split, s)
-                   : dispatch_split<4, Tin, Tout, false>(a, split, s);
-    if (N <= 8)
-        return vec ? dispatch_split<8, Tin, Tout, true>(a, split, s)
-                   : dispatch_split<8, Tin, Tout, false>(a, split, s);
-    return vec ? dispatch_split<16, Tin, Tout, true>(a, split, s)
-               : dispatch_split<16, Tin, Tout, false>(a, split, s);
+    if (N <= 4) return vec ? dispatch_cfg<4, Tin, Tout, true>(a, s) : dispatch_cfg<4, Tin, Tout, false>(a, s);
+    if (N <= 8) return vec ? dispatch_cfg<8, Tin, Tout, true>(a, s) : dispatch_cfg<8, Tin, Tout, false>(a, s);
+    return vec ? dispatch_cfg<16, Tin, Tout, true>(a, s) : dispatch_cfg<16, Tin, Tout, false>(a, s);
 }
 
 template <int NP, int J, typename Tin, typename Tout>
@@ -159,13 +183,12 @@ int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_
     const int ein = in_dtype == SSM_F32 ? 4 : 8;
     const int eout = out_dtype == SSM_F32 ? 4 : 8;
     const bool vec = (seqlen % ein == 0) && (seqlen % eout == 0);
-    const int split = choose_split(channels);
 
-    if (in_dtype == SSM_F32 && out_dtype == SSM_F32) return dispatch_np<float, float>(a, split, vec, stream);
+    if (in_dtype == SSM_F32 && out_dtype == SSM_F32) return dispatch_np<float, float>(a, vec, stream);
     if (in_dtype == SSM_BF16 && out_dtype == SSM_BF16)
-        return dispatch_np<__nv_bfloat16, __nv_bfloat16>(a, split, vec, stream);
-    if (in_dtype == SSM_BF16) return dispatch_np<__nv_bfloat16, float>(a, split, vec, stream);
-    return dispatch_np<float, __nv_bfloat16>(a, split, vec, stream);
+        return dispatch_np<__nv_bfloat16, __nv_bfloat16>(a, vec, stream);
+    if (in_dtype == SSM_BF16) return dispatch_np<__nv_bfloat16, float>(a, vec, stream);
+    return dispatch_np<float, __nv_bfloat16>(a, vec, stream);
 }
 
 int ssm_state_step(float *state, const void *x, const void *delta, const float *A,

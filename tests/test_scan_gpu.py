@@ -14,16 +14,21 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.fixture(params=["1", "4"], ids=["split1", "split4"])
+@pytest.fixture(params=[None, "3"], ids=["oneCTA", "segments3"])
 def split(request):
-    """Both kernel shapes: one warp per channel group, and four stitched time sub-chunks."""
-    old = os.environ.get("SSM_SCAN_SPLIT")
-    os.environ["SSM_SCAN_SPLIT"] = request.param
-    yield int(request.param)
-    if old is None:
-        os.environ.pop("SSM_SCAN_SPLIT", None)
+    """Both scan paths: one CTA per channel group over the whole sequence, and the
+    sequence cut into (up to) 3 segments -- pass 1 from a zero state, pass 2 carrying
+    the true state into every later segment."""
+    old = os.environ.get("SSM_SCAN_SEGMENTS")
+    if request.param is None:
+        os.environ.pop("SSM_SCAN_SEGMENTS", None)
     else:
-        os.environ["SSM_SCAN_SPLIT"] = old
+        os.environ["SSM_SCAN_SEGMENTS"] = request.param
+    yield request.param
+    if old is None:
+        os.environ.pop("SSM_SCAN_SEGMENTS", None)
+    else:
+        os.environ["SSM_SCAN_SEGMENTS"] = old
 
 
 def run_gpu(ssm, inp, out_dtype, use_z=True, use_D=True, use_bias=True, softplus=True):
@@ -173,3 +178,38 @@ def test_misaligned_pointer_rejected_on_device(cuda_lib):
         cuda_lib.ssm_selective_scan_fwd(inp["x"], inp["delta"], None, True, inp["A"], inp["B"],
                                         inp["C"], None, None, y, None)
     assert e.value.status == cuda_lib.SSM_ERR_ALIGNMENT
+
+
+@pytest.mark.parametrize("nseg", ["2", "5"])
+def test_segment_carry_never_dies(cuda_lib, nseg, monkeypatch):
+    """A = 0 keeps exp(A * S) = 1: the carry reaches every token of every later segment,
+    so pass 2 must re-scan whole segments."""
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", nseg)
+    inp = inputs.make_scan_inputs(1, 40, 700, 16, torch.float32, device=DEV, seed=21)
+    inp["A"][:, :3] = 0.0
+    inp["A"][:, 3:8] = 0.05          # a slowly growing state as well
+    y, fs = run_gpu(cuda_lib, inp, torch.float32)
+    yr, fr = run_oracle(inp)
+    assert_parity(y, yr, torch.float32, what="y")
+    assert_parity(fs, fr, torch.float32, what="final_state")
+
+
+def test_segment_carry_dies_at_once(cuda_lib, monkeypatch):
+    """Huge steps wipe the carry within one token: pass 2 stops after its first tile and
+    the pass-1 output stands."""
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", "4")
+    inp = inputs.make_scan_inputs(2, 33, 512, 16, torch.bfloat16, device=DEV, seed=22)
+    inp["delta_bias"].fill_(60.0)
+    y, fs = run_gpu(cuda_lib, inp, torch.bfloat16)
+    yr, fr = run_oracle(inp)
+    assert_parity(y, yr, torch.bfloat16, torch.bfloat16, what="y")
+    assert_parity(fs, fr, torch.bfloat16, torch.float32, what="final_state")
+
+
+def test_long_sequence_default_segmentation(cuda_lib):
+    """Few channels and a long sequence choose the segmented path on their own."""
+    inp = inputs.make_scan_inputs(1, 64, 40000, 16, torch.bfloat16, device=DEV, seed=23)
+    y, fs = run_gpu(cuda_lib, inp, torch.float32)
+    yr, fr = run_oracle(inp)
+    assert_parity(y, yr, torch.bfloat16, torch.float32, what="y")
+    assert_parity(fs, fr, torch.bfloat16, torch.float32, what="final_state")
