@@ -22,34 +22,39 @@ bool valid_dtype(int t) { return t == SSM_F32 || t == SSM_BF16; }
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA; }
 
-constexpr int kSmCount = 148;          // B200
 constexpr int kMinSegTokens = 4096;     // shortest segment worth a carry correction
 
-// Segments per sequence: 1 while the channel groups alone fill the GPU; otherwise enough
-// segments for about three CTAs per SM, each at least kMinSegTokens long.
-// SSM_SCAN_SEGMENTS=k forces k (used by the tests to reach the two-pass path).
-int choose_segments(long long channel_groups, int seqlen) {
+// Segments per sequence: 1 while the channel groups alone fill every resident CTA slot
+// (`slots` = SMs x resident CTAs per SM); otherwise as many as fit in one wave of slots,
+// each at least kMinSegTokens long.  SSM_SCAN_SEGMENTS=k forces k (used by the tests to
+// reach the two-pass path).
+int choose_segments(long long channel_groups, int seqlen, long long slots) {
     if (const char *e = std::getenv("SSM_SCAN_SEGMENTS")) {
         const int v = std::atoi(e);
         if (v >= 1) return v;
     }
-    if (channel_groups >= 2LL * kSmCount) return 1;
-    const long long want = (3LL * kSmCount + channel_groups - 1) / channel_groups;
+    if (2 * channel_groups >= slots) return 1;
+    const long long want = slots / channel_groups;
     const long long room = seqlen / kMinSegTokens;
     return int(std::max(1LL, std::min(want, room)));
+}
+
+// Resident CTA slots of a kernel on the current device (0 if the query fails).
+template <class Kernel>
+long long resident_slots(Kernel kernel, int threads, size_t smem) {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess)
+        return 0;
+    return (long long)sms * per_sm;
 }
 
 template <class Cfg, bool SEG>
 int launch_scan_kernel(const ssm::ScanArgs &a, long long blocks, cudaStream_t stream) {
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
     if (blocks == 0) return SSM_OK;
-    const size_t smem = Cfg::SMEM_BYTES;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, SEG>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess) return SSM_ERR_CUDA;
-    }
-    ssm::scan_fwd_kernel<Cfg, SEG><<<unsigned(blocks), Cfg::NTHREADS, smem, stream>>>(a);
+    ssm::scan_fwd_kernel<Cfg, SEG><<<unsigned(blocks), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(a);
     return status_of(cudaGetLastError());
 }
 
@@ -62,7 +67,16 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     if (groups > INT_MAX) return SSM_ERR_UNSUPPORTED;
     a.groups_per_seq = int(groups);
     const long long cgroups = groups * a.batch;
-    int nseg = choose_segments(cgroups, a.seqlen);
+    const size_t smem = Cfg::SMEM_BYTES;
+    if (smem > 48 * 1024) {   // opt in to large shared memory for both kernel variants
+        if (cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess ||
+            cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess)
+            return SSM_ERR_CUDA;
+    }
+    const long long slots = resident_slots(ssm::scan_fwd_kernel<Cfg, true>, Cfg::NTHREADS, smem);
+    int nseg = choose_segments(cgroups, a.seqlen, slots > 0 ? slots : 2 * cgroups);
     long long seg_len = (a.seqlen + nseg - 1) / nseg;
     seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
     nseg = int((a.seqlen + seg_len - 1) / seg_len);
