@@ -18,8 +18,10 @@
  * state of fixed size").
  *
  * Conventions for every entry point:
- *  - All tensor pointers are DEVICE pointers owned by the caller; the library
- *    allocates no memory and keeps no state between calls.
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library keeps
+ *    no state between calls.  ssm_selective_scan_fwd may take a temporary scratch
+ *    buffer with cudaMallocAsync / cudaFreeAsync on cuda_stream (long sequences with
+ *    few channels, see below); every other call allocates nothing.
  *  - Every pointer must be 16-byte aligned (SSM_ERR_ALIGNMENT otherwise).
  *  - The call is asynchronous on `cuda_stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and never synchronises.  Argument errors are returned before
@@ -46,7 +48,8 @@ typedef enum {
     SSM_ERR_INVALID_ARG = 1,   /* null required pointer, negative size, bad dtype code   */
     SSM_ERR_UNSUPPORTED = 2,   /* dstate outside 1..16, sizes beyond the int32 index range */
     SSM_ERR_ALIGNMENT = 3,     /* a pointer not 16-byte aligned                            */
-    SSM_ERR_CUDA = 4           /* the CUDA runtime reported an error at launch             */
+    SSM_ERR_CUDA = 4,          /* the CUDA runtime reported an error at launch             */
+    SSM_ERR_SCRATCH = 5        /* ssm_selective_scan_fwd_noalloc: fixed scratch too small  */
 } ssm_status;
 
 /*
@@ -66,12 +69,47 @@ typedef enum {
  * state); 1 <= dstate <= 16; batch*dim*seqlen and batch*seqlen*dstate must be below 2^62
  * and seqlen below 2^31.
  * The N-wide state never leaves the chip: only y and final_state are written.
+ * When batch * ceil(dim / 32) CTAs cannot fill the GPU, each sequence is cut into segments
+ * scanned in parallel and stitched by their carries; their end states (batch * dim *
+ * segments * (padded dstate + 1) floats, a few MiB at most) go to a stream-ordered
+ * temporary buffer that is freed on the same stream before the call returns.
  */
 int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_bias,
                            int delta_softplus, const float *A, const void *B, const void *C,
                            const float *D, const void *z, void *y, float *final_state,
                            int batch, int dim, int seqlen, int dstate,
                            int in_dtype, int out_dtype, void *cuda_stream);
+
+/*
+ * Allocation-free variant of ssm_selective_scan_fwd: same arguments, same results, and no
+ * memory allocation of any kind (no cudaMalloc, cudaMallocAsync or cudaFree).  The pages
+ * have no counterpart to this call; it exists for callers that are not allowed to
+ * allocate device memory while they run: a serving engine that has handed all free
+ * device memory to its own pool before the first request, code running under an
+ * allocator policy that forbids the library to allocate behind its back, or a latency-
+ * critical loop that must not touch the allocator after start-up.
+ *
+ * Where ssm_selective_scan_fwd takes a stream-ordered temporary buffer (long sequences
+ * with few channels are scanned in segments whose end states must be kept between two
+ * passes), this call uses a fixed 4 MiB array in device memory instead.  That array
+ * exists on every GPU that loads the library and stays there until the process exits.
+ *  - The first call on a device looks up the array's device address (a one-time set-up
+ *    per device, done with that device current); make that first call before any CUDA
+ *    stream capture on the device.
+ *  - A call whose segmented scan would need more than 4 MiB of scratch (batch * dim *
+ *    segments * (padded dstate + 1) floats, padded dstate = 4, 8 or 16) returns
+ *    SSM_ERR_SCRATCH and launches nothing.  Calls that need no segments work at any size.
+ *  - All calls share the array and it keeps the contents of the last call.  Nothing in it
+ *    has to start at zero: each call writes every entry it later reads.  Two calls whose
+ *    kernels may overlap on the GPU (different streams, or different host threads without
+ *    ordering between their streams) race on the array and give wrong results; serialise
+ *    them on one stream.
+ */
+int ssm_selective_scan_fwd_noalloc(const void *x, const void *delta, const float *delta_bias,
+                                   int delta_softplus, const float *A, const void *B, const void *C,
+                                   const float *D, const void *z, void *y, float *final_state,
+                                   int batch, int dim, int seqlen, int dstate,
+                                   int in_dtype, int out_dtype, void *cuda_stream);
 
 /*
  * One decode step: every (b, d) channel takes one token and its state is updated in place.

@@ -9,6 +9,7 @@ from ._lib import (  # noqa: F401
     SSM_ERR_ALIGNMENT,
     SSM_ERR_CUDA,
     SSM_ERR_INVALID_ARG,
+    SSM_ERR_SCRATCH,
     SSM_ERR_UNSUPPORTED,
     SSM_F32,
     SSM_OK,
@@ -16,6 +17,7 @@ from ._lib import (  # noqa: F401
     load_library,
     selective_scan,
     ssm_selective_scan_fwd,
+    ssm_selective_scan_fwd_noalloc,
     ssm_state_step,
     ssm_status_string,
     ssm_version,

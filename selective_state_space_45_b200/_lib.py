@@ -16,7 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libssm.so")
 
 SSM_F32, SSM_BF16 = 0, 1
-SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_ALIGNMENT, SSM_ERR_CUDA = range(5)
+SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_ALIGNMENT, SSM_ERR_CUDA, SSM_ERR_SCRATCH = range(6)
 
 _DTYPE_CODE = {torch.float32: SSM_F32, torch.bfloat16: SSM_BF16}
 
@@ -46,6 +46,8 @@ def load_library(path: str | None = None):
         lib.ssm_selective_scan_fwd.restype = i
         lib.ssm_selective_scan_fwd.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp,
                                                i, i, i, i, i, i, vp]
+        lib.ssm_selective_scan_fwd_noalloc.restype = i
+        lib.ssm_selective_scan_fwd_noalloc.argtypes = list(lib.ssm_selective_scan_fwd.argtypes)
         lib.ssm_state_step.restype = i
         lib.ssm_state_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
         lib.ssm_status_string.restype = ctypes.c_char_p
@@ -96,6 +98,18 @@ def ssm_selective_scan_fwd(x, delta, delta_bias, delta_softplus, A, B, C, D, z, 
     batch, dim, L = x.shape
     N = A.shape[1]
     _check(load_library().ssm_selective_scan_fwd(
+        _ptr(x), _ptr(delta), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(A), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), _ptr(y), _ptr(final_state), batch, dim, L, N,
+        _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, x, y)))
+
+
+def ssm_selective_scan_fwd_noalloc(x, delta, delta_bias, delta_softplus, A, B, C, D, z, y,
+                                   final_state, stream=None):
+    """Allocation-free variant of ``ssm_selective_scan_fwd`` (see include/ssm.h): same
+    arguments and results; long sequences use a fixed device array for their scratch."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    _check(load_library().ssm_selective_scan_fwd_noalloc(
         _ptr(x), _ptr(delta), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(A), _ptr(B),
         _ptr(C), _ptr(D), _ptr(z), _ptr(y), _ptr(final_state), batch, dim, L, N,
         _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, x, y)))

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/ssm.h"
 #include "scan_fwd.cuh"
@@ -148,6 +149,99 @@ int launch_step(const ssm::StepArgs &a, cudaStream_t s) {
     return launch_step_np<16, Tin, Tout>(a, s);
 }
 
+
+// ---------------------------------------------------------------------------------
+// Allocation-free variant (ssm_selective_scan_fwd_noalloc).  The segment aggregates of
+// the two-pass scan live in this file-scope device array instead of a stream-ordered
+// allocation.  Every GPU that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;      // 4 MiB per GPU
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code the array's
+// name stands for a host-side shadow, not for device memory, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(float **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SSM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+            return SSM_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<float *>(ptr);
+    }
+    *out = g_noalloc_ptr[dev];
+    return SSM_OK;
+}
+
+// Same scan as run_scan, with the segment aggregates in the static array: nothing is
+// allocated.  Pass 1 writes every (channel, segment) row that pass 2 reads within the
+// same call, so the array needs no clearing between calls.
+template <class Cfg>
+int run_scan_noalloc(const ssm::ScanArgs &a0, cudaStream_t stream) {
+    ssm::ScanArgs a = a0;
+    const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
+    if (groups > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    a.groups_per_seq = int(groups);
+    const long long cgroups = groups * a.batch;
+    const size_t smem = Cfg::SMEM_BYTES;
+    if (smem > 48 * 1024) {
+        if (cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess ||
+            cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess)
+            return SSM_ERR_CUDA;
+    }
+    const long long slots = resident_slots(ssm::scan_fwd_kernel<Cfg, true>, Cfg::NTHREADS, smem);
+    int nseg = choose_segments(cgroups, a.seqlen, slots > 0 ? slots : 2 * cgroups);
+    long long seg_len = (a.seqlen + nseg - 1) / nseg;
+    seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
+    nseg = int((a.seqlen + seg_len - 1) / seg_len);
+    if (nseg <= 1) {
+        a.pass = 0;
+        a.nseg = 1;
+        a.seg_len = a.seqlen;
+        return launch_scan_kernel<Cfg, false>(a, cgroups, stream);
+    }
+    const size_t rows = size_t(a.batch) * a.dim * nseg;
+    if (rows * (Cfg::NP + 1) > kNoAllocScratchFloats) return SSM_ERR_SCRATCH;
+    float *ws = nullptr;
+    const int st0 = noalloc_scratch(&ws);
+    if (st0 != SSM_OK) return st0;
+    a.nseg = nseg;
+    a.seg_len = int(seg_len);
+    a.seg_h = ws;
+    a.seg_s = ws + rows * Cfg::NP;
+    a.pass = 1;
+    int st = launch_scan_kernel<Cfg, true>(a, cgroups * nseg, stream);
+    if (st == SSM_OK) {
+        a.pass = 2;
+        st = launch_scan_kernel<Cfg, true>(a, cgroups * (nseg - 1), stream);
+    }
+    return st;
+}
+
+template <int NP, typename Tin, typename Tout, bool VEC>
+int dispatch_cfg_noalloc(const ssm::ScanArgs &a, cudaStream_t s) {
+    if constexpr (NP == 16) return run_scan_noalloc<ssm::ScanCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>>(a, s);
+    else if constexpr (NP == 8) return run_scan_noalloc<ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>>(a, s);
+    else return run_scan_noalloc<ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>>(a, s);
+}
+
+template <typename Tin, typename Tout>
+int dispatch_np_noalloc(const ssm::ScanArgs &a, bool vec, cudaStream_t s) {
+    const int N = a.dstate;
+    if (N <= 4) return vec ? dispatch_cfg_noalloc<4, Tin, Tout, true>(a, s) : dispatch_cfg_noalloc<4, Tin, Tout, false>(a, s);
+    if (N <= 8) return vec ? dispatch_cfg_noalloc<8, Tin, Tout, true>(a, s) : dispatch_cfg_noalloc<8, Tin, Tout, false>(a, s);
+    return vec ? dispatch_cfg_noalloc<16, Tin, Tout, true>(a, s) : dispatch_cfg_noalloc<16, Tin, Tout, false>(a, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -161,6 +255,8 @@ const char *ssm_status_string(int status) {
     case SSM_ERR_UNSUPPORTED: return "unsupported size (dstate must be 1..16; grid too large)";
     case SSM_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case SSM_ERR_CUDA: return "CUDA runtime error at launch";
+    case SSM_ERR_SCRATCH:
+        return "the allocation-free scan needs more scratch than its fixed 4 MiB device array";
     default: return "unknown status";
     }
 }
@@ -203,6 +299,43 @@ int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_
         return dispatch_np<__nv_bfloat16, __nv_bfloat16>(a, vec, stream);
     if (in_dtype == SSM_BF16) return dispatch_np<__nv_bfloat16, float>(a, vec, stream);
     return dispatch_np<float, __nv_bfloat16>(a, vec, stream);
+}
+
+int ssm_selective_scan_fwd_noalloc(const void *x, const void *delta, const float *delta_bias,
+                                   int delta_softplus, const float *A, const void *B, const void *C,
+                                   const float *D, const void *z, void *y, float *final_state,
+                                   int batch, int dim, int seqlen, int dstate,
+                                   int in_dtype, int out_dtype, void *cuda_stream) {
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return SSM_ERR_INVALID_ARG;
+    if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1) return SSM_ERR_INVALID_ARG;
+    if (dstate > 16) return SSM_ERR_UNSUPPORTED;
+    const long long channels = (long long)batch * dim;
+    const bool work = channels > 0 && seqlen > 0;
+    if (work && (!x || !delta || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, delta, delta_bias, A, B, C, D, z, y, final_state};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSM_ERR_ALIGNMENT;
+    if (channels == 0) return SSM_OK;
+    if (!work && !final_state) return SSM_OK;
+
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (!work)   // empty sequences: the final state is the zero start state
+        return status_of(cudaMemsetAsync(final_state, 0, size_t(channels) * dstate * sizeof(float), stream));
+
+    ssm::ScanArgs a{};
+    a.x = x; a.delta = delta; a.delta_bias = delta_bias; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.z = z; a.y = y; a.final_state = final_state;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = dstate;
+    a.softplus = delta_softplus ? 1 : 0;
+    const int ein = in_dtype == SSM_F32 ? 4 : 8;
+    const int eout = out_dtype == SSM_F32 ? 4 : 8;
+    const bool vec = (seqlen % ein == 0) && (seqlen % eout == 0);
+
+    if (in_dtype == SSM_F32 && out_dtype == SSM_F32) return dispatch_np_noalloc<float, float>(a, vec, stream);
+    if (in_dtype == SSM_BF16 && out_dtype == SSM_BF16)
+        return dispatch_np_noalloc<__nv_bfloat16, __nv_bfloat16>(a, vec, stream);
+    if (in_dtype == SSM_BF16) return dispatch_np_noalloc<__nv_bfloat16, float>(a, vec, stream);
+    return dispatch_np_noalloc<float, __nv_bfloat16>(a, vec, stream);
 }
 
 int ssm_state_step(float *state, const void *x, const void *delta, const float *A,

@@ -31,7 +31,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for expected in ("ssm_selective_scan_fwd", "ssm_state_step", "ssm_status_string", "ssm_version"):
+    for expected in ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_noalloc", "ssm_state_step",
+                     "ssm_status_string", "ssm_version"):
         assert expected in names
 
 
@@ -43,7 +44,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_status_strings_and_version(lib):
     assert ssm.ssm_status_string(ssm.SSM_OK) == "ok"
-    for code in range(1, 5):
+    for code in range(1, 6):
         s = ssm.ssm_status_string(code)
         assert s and s != "unknown status"
     assert ssm.ssm_status_string(99) == "unknown status"
