@@ -107,9 +107,17 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
 }
 
 // Tile shape per padded state width: 32-token tiles; 32 channels per CTA (64 at N <= 4).
+#ifndef SSM_SCAN16_MINB
+#define SSM_SCAN16_MINB 4     // resident CTAs per SM the 16-state kernel's registers target
+#endif
+#ifndef SSM_SCAN16_NSTAGE
+#define SSM_SCAN16_NSTAGE 3   // cp.async ring depth of the 16-state kernel
+#endif
+
 template <int NP, typename Tin, typename Tout, bool VEC>
 int dispatch_cfg(const ssm::ScanArgs &a, cudaStream_t s) {
-    if constexpr (NP == 16) return run_scan<ssm::ScanCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>>(a, s);
+    if constexpr (NP == 16)
+        return run_scan<ssm::ScanCfg<16, 1, 32, SSM_SCAN16_NSTAGE, Tin, Tout, VEC, SSM_SCAN16_MINB>>(a, s);
     else if constexpr (NP == 8) return run_scan<ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>>(a, s);
     else return run_scan<ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>>(a, s);
 }
@@ -229,7 +237,8 @@ int run_scan_noalloc(const ssm::ScanArgs &a0, cudaStream_t stream) {
 
 template <int NP, typename Tin, typename Tout, bool VEC>
 int dispatch_cfg_noalloc(const ssm::ScanArgs &a, cudaStream_t s) {
-    if constexpr (NP == 16) return run_scan_noalloc<ssm::ScanCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>>(a, s);
+    if constexpr (NP == 16)
+        return run_scan_noalloc<ssm::ScanCfg<16, 1, 32, SSM_SCAN16_NSTAGE, Tin, Tout, VEC, SSM_SCAN16_MINB>>(a, s);
     else if constexpr (NP == 8) return run_scan_noalloc<ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>>(a, s);
     else return run_scan_noalloc<ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>>(a, s);
 }
