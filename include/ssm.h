@@ -81,6 +81,26 @@ int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_
                            int in_dtype, int out_dtype, void *cuda_stream);
 
 /*
+ * ssm_selective_scan_fwd with two options (ssm_selective_scan_fwd passes NULL and 0):
+ *   initial_state : [batch][dim][dstate] fp32, or NULL.  The scan starts from this state
+ *                   instead of zero, e.g. to continue a sequence whose earlier tokens
+ *                   were scanned by a previous call (its final_state).  With seqlen == 0
+ *                   the final state is a copy of it.
+ *   zoh_exact     : nonzero -> exact zero-order-hold input gain
+ *                   Bbar = (exp(Delta a) - 1) / a * B (the limit Delta * B where a == 0)
+ *                   instead of the Euler gain Delta * B ("Module 19: State-Space Models
+ *                   (Mamba)", learnllm, "The Math: The State-Space Recurrence"; the
+ *                   understandingdata page's ZOH numbers use this gain).
+ * All other arguments, layouts and errors as ssm_selective_scan_fwd.
+ */
+int ssm_selective_scan_fwd_ex(const void *x, const void *delta, const float *delta_bias,
+                              int delta_softplus, const float *A, const void *B, const void *C,
+                              const float *D, const void *z, void *y, float *final_state,
+                              const float *initial_state, int zoh_exact,
+                              int batch, int dim, int seqlen, int dstate,
+                              int in_dtype, int out_dtype, void *cuda_stream);
+
+/*
  * Allocation-free variant of ssm_selective_scan_fwd: same arguments, same results, and no
  * memory allocation of any kind (no cudaMalloc, cudaMallocAsync or cudaFree).  The pages
  * have no counterpart to this call; it exists for callers that are not allowed to

@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     load_library,
     selective_scan,
     ssm_selective_scan_fwd,
+    ssm_selective_scan_fwd_ex,
     ssm_selective_scan_fwd_noalloc,
     ssm_state_step,
     ssm_status_string,

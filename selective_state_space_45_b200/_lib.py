@@ -46,6 +46,9 @@ def load_library(path: str | None = None):
         lib.ssm_selective_scan_fwd.restype = i
         lib.ssm_selective_scan_fwd.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp,
                                                i, i, i, i, i, i, vp]
+        lib.ssm_selective_scan_fwd_ex.restype = i
+        lib.ssm_selective_scan_fwd_ex.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, vp, i,
+                                                  i, i, i, i, i, i, vp]
         lib.ssm_selective_scan_fwd_noalloc.restype = i
         lib.ssm_selective_scan_fwd_noalloc.argtypes = list(lib.ssm_selective_scan_fwd.argtypes)
         lib.ssm_state_step.restype = i
@@ -103,6 +106,19 @@ def ssm_selective_scan_fwd(x, delta, delta_bias, delta_softplus, A, B, C, D, z, 
         _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, x, y)))
 
 
+def ssm_selective_scan_fwd_ex(x, delta, delta_bias, delta_softplus, A, B, C, D, z, y, final_state,
+                              initial_state=None, zoh_exact=False, stream=None):
+    """``ssm_selective_scan_fwd`` with a start state and the exact zero-order-hold gain
+    (see include/ssm.h); initial_state is [batch, dim, N] fp32 or None."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    _check(load_library().ssm_selective_scan_fwd_ex(
+        _ptr(x), _ptr(delta), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(A), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), _ptr(y), _ptr(final_state), _ptr(initial_state),
+        int(bool(zoh_exact)), batch, dim, L, N, _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype],
+        _stream(stream, x, y)))
+
+
 def ssm_selective_scan_fwd_noalloc(x, delta, delta_bias, delta_softplus, A, B, C, D, z, y,
                                    final_state, stream=None):
     """Allocation-free variant of ``ssm_selective_scan_fwd`` (see include/ssm.h): same
@@ -125,11 +141,13 @@ def ssm_state_step(state, x, delta, A, B, C, D, z, y, stream=None):
 
 
 def selective_scan(x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
-                   out_dtype=None, return_final_state=True, stream=None):
-    """Allocate y (and the final state) with torch and run ``ssm_selective_scan_fwd``."""
+                   out_dtype=None, return_final_state=True, initial_state=None, zoh_exact=False,
+                   stream=None):
+    """Allocate y (and the final state) with torch and run the scan."""
     batch, dim, L = x.shape
     y = torch.empty((batch, dim, L), device=x.device, dtype=out_dtype or x.dtype)
     fs = (torch.empty((batch, dim, A.shape[1]), device=x.device, dtype=torch.float32)
           if return_final_state else None)
-    ssm_selective_scan_fwd(x, delta, delta_bias, delta_softplus, A, B, C, D, z, y, fs, stream)
+    ssm_selective_scan_fwd_ex(x, delta, delta_bias, delta_softplus, A, B, C, D, z, y, fs,
+                              initial_state, zoh_exact, stream)
     return (y, fs) if return_final_state else y

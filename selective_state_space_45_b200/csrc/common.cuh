@@ -47,6 +47,17 @@ __device__ __forceinline__ float softplus_f(float v) {
     return fmaxf(v, 0.f) + log1p_unit(ex2_approx(-fabsf(v) * kLog2e));
 }
 
+// expm1(v) for |v| < 0.1 from its Taylor series through v^5 (truncation below 1.4e-8
+// relative): near 0, exp(v) - 1 computed from exp(v) would lose the leading digits.
+__device__ __forceinline__ float expm1_small(float v) {
+    float p = 1.f / 120.f;
+    p = fmaf(p, v, 1.f / 24.f);
+    p = fmaf(p, v, 1.f / 6.f);
+    p = fmaf(p, v, 0.5f);
+    p = fmaf(p, v, 1.f);
+    return v * p;
+}
+
 // SiLU(z) = z * sigmoid(z) = z / (1 + e^-z).
 __device__ __forceinline__ float silu_f(float z) {
     return z * rcp_approx(1.f + ex2_approx(-z * kLog2e));

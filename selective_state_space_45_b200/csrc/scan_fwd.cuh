@@ -55,6 +55,7 @@ struct ScanArgs {
     float *final_state;
     int batch, dim, seqlen, dstate;
     int softplus;
+    int zoh;              // host side: exact zero-order-hold gain requested
     int groups_per_seq;   // ceil(dim / CH)
     // segmented scan (long sequences): pass 0 = whole sequence in one CTA,
     // 1 = segments from a zero state, 2 = carry correction of segments 1..nseg-1
@@ -63,6 +64,7 @@ struct ScanArgs {
     int seg_len;          // tokens per segment, a multiple of the tile
     float *seg_h;         // [batch*dim][nseg][NP] end states of pass 1
     float *seg_s;         // [batch*dim][nseg] step sums of pass 1
+    const float *h0;      // [batch][dim][dstate] start state, or null for zero
 };
 
 template <int NP_, int CG_, int T_, int NSTAGE_, typename Tin_, typename Tout_, bool VEC_, int MINB_>
@@ -224,7 +226,9 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
 }
 
 
-template <class Cfg, bool SEG>
+// SEG: segment passes 1/2 (else pass 0, the whole sequence).  ZOH: exact zero-order-hold
+// input gain (exp(Delta a) - 1) / a * B instead of the Euler gain Delta * B.
+template <class Cfg, bool SEG, bool ZOH>
 __global__ void __launch_bounds__(Cfg::NTHREADS, Cfg::MINB)
 scan_fwd_kernel(const ScanArgs p) {
     using Tin = typename Cfg::Tin;
@@ -263,6 +267,15 @@ scan_fwd_kernel(const ScanArgs p) {
         const int n = 4 * q + s;
         A2[s] = (dvalid && n < N) ? p.A[size_t(d0 + c) * N + n] * kLog2e : 0.f;
     }
+    // exact ZOH: 1 / a per state (0 where a = 0, whose gain is the limit Delta)
+    float invA[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (ZOH) {
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const float a = A2[s] * (1.f / kLog2e);
+            invA[s] = a != 0.f ? 1.f / a : 0.f;
+        }
+    }
     // per chunk task: its channel is the same in every tile, so bias and D live in registers
     float tbias[Cfg::TASKS_PER_THREAD], tD[Cfg::TASKS_PER_THREAD];
 #pragma unroll
@@ -286,6 +299,13 @@ scan_fwd_kernel(const ScanArgs p) {
     }
 
     float h[4] = {0.f, 0.f, 0.f, 0.f};
+    if (p.h0 != nullptr && dvalid && (!SEG || (p.pass == 1 && seg == 0))) {
+        // a given start state enters the first token range (pass 2 folds it in through
+        // segment 0's end state)
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            if (4 * q + s < N) h[s] = p.h0[chrow * N + 4 * q + s];
+    }
     float hin[4] = {0.f, 0.f, 0.f, 0.f};   // carry into the segment (pass 2)
     float sdl = 0.f;                        // running sum of this lane's steps in the range
     if constexpr (SEG) {
@@ -349,7 +369,7 @@ scan_fwd_kernel(const ScanArgs p) {
                     float dl = dr[u] + bias;
                     if (p.softplus) dl = softplus_f(dl);
                     o[2 * u] = dl;
-                    o[2 * u + 1] = dl * xr[u];
+                    o[2 * u + 1] = ZOH ? xr[u] : dl * xr[u];
                 }
             } else {
                 const bool cok = cc < nch;
@@ -359,7 +379,7 @@ scan_fwd_kernel(const ScanArgs p) {
                     if (p.softplus) dl = softplus_f(dl);
                     const bool ok = cok && (t0 + 8 * t8 + u < L);   // past L / dim: no-op token
                     o[2 * u] = ok ? dl : 0.f;
-                    o[2 * u + 1] = ok ? dl * xr[u] : 0.f;
+                    o[2 * u + 1] = ok ? (ZOH ? xr[u] : dl * xr[u]) : 0.f;
                 }
             }
 #pragma unroll
@@ -400,7 +420,7 @@ scan_fwd_kernel(const ScanArgs p) {
             float *ypr = yp + (q * CH + c) * Cfg::YP_ROW;
             // decays a = exp(Delta*A) and writes w = Delta*x*B of the 4 tokens of group g
             auto decay_write = [&](int g, float (&a)[4][4], float (&w)[4][4]) {
-                const float4 d01 = pp[(2 * g) * CH];   // (Delta, Delta*x) of tokens 4g, 4g+1
+                const float4 d01 = pp[(2 * g) * CH];   // (Delta, Delta*x or x) of tokens 4g, 4g+1
                 const float4 d23 = pp[(2 * g + 1) * CH];
                 const float dl[4] = {d01.x, d01.z, d23.x, d23.z};
                 const float dx[4] = {d01.y, d01.w, d23.y, d23.w};
@@ -412,7 +432,14 @@ scan_fwd_kernel(const ScanArgs p) {
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
                         a[u][s] = ex2_approx(dl[u] * A2[s]);
-                        w[u][s] = dx[u] * bb[s];
+                        if constexpr (ZOH) {   // dx holds x here; gain = expm1(Delta a) / a
+                            const float v = dl[u] * A2[s] * (1.f / kLog2e);
+                            const float em1 = fabsf(v) < 0.1f ? expm1_small(v) : a[u][s] - 1.f;
+                            const float gain = invA[s] != 0.f ? em1 * invA[s] : dl[u];
+                            w[u][s] = gain * dx[u] * bb[s];
+                        } else {
+                            w[u][s] = dx[u] * bb[s];
+                        }
                     }
                 }
             };

@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/ssm.h"
 #include "scan_fwd.cuh"
@@ -51,17 +52,17 @@ long long resident_slots(Kernel kernel, int threads, size_t smem) {
     return (long long)sms * per_sm;
 }
 
-template <class Cfg, bool SEG>
+template <class Cfg, bool SEG, bool ZOH = false>
 int launch_scan_kernel(const ssm::ScanArgs &a, long long blocks, cudaStream_t stream) {
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
     if (blocks == 0) return SSM_OK;
-    ssm::scan_fwd_kernel<Cfg, SEG><<<unsigned(blocks), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(a);
+    ssm::scan_fwd_kernel<Cfg, SEG, ZOH><<<unsigned(blocks), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(a);
     return status_of(cudaGetLastError());
 }
 
 // One scan: a single pass when the sequence fits one CTA per channel group, else the two
 // segment passes with a stream-ordered scratch buffer of batch*dim*nseg*(NP+1) floats.
-template <class Cfg>
+template <class Cfg, bool ZOH>
 int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     ssm::ScanArgs a = a0;
     const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
@@ -70,13 +71,13 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     const long long cgroups = groups * a.batch;
     const size_t smem = Cfg::SMEM_BYTES;
     if (smem > 48 * 1024) {   // opt in to large shared memory for both kernel variants
-        if (cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, false, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, true, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(smem)) != cudaSuccess)
             return SSM_ERR_CUDA;
     }
-    const long long slots = resident_slots(ssm::scan_fwd_kernel<Cfg, true>, Cfg::NTHREADS, smem);
+    const long long slots = resident_slots(ssm::scan_fwd_kernel<Cfg, true, ZOH>, Cfg::NTHREADS, smem);
     int nseg = choose_segments(cgroups, a.seqlen, slots > 0 ? slots : 2 * cgroups);
     long long seg_len = (a.seqlen + nseg - 1) / nseg;
     seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
@@ -85,7 +86,7 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
         a.pass = 0;
         a.nseg = 1;
         a.seg_len = a.seqlen;
-        return launch_scan_kernel<Cfg, false>(a, cgroups, stream);
+        return launch_scan_kernel<Cfg, false, ZOH>(a, cgroups, stream);
     }
     const size_t rows = size_t(a.batch) * a.dim * nseg;
     const size_t bytes = rows * Cfg::NP * sizeof(float) + rows * sizeof(float);
@@ -96,10 +97,10 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     a.seg_h = static_cast<float *>(ws);
     a.seg_s = a.seg_h + rows * Cfg::NP;
     a.pass = 1;
-    int st = launch_scan_kernel<Cfg, true>(a, cgroups * nseg, stream);
+    int st = launch_scan_kernel<Cfg, true, ZOH>(a, cgroups * nseg, stream);
     if (st == SSM_OK) {
         a.pass = 2;
-        st = launch_scan_kernel<Cfg, true>(a, cgroups * (nseg - 1), stream);
+        st = launch_scan_kernel<Cfg, true, ZOH>(a, cgroups * (nseg - 1), stream);
     }
     const cudaError_t fe = cudaFreeAsync(ws, stream);
     if (st == SSM_OK && fe != cudaSuccess) st = SSM_ERR_CUDA;
@@ -116,10 +117,11 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
 
 template <int NP, typename Tin, typename Tout, bool VEC>
 int dispatch_cfg(const ssm::ScanArgs &a, cudaStream_t s) {
-    if constexpr (NP == 16)
-        return run_scan<ssm::ScanCfg<16, 1, 32, SSM_SCAN16_NSTAGE, Tin, Tout, VEC, SSM_SCAN16_MINB>>(a, s);
-    else if constexpr (NP == 8) return run_scan<ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>>(a, s);
-    else return run_scan<ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>>(a, s);
+    using C16 = ssm::ScanCfg<16, 1, 32, SSM_SCAN16_NSTAGE, Tin, Tout, VEC, SSM_SCAN16_MINB>;
+    using C8 = ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>;
+    using C4 = ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>;
+    using Cfg = std::conditional_t<NP == 16, C16, std::conditional_t<NP == 8, C8, C4>>;
+    return a.zoh ? run_scan<Cfg, true>(a, s) : run_scan<Cfg, false>(a, s);
 }
 
 template <typename Tin, typename Tout>
@@ -200,13 +202,13 @@ int run_scan_noalloc(const ssm::ScanArgs &a0, cudaStream_t stream) {
     const long long cgroups = groups * a.batch;
     const size_t smem = Cfg::SMEM_BYTES;
     if (smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(smem)) != cudaSuccess)
             return SSM_ERR_CUDA;
     }
-    const long long slots = resident_slots(ssm::scan_fwd_kernel<Cfg, true>, Cfg::NTHREADS, smem);
+    const long long slots = resident_slots(ssm::scan_fwd_kernel<Cfg, true, false>, Cfg::NTHREADS, smem);
     int nseg = choose_segments(cgroups, a.seqlen, slots > 0 ? slots : 2 * cgroups);
     long long seg_len = (a.seqlen + nseg - 1) / nseg;
     seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
@@ -275,27 +277,43 @@ int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_
                            const float *D, const void *z, void *y, float *final_state,
                            int batch, int dim, int seqlen, int dstate,
                            int in_dtype, int out_dtype, void *cuda_stream) {
+    return ssm_selective_scan_fwd_ex(x, delta, delta_bias, delta_softplus, A, B, C, D, z, y,
+                                     final_state, nullptr, 0, batch, dim, seqlen, dstate,
+                                     in_dtype, out_dtype, cuda_stream);
+}
+
+int ssm_selective_scan_fwd_ex(const void *x, const void *delta, const float *delta_bias,
+                              int delta_softplus, const float *A, const void *B, const void *C,
+                              const float *D, const void *z, void *y, float *final_state,
+                              const float *initial_state, int zoh_exact,
+                              int batch, int dim, int seqlen, int dstate,
+                              int in_dtype, int out_dtype, void *cuda_stream) {
     if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return SSM_ERR_INVALID_ARG;
     if (batch < 0 || dim < 0 || seqlen < 0 || dstate < 1) return SSM_ERR_INVALID_ARG;
     if (dstate > 16) return SSM_ERR_UNSUPPORTED;
     const long long channels = (long long)batch * dim;
     const bool work = channels > 0 && seqlen > 0;
     if (work && (!x || !delta || !A || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
-    const void *ptrs[] = {x, delta, delta_bias, A, B, C, D, z, y, final_state};
+    const void *ptrs[] = {x, delta, delta_bias, A, B, C, D, z, y, final_state, initial_state};
     for (const void *q : ptrs)
         if (q && !aligned16(q)) return SSM_ERR_ALIGNMENT;
     if (channels == 0) return SSM_OK;
     if (!work && !final_state) return SSM_OK;
 
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    if (!work)   // empty sequences: the final state is the zero start state
-        return status_of(cudaMemsetAsync(final_state, 0, size_t(channels) * dstate * sizeof(float), stream));
+    if (!work) {   // empty sequences: the final state is the start state
+        const size_t bytes = size_t(channels) * dstate * sizeof(float);
+        if (initial_state)
+            return status_of(cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, stream));
+        return status_of(cudaMemsetAsync(final_state, 0, bytes, stream));
+    }
 
     ssm::ScanArgs a{};
     a.x = x; a.delta = delta; a.delta_bias = delta_bias; a.A = A; a.B = B; a.C = C; a.D = D;
-    a.z = z; a.y = y; a.final_state = final_state;
+    a.z = z; a.y = y; a.final_state = final_state; a.h0 = initial_state;
     a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = dstate;
     a.softplus = delta_softplus ? 1 : 0;
+    a.zoh = zoh_exact ? 1 : 0;
 
     // 16-byte staging needs every row of x/delta/z/y and every sequence's B/C block to
     // start on a 16-byte boundary: seqlen a multiple of the 16-byte element count.

@@ -31,7 +31,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for expected in ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_noalloc", "ssm_state_step",
+    for expected in ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_scan_fwd_noalloc",
+                     "ssm_state_step",
                      "ssm_status_string", "ssm_version"):
         assert expected in names
 

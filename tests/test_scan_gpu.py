@@ -213,3 +213,61 @@ def test_long_sequence_default_segmentation(cuda_lib):
     yr, fr = run_oracle(inp)
     assert_parity(y, yr, torch.bfloat16, torch.float32, what="y")
     assert_parity(fs, fr, torch.bfloat16, torch.float32, what="final_state")
+
+
+def run_gpu_ex(ssm, inp, out_dtype, h0=None, zoh=False):
+    x = inp["x"]
+    y = torch.empty(x.shape, device=DEV, dtype=out_dtype)
+    fs = torch.empty(x.shape[0], x.shape[1], inp["A"].shape[1], device=DEV, dtype=torch.float32)
+    ssm.ssm_selective_scan_fwd_ex(x, inp["delta"], inp["delta_bias"], True, inp["A"], inp["B"],
+                                  inp["C"], inp["D"], inp["z"], y, fs, h0, zoh)
+    torch.cuda.synchronize()
+    return y, fs
+
+
+@pytest.mark.parametrize("batch,dim,L,N,din,dout", [
+    (2, 37, 1000, 16, torch.bfloat16, torch.bfloat16),
+    (3, 21, 331, 5, torch.float32, torch.float32),
+    (1, 40, 256, 8, torch.bfloat16, torch.float32),
+])
+@pytest.mark.parametrize("h0,zoh", [(True, False), (False, True), (True, True)],
+                         ids=["state", "zoh", "state+zoh"])
+def test_initial_state_and_exact_zoh(cuda_lib, split, batch, dim, L, N, din, dout, h0, zoh):
+    inp = inputs.make_scan_inputs(batch, dim, L, N, din, device=DEV, seed=batch + L + N + 7)
+    if zoh:
+        inp["A"][:, 0] = 0.0          # the a = 0 limit of the exact gain is Delta * B
+    state = (torch.randn(batch, dim, N, device=DEV, generator=torch.Generator(DEV).manual_seed(8))
+             if h0 else None)
+    y, fs = run_gpu_ex(cuda_lib, inp, dout, state, zoh)
+    yr, fr = oracle.scan(x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"],
+                         D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True,
+                         h0=None if state is None else state, zoh_exact=zoh)
+    assert_parity(y, yr, din, dout, what="y")
+    assert_parity(fs, fr, din, torch.float32, what="final_state")
+
+
+def test_continuation_equals_one_scan(cuda_lib):
+    """Scanning L tokens, then the next L tokens from the returned state, gives the same
+    outputs as one scan over 2L tokens (prefill continued across calls)."""
+    inp = inputs.make_scan_inputs(2, 48, 1024, 16, torch.float32, device=DEV, seed=41)
+    y_all, f_all = run_gpu_ex(cuda_lib, inp, torch.float32)
+    half = {k: (v[..., :512].contiguous() if k in ("x", "delta", "z") else
+                v[:, :512].contiguous() if k in ("B", "C") else v) for k, v in inp.items()}
+    rest = {k: (v[..., 512:].contiguous() if k in ("x", "delta", "z") else
+                v[:, 512:].contiguous() if k in ("B", "C") else v) for k, v in inp.items()}
+    y1, f1 = run_gpu_ex(cuda_lib, half, torch.float32)
+    y2, f2 = run_gpu_ex(cuda_lib, rest, torch.float32, h0=f1)
+    assert_parity(torch.cat([y1, y2], dim=-1), to64(y_all), torch.float32, what="y halves vs whole")
+    assert_parity(f2, to64(f_all), torch.float32, what="final state halves vs whole")
+
+
+def test_empty_sequence_returns_initial_state(cuda_lib):
+    h0 = torch.randn(2, 3, 16, device=DEV)
+    x = torch.empty(2, 3, 0, device=DEV)
+    y = torch.empty(2, 3, 0, device=DEV)
+    fs = torch.zeros(2, 3, 16, device=DEV)
+    Bm = torch.empty(2, 0, 16, device=DEV)
+    cuda_lib.ssm_selective_scan_fwd_ex(x, x, None, True, -torch.ones(3, 16, device=DEV), Bm, Bm,
+                                       None, None, y, fs, h0, False)
+    torch.cuda.synchronize()
+    assert torch.equal(fs, h0)
