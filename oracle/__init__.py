@@ -7,6 +7,8 @@ from .oracle import (  # noqa: F401
     affine_scan_hillis_steele,
     affine_scan_loop,
     build,
+    causal_conv1d,
+    conv1d_step,
     lti_conv,
     lti_kernel,
     scan,

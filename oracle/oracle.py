@@ -21,6 +21,9 @@ Functions and the passages they follow:
 ``scan_parallel_reference``   the whole selective scan routed through the Hillis-Steele
                               rounds over N-expanded pairs (tiny inputs only): an
                               implementation independent of the C loop.
+``causal_conv1d`` / ``conv1d_step``  the causal depthwise convolution with SiLU in front of
+                              the scan, and its one-token window form: learnllm "Module 19",
+                              "The Causal Convolution"; xmarva lesson 10, sections 4 and 7.
 ``lti_kernel`` / ``lti_conv`` the convolutional face of a time-invariant SSM,
                               K = (C Bbar, C Abar Bbar, C Abar^2 Bbar, ...), y = K * x:
                               learnllm "Two Faces: Recurrent = Convolutional".
@@ -64,6 +67,10 @@ def _load():
                                         p, p, i64, i64, i64, i64, ctypes.c_int]
             lib.oracle_step.restype = None
             lib.oracle_step.argtypes = [p, p, p, p, p, p, p, p, p, i64, i64, i64]
+            lib.oracle_causal_conv1d.restype = None
+            lib.oracle_causal_conv1d.argtypes = [p, p, p, p, ctypes.c_int, p, p, i64, i64, i64, i64]
+            lib.oracle_conv1d_step.restype = None
+            lib.oracle_conv1d_step.argtypes = [p, p, p, p, ctypes.c_int, p, i64, i64, i64]
             _lib = lib
     return _lib
 
@@ -137,6 +144,41 @@ def step(state, x, delta, A, B, C, D=None, z=None):
     _load().oracle_step(_ptr(st), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
                         _ptr(z), _ptr(y), batch, dim, N)
     return y, st
+
+
+def causal_conv1d(x, weight, bias=None, hist=None, silu=True):
+    """Causal depthwise convolution (+ bias, + SiLU) in fp64: returns ``(u, window)``.
+
+    x: [batch, dim, L]; weight: [dim, K]; bias: [dim]; hist: [batch, dim, K-1] (the K-1
+    inputs before x, oldest first; zeros if None).  window: the last K-1 inputs, [batch,
+    dim, K-1], for a decode step to continue from.
+    """
+    x = _f64(x)
+    batch, dim, L = x.shape
+    w = _f64(weight)
+    K = w.shape[1]
+    w = _f64(weight, (dim, K))
+    bias = _f64(bias, (dim,))
+    hist = _f64(hist, (batch, dim, K - 1))
+    u = np.empty((batch, dim, L))
+    win = np.empty((batch, dim, K - 1))
+    _load().oracle_causal_conv1d(_ptr(x), _ptr(w), _ptr(bias), _ptr(hist), int(bool(silu)),
+                                 _ptr(u), _ptr(win), batch, dim, L, K)
+    return u, win
+
+
+def conv1d_step(window, x, weight, bias=None, silu=True):
+    """One decode token of the convolution in fp64: returns ``(u, new_window)``.
+    window: [batch, dim, K-1]; x: [batch, dim]; weight: [dim, K]."""
+    win = _f64(window).copy()
+    batch, dim, km1 = win.shape
+    w = _f64(weight, (dim, km1 + 1))
+    x = _f64(x, (batch, dim))
+    bias = _f64(bias, (dim,))
+    u = np.empty((batch, dim))
+    _load().oracle_conv1d_step(_ptr(win), _ptr(x), _ptr(w), _ptr(bias), int(bool(silu)), _ptr(u),
+                               batch, dim, km1 + 1)
+    return u, win
 
 
 # ----------------------------------------------------------------------------------

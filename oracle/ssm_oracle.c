@@ -164,3 +164,68 @@ void oracle_step(double *state, const double *x, const double *delta, const doub
                                 z != NULL, z ? z[i] : 0.0, 0);
         }
 }
+
+/*
+ * Causal depthwise convolution of width K, optional bias and SiLU, per (sequence, channel):
+ *   u[b,d,t] = act( bias[d] + sum_{i=0..K-1} w[d,i] * xe[b,d,t-(K-1)+i] )
+ * where xe is the input preceded by K-1 history values (hist[b,d,0..K-2], oldest first;
+ * zeros when hist is NULL -- the left padding by K-1 of the learnllm lesson, section "The
+ * Causal Convolution", and of the xmarva lesson's conv1d(padding=k-1)[..., :L], section 4).
+ * act is SiLU when silu != 0 (both pages apply SiLU to the convolution output).
+ * hist_out[b,d,0..K-2] (optional) receives the last K-1 values of xe: the window a decode
+ * step continues from (xmarva lesson, section 7).
+ *   x, u: [batch][dim][seqlen]; w: [dim][K]; bias: [dim] or NULL; hist, hist_out: [batch][dim][K-1]
+ */
+void oracle_causal_conv1d(const double *x, const double *w, const double *bias, const double *hist,
+                          int silu, double *u, double *hist_out,
+                          int64_t batch, int64_t dim, int64_t seqlen, int64_t K)
+{
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t row = b * dim + d;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                double acc = bias ? bias[d] : 0.0;
+                for (int64_t i = 0; i < K; ++i) {
+                    const int64_t src = t - (K - 1) + i;       /* index into x; < 0 means history */
+                    double v;
+                    if (src >= 0)
+                        v = x[row * seqlen + src];
+                    else
+                        v = hist ? hist[row * (K - 1) + (K - 1) + src] : 0.0;
+                    acc += w[d * K + i] * v;
+                }
+                u[row * seqlen + t] = silu ? oracle_silu(acc) : acc;
+            }
+            if (hist_out)
+                for (int64_t j = 0; j < K - 1; ++j) {
+                    const int64_t src = seqlen - (K - 1) + j;
+                    hist_out[row * (K - 1) + j] =
+                        src >= 0 ? x[row * seqlen + src]
+                                 : (hist ? hist[row * (K - 1) + (K - 1) + src] : 0.0);
+                }
+        }
+}
+
+/*
+ * One decode token of the convolution: window[b,d,0..K-2] holds the previous K-1 inputs
+ * (oldest first); u = act(bias + sum_{i<K-1} w[i] window[i] + w[K-1] x); the window then
+ * drops its oldest value and appends x.   window: [batch][dim][K-1] in/out; x, u: [batch][dim].
+ */
+void oracle_conv1d_step(double *window, const double *x, const double *w, const double *bias,
+                        int silu, double *u, int64_t batch, int64_t dim, int64_t K)
+{
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t row = b * dim + d;
+            double *win = window + row * (K - 1);
+            double acc = bias ? bias[d] : 0.0;
+            for (int64_t i = 0; i < K - 1; ++i)
+                acc += w[d * K + i] * win[i];
+            acc += w[d * K + K - 1] * x[row];
+            u[row] = silu ? oracle_silu(acc) : acc;
+            for (int64_t i = 0; i + 1 < K - 1; ++i)
+                win[i] = win[i + 1];
+            if (K > 1)
+                win[K - 2] = x[row];
+        }
+}

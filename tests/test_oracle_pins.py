@@ -285,3 +285,109 @@ def test_empty_sequence_keeps_initial_state():
                         B=np.zeros((2, 0, 4)), C=np.zeros((2, 0, 4)))
     assert y.shape == (2, 3, 0)
     assert np.all(hN == 0.0)
+
+
+# ----------------------------------------------------------------------------------
+# the causal depthwise convolution in front of the scan (learnllm "Module 19", "The
+# Causal Convolution"; xmarva lesson 10, sections 4 and 7)
+# ----------------------------------------------------------------------------------
+
+def _conv_case(rng, batch, dim, L, K):
+    return (rng.normal(size=(batch, dim, L)), rng.normal(size=(dim, K)) * 0.5,
+            rng.normal(size=dim) * 0.1)
+
+
+@pytest.mark.parametrize("K", [1, 2, 4])
+def test_conv_impulse_returns_reversed_taps(K):
+    # output t reads x_{t-K+1..t} with tap i on x_{t-K+1+i}: a spike at t = 0 shows the
+    # taps last-first, then only the bias is left
+    w = np.arange(1, K + 1, dtype=np.float64).reshape(1, K) * 0.25
+    L = K + 3
+    x = np.zeros((1, 1, L))
+    x[0, 0, 0] = 1.0
+    u, _ = oracle.causal_conv1d(x, w, bias=np.array([0.125]), silu=False)
+    expect = np.full(L, 0.125)
+    expect[:K] += w[0, ::-1]
+    np.testing.assert_array_equal(u[0, 0], expect)
+
+
+def test_conv_first_token_sees_only_its_own_tap():
+    rng = np.random.default_rng(3)
+    x, w, b = _conv_case(rng, 2, 3, 6, 4)
+    u, _ = oracle.causal_conv1d(x, w, bias=b, silu=False)
+    np.testing.assert_allclose(u[..., 0], b[None, :] + w[None, :, 3] * x[..., 0], rtol=1e-15)
+
+
+def test_conv_equals_textbook_full_convolution_cropped():
+    rng = np.random.default_rng(5)
+    x, w, b = _conv_case(rng, 2, 5, 23, 4)
+    u, win = oracle.causal_conv1d(x, w, bias=b, silu=False)
+    for bi in range(2):
+        for d in range(5):
+            full = np.convolve(x[bi, d], w[d, ::-1])       # true convolution, length L + K - 1
+            np.testing.assert_allclose(u[bi, d], full[:23] + b[d], rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(win, x[..., -3:])
+
+
+def test_conv_equals_torch_grouped_conv1d_left_padded():
+    # the block's own formulation: nn.Conv1d(groups=d_inner, padding=k-1), cropped to L
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(9)
+    x, w, b = _conv_case(rng, 3, 6, 17, 4)
+    u, _ = oracle.causal_conv1d(x, w, bias=b, silu=True)
+    ref = torch.nn.functional.conv1d(torch.from_numpy(x), torch.from_numpy(w)[:, None, :],
+                                     torch.from_numpy(b), padding=3, groups=6)[..., :17]
+    ref = torch.nn.functional.silu(ref).numpy()
+    np.testing.assert_allclose(u, ref, rtol=1e-13, atol=1e-14)
+
+
+def test_conv_silu_closed_values():
+    # pre-activations 0, ln 3, -ln 3 through a single unit tap: SiLU v = v sigmoid(v)
+    v = np.array([0.0, math.log(3.0), -math.log(3.0)])
+    u, _ = oracle.causal_conv1d(v.reshape(1, 1, 3), np.array([[0.0, 1.0]]), silu=True)
+    np.testing.assert_allclose(u[0, 0], v * np.array([0.5, 0.75, 0.25]), rtol=1e-15, atol=0)
+
+
+def test_conv_is_causal_and_depthwise():
+    rng = np.random.default_rng(13)
+    x, w, b = _conv_case(rng, 2, 4, 30, 4)
+    u, _ = oracle.causal_conv1d(x, w, bias=b)
+    t0 = 11
+    x2 = x.copy()
+    x2[:, 1, t0] += 3.0
+    u2, _ = oracle.causal_conv1d(x2, w, bias=b)
+    assert np.array_equal(u2[..., :t0], u[..., :t0])           # nothing before the edit moves
+    assert np.array_equal(u2[:, [0, 2, 3]], u[:, [0, 2, 3]])   # other channels never mix in
+    assert not np.array_equal(u2[:, 1, t0:t0 + 4], u[:, 1, t0:t0 + 4])
+    assert np.array_equal(u2[:, 1, t0 + 4:], u[:, 1, t0 + 4:])  # the edit leaves after K taps
+
+
+@pytest.mark.parametrize("split", [0, 1, 2, 9, 20])
+def test_conv_resumes_from_carried_window(split):
+    rng = np.random.default_rng(17)
+    x, w, b = _conv_case(rng, 2, 3, 20, 4)
+    u, win = oracle.causal_conv1d(x, w, bias=b)
+    u1, w1 = oracle.causal_conv1d(x[..., :split], w, bias=b)
+    u2, w2 = oracle.causal_conv1d(x[..., split:], w, bias=b, hist=w1)
+    np.testing.assert_array_equal(np.concatenate([u1, u2], axis=-1), u)
+    np.testing.assert_array_equal(w2, win)
+
+
+def test_conv_decode_steps_chain_to_the_full_convolution():
+    rng = np.random.default_rng(19)
+    x, w, b = _conv_case(rng, 2, 5, 13, 4)
+    hist = rng.normal(size=(2, 5, 3))
+    u, win = oracle.causal_conv1d(x, w, bias=b, hist=hist)
+    state = hist
+    for t in range(13):
+        ut, state = oracle.conv1d_step(state, x[..., t], w, bias=b)
+        np.testing.assert_allclose(ut, u[..., t], rtol=1e-14, atol=1e-15)
+    np.testing.assert_array_equal(state, win)
+
+
+def test_conv_width_one_is_pointwise():
+    rng = np.random.default_rng(23)
+    x, w, b = _conv_case(rng, 1, 3, 5, 1)
+    u, win = oracle.causal_conv1d(x, w, bias=b, silu=False)
+    np.testing.assert_allclose(u, w[None, :, :1] * x + b[None, :, None], rtol=1e-15)
+    assert win.shape == (1, 3, 0)
