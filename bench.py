@@ -3,13 +3,16 @@
 
 One JSON line on rank 0.  A step is one pass of the whole hot path over one batch:
 for the scan workloads one ``ssm_selective_scan_fwd`` call (discretise, recurrence,
-readout, skip, gate, final state), for the decode workload one ``ssm_state_step`` call.
+readout, skip, gate, final state), for the decode workload one ``ssm_state_step`` call;
+the conv workloads time the causal convolution in front of the scan
+(``ssm_causal_conv1d_fwd`` with its final window, or one ``ssm_causal_conv1d_step``).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mamba130m]
   python bench.py --impl reference ...        # the fp64 CPU oracle, timed on host cores
 
 Workloads (selective_state_space_45_b200.inputs.CONFIGS): mamba130m (default: batch 8,
-L 2048, d_inner 1536, N 16, bf16 in/out, fp32 state), mamba2p8b, long1m, decode.
+L 2048, d_inner 1536, N 16, bf16 in/out, fp32 state), mamba2p8b, long1m, decode, and the
+convolution's conv130m, conv2p8b, convstep.
 Multi-GPU: every rank runs its own replica (channels are independent; the path has no
 exchange step), timing is the max over ranks, value counts all ranks' work.
 """
@@ -48,7 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba130m",
-                    choices=["mamba130m", "mamba2p8b", "long1m", "decode", "tiny"])
+                    choices=["mamba130m", "mamba2p8b", "long1m", "decode", "tiny",
+                             "conv130m", "conv2p8b", "convstep"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0,
@@ -194,6 +198,30 @@ def scan_counts(batch, dim, L, N, in_size, out_size):
                 tokch=batch * L * dim)
 
 
+def conv_counts(batch, dim, L, K, in_size, out_size):
+    streams = batch * dim * L * (in_size + out_size)              # x in; u out
+    params = dim * (K + 1) * 4                                     # taps and bias
+    window = batch * dim * (K - 1) * 4                             # final window out
+    return dict(bytes=streams + params + window, exps=batch * dim * L, tokch=batch * dim * L)
+
+
+def conv_step_counts(batch, dim, K, in_size, out_size):
+    window = 2 * batch * dim * (K - 1) * 4                         # read + write in place
+    streams = batch * dim * (in_size + out_size)                   # x in; u out
+    params = dim * (K + 1) * 4
+    return dict(bytes=window + streams + params, exps=batch * dim, tokch=batch * dim)
+
+
+def workload_kind(name):
+    if name == "decode":
+        return "decode"
+    if name == "convstep":
+        return "convstep"
+    if name.startswith("conv"):
+        return "conv"
+    return "scan"
+
+
 def step_counts(batch, dim, N, in_size, out_size):
     state = 2 * batch * dim * N * 4                                # read + write in place
     streams = batch * dim * (3 * in_size + out_size)               # x, delta, z in; y out
@@ -211,14 +239,18 @@ class Workload:
         from selective_state_space_45_b200 import inputs
         self.name, self.device = name, device
         self.cfg = dict(inputs.CONFIGS[name])
-        self.kind = "decode" if name == "decode" else "scan"
+        self.kind = workload_kind(name)
         c = self.cfg
         dt = c["dtype"]
         esz = torch.tensor([], dtype=dt).element_size()
         if self.kind == "scan":
             self.counts = scan_counts(c["batch"], c["dim"], c["seqlen"], c["dstate"], esz, esz)
-        else:
+        elif self.kind == "decode":
             self.counts = step_counts(c["batch"], c["dim"], c["dstate"], esz, esz)
+        elif self.kind == "conv":
+            self.counts = conv_counts(c["batch"], c["dim"], c["seqlen"], c["width"], esz, esz)
+        else:
+            self.counts = conv_step_counts(c["batch"], c["dim"], c["width"], esz, esz)
         per_set = self.counts["bytes"]
         self.nsets = max(1, min(4, -(-int(2.5 * L2_BYTES) // per_set)))
         self.sets = []
@@ -227,8 +259,12 @@ class Workload:
             if self.kind == "scan":
                 inp["y"] = torch.empty(inp["x"].shape, device=device, dtype=dt)
                 inp["fs"] = torch.empty(c["batch"], c["dim"], c["dstate"], device=device)
+            elif self.kind == "conv":
+                inp["u"] = torch.empty(inp["x"].shape, device=device, dtype=dt)
+                inp["fw"] = torch.empty(c["batch"], c["dim"], c["width"] - 1, device=device)
             else:
-                inp["y"] = torch.empty(c["batch"], c["dim"], device=device, dtype=dt)
+                inp["y" if self.kind == "decode" else "u"] = torch.empty(
+                    c["batch"], c["dim"], device=device, dtype=dt)
             self.sets.append(inp)
 
     def launch(self, i, stream=None):
@@ -237,13 +273,28 @@ class Workload:
         if self.kind == "scan":
             ssm.ssm_selective_scan_fwd(s["x"], s["delta"], s["delta_bias"], True, s["A"], s["B"],
                                        s["C"], s["D"], s["z"], s["y"], s["fs"], stream)
-        else:
+        elif self.kind == "decode":
             t = (i // self.nsets) % s["x"].shape[0]
             ssm.ssm_state_step(s["state"], s["x"][t], s["delta"][t], s["A"], s["B"][t], s["C"][t],
                                s["D"], s["z"][t], s["y"], stream)
+        elif self.kind == "conv":
+            ssm.ssm_causal_conv1d_fwd(s["x"], s["weight"], s["bias"], None, s["u"], s["fw"], True,
+                                      stream)
+        else:
+            t = (i // self.nsets) % s["x"].shape[0]
+            ssm.ssm_causal_conv1d_step(s["window"], s["x"][t], s["weight"], s["bias"], s["u"], True,
+                                       stream)
 
     def description(self):
         c = self.cfg
+        io = str(c["dtype"]).split(".")[-1]
+        if self.kind == "conv":
+            return ("%s-shaped causal depthwise conv1d + SiLU: batch %d, L %d, d_inner %d, width %d, "
+                    "%s x and u, fp32 taps/bias/final window" % (self.name[4:], c["batch"], c["seqlen"],
+                                                                 c["dim"], c["width"], io))
+        if self.kind == "convstep":
+            return ("decode conv1d step: batch %d, d_inner %d, width %d, fp32 window in place, one %s "
+                    "token per sequence" % (c["batch"], c["dim"], c["width"], io))
         if self.kind == "scan":
             return ("%s-shaped selective scan: batch %d, L %d, d_inner %d, N %d, %s x/delta/z/B/C "
                     "and y, fp32 A/D/bias/state" % (self.name, c["batch"], c["seqlen"], c["dim"],
@@ -253,7 +304,8 @@ class Workload:
 
 
 def kernel_name(kind):
-    return "scan_fwd_kernel" if kind == "scan" else "state_step_kernel"
+    return dict(scan="scan_fwd_kernel", decode="state_step_kernel", conv="causal_conv1d_vec_kernel",
+                convstep="conv1d_step_kernel")[kind]
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -271,6 +323,21 @@ def _oracle_sample(name, n_target_tokch, seed=0):
     import torch
     from selective_state_space_45_b200 import inputs
     c = inputs.CONFIGS[name]
+    kind = workload_kind(name)
+    if kind == "convstep":
+        k = int(max(1, min(c["dim"], n_target_tokch // c["batch"])))
+        inp = inputs.make_conv_step_inputs(c["batch"], k, 1, c["width"], c["dtype"], device="cpu",
+                                           seed=seed)
+        sample = dict(window=inp["window"], x=inp["x"][0], weight=inp["weight"], bias=inp["bias"])
+        return kind, sample, c["batch"] * k, "%d sequences x %d of %d channels, one token" % (
+            c["batch"], k, c["dim"])
+    if kind == "conv":
+        per_channel = c["batch"] * c["seqlen"]
+        k = int(max(1, min(c["dim"], n_target_tokch // per_channel)))
+        inp = inputs.make_conv_inputs(c["batch"], k, c["seqlen"], c["width"], c["dtype"], device="cpu",
+                                      seed=seed)
+        return kind, inp, per_channel * k, "%d sequences x %d of %d channels, all %d tokens" % (
+            c["batch"], k, c["dim"], c["seqlen"])
     if name == "decode":
         k = int(max(1, min(c["dim"], n_target_tokch // c["batch"])))
         inp = inputs.make_decode_inputs(c["batch"], k, c["dstate"], 1, c["dtype"], device="cpu",
@@ -298,6 +365,10 @@ def _oracle_call(kind, inp, threads):
     if kind == "scan":
         oracle.scan(x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], D=inp["D"],
                     z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True, nthreads=threads)
+    elif kind == "conv":
+        oracle.causal_conv1d(inp["x"], inp["weight"], bias=inp["bias"])
+    elif kind == "convstep":
+        oracle.conv1d_step(inp["window"], inp["x"], inp["weight"], bias=inp["bias"])
     else:
         oracle.step(inp["state"], inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
                     z=inp["z"])
@@ -357,12 +428,20 @@ def time_e2e(wl, steps, stream):
     import torch
     import selective_state_space_45_b200 as ssm
     dev = wl.sets[0]
-    names_in = (["x", "delta", "z", "B", "C", "A", "D", "delta_bias"] if wl.kind == "scan"
-                else ["state", "x", "delta", "z", "B", "C", "A", "D"])
-    names_out = ["y", "fs"] if wl.kind == "scan" else ["y", "state"]
+    # per-token inputs of the decode kinds are [steps, ...]: one token's slice travels
+    per_token = {"decode": ("x", "delta", "z", "B", "C"), "convstep": ("x",)}.get(wl.kind, ())
+    names_in, names_out = dict(
+        scan=(["x", "delta", "z", "B", "C", "A", "D", "delta_bias"], ["y", "fs"]),
+        decode=(["state", "x", "delta", "z", "B", "C", "A", "D"], ["y", "state"]),
+        conv=(["x", "weight", "bias"], ["u", "fw"]),
+        convstep=(["window", "x", "weight", "bias"], ["u", "window"]))[wl.kind]
+
+    def dev_view(n):
+        return dev[n][0] if n in per_token else dev[n]
+
     host = {}
     for n in names_in:
-        src = dev[n][0] if (wl.kind == "decode" and n in ("x", "delta", "z", "B", "C")) else dev[n]
+        src = dev_view(n)
         host[n] = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
         host[n].copy_(src)
     outs = {n: torch.empty(dev[n].shape, dtype=dev[n].dtype, pin_memory=True) for n in names_out}
@@ -371,14 +450,17 @@ def time_e2e(wl, steps, stream):
 
     def one():
         for n in names_in:
-            dst = dev[n][0] if (wl.kind == "decode" and n in ("x", "delta", "z", "B", "C")) else dev[n]
-            dst.copy_(host[n], non_blocking=True)
+            dev_view(n).copy_(host[n], non_blocking=True)
         if wl.kind == "scan":
             ssm.ssm_selective_scan_fwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"],
                                        dev["B"], dev["C"], dev["D"], dev["z"], dev["y"], dev["fs"])
-        else:
+        elif wl.kind == "decode":
             ssm.ssm_state_step(dev["state"], dev["x"][0], dev["delta"][0], dev["A"], dev["B"][0],
                                dev["C"][0], dev["D"], dev["z"][0], dev["y"])
+        elif wl.kind == "conv":
+            ssm.ssm_causal_conv1d_fwd(dev["x"], dev["weight"], dev["bias"], None, dev["u"], dev["fw"])
+        else:
+            ssm.ssm_causal_conv1d_step(dev["window"], dev["x"][0], dev["weight"], dev["bias"], dev["u"])
         for n in names_out:
             outs[n].copy_(dev[n], non_blocking=True)
 
@@ -470,11 +552,15 @@ def run_ours(args):
 
     if rank == 0:
         c = wl.cfg
-        config = dict(workload=wl.description(), batch=c["batch"], d_inner=c["dim"], dstate=c["dstate"],
+        config = dict(workload=wl.description(), batch=c["batch"], d_inner=c["dim"],
                       parallelism="replicas x%d" % world,
                       l2=("%d rotating input sets of %.0f MB (%.0f MB touched per cycle) > 126 MB L2"
                           % (wl.nsets, wl.counts["bytes"] / 1e6, wl.nsets * wl.counts["bytes"] / 1e6)))
-        if wl.kind == "scan":
+        if "dstate" in c:
+            config.update(dstate=c["dstate"])
+        if "width" in c:
+            config.update(width=c["width"])
+        if "seqlen" in c:
             config.update(seqlen=c["seqlen"], global_batch=c["batch"] * world)
         line = dict(metric=METRIC, value=total_units / sec, unit=UNIT, n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=1e3 * sec / args.steps, higher_is_better=True,

@@ -1,11 +1,13 @@
 /*
  * ssm.h -- C ABI of the B200 selective state-space scan library (libssm.so).
  *
- * Two operations:
+ * Operations:
  *   ssm_selective_scan_fwd  the selective scan (S6) over a whole sequence;
- *   ssm_state_step          one decode token on a carried state, updated in place.
+ *   ssm_state_step          one decode token on a carried state, updated in place;
+ *   ssm_causal_conv1d_fwd   the causal depthwise convolution + SiLU that feeds the scan;
+ *   ssm_causal_conv1d_step  its one-token form on a carried window, updated in place.
  *
- * Both compute, per sequence b and channel d, with an N-wide fp32 state h:
+ * The scan and the state step compute, per sequence b and channel d, with an N-wide fp32 state h:
  *     Delta_t = softplus(delta[b,d,t] + delta_bias[d])   (bias and softplus optional)
  *     h_n    <- exp(Delta_t * A[d,n]) * h_n + Delta_t * B[b,t,n] * x[b,d,t]
  *     y[b,d,t] = (sum_n C[b,t,n] * h_n + D[d] * x[b,d,t]) * SiLU(z[b,d,t])
@@ -30,6 +32,8 @@
  *  - dtype codes: SSM_F32 (fp32) or SSM_BF16 (bf16).  A, D, delta_bias and the state
  *    are always fp32; the state arithmetic is fp32 whatever the input dtype.
  *  - dstate (N) must be in 1..16 (SSM_ERR_UNSUPPORTED above 16).
+ *  - Output buffers must not overlap input buffers (the convolution checks and returns
+ *    SSM_ERR_INVALID_ARG; for the scan the result of an overlap is undefined).
  */
 #ifndef SSM_H_
 #define SSM_H_
@@ -46,7 +50,7 @@ typedef enum {
 typedef enum {
     SSM_OK = 0,
     SSM_ERR_INVALID_ARG = 1,   /* null required pointer, negative size, bad dtype code   */
-    SSM_ERR_UNSUPPORTED = 2,   /* dstate outside 1..16, sizes beyond the int32 index range */
+    SSM_ERR_UNSUPPORTED = 2,   /* dstate above 16, conv width above 8, sizes out of range */
     SSM_ERR_ALIGNMENT = 3,     /* a pointer not 16-byte aligned                            */
     SSM_ERR_CUDA = 4,          /* the CUDA runtime reported an error at launch             */
     SSM_ERR_SCRATCH = 5        /* ssm_selective_scan_fwd_noalloc: fixed scratch too small  */
@@ -147,6 +151,48 @@ int ssm_state_step(float *state, const void *x, const void *delta, const float *
                    const void *B, const void *C, const float *D, const void *z, void *y,
                    int batch, int dim, int dstate, int in_dtype, int out_dtype,
                    void *cuda_stream);
+
+/*
+ * Causal depthwise convolution, bias and SiLU over whole sequences (the filter in front of
+ * the scan: "Module 19: State-Space Models (Mamba)", learnllm, section "The Causal
+ * Convolution"; xmarva lesson 10, section 4 "The Mamba block").  Per sequence b, channel d
+ * and position t, with K = width and xe the input preceded by the K-1 window values:
+ *     u[b,d,t] = act( bias[d] + sum_{i<K} weight[d,i] * xe[b,d,t-K+1+i] )
+ * act = SiLU when silu != 0, else the identity.  Output t never reads a later input.
+ *
+ *   x, u           : [batch][dim][seqlen], in_dtype / out_dtype (u written).
+ *   weight         : [dim][width] fp32, tap i multiplies the input K-1-i steps back.
+ *   bias           : [dim] fp32 or NULL (zero).
+ *   initial_window : [batch][dim][width-1] fp32 or NULL: the width-1 inputs before
+ *                    position 0, oldest first (NULL = zeros, the left pad).
+ *   final_window   : [batch][dim][width-1] fp32 or NULL: receives the last width-1
+ *                    inputs (window included when seqlen < width-1), the window that
+ *                    ssm_causal_conv1d_step continues from.
+ * width must be 1..8 (SSM_ERR_UNSUPPORTED above 8).  Widths 1..4 with seqlen a multiple
+ * of 8 (bf16 input) or 4 (fp32 input) take the vectorised kernel; others a per-element
+ * kernel with the same results.  u may not overlap x; final_window may not overlap
+ * initial_window, x or u (SSM_ERR_INVALID_ARG).  seqlen = 0 copies the window through.
+ */
+int ssm_causal_conv1d_fwd(const void *x, const float *weight, const float *bias,
+                          const float *initial_window, void *u, float *final_window,
+                          int batch, int dim, int seqlen, int width, int silu,
+                          int in_dtype, int out_dtype, void *cuda_stream);
+
+/*
+ * One decode token of the convolution (xmarva lesson 10, section 7 "Generation with a
+ * state of fixed size": the block keeps the last inputs of its convolution next to h).
+ *
+ *   window : [batch][dim][width-1] fp32, the previous width-1 inputs, oldest first; read,
+ *            then overwritten with the window shifted by one and x appended.  May be NULL
+ *            when width = 1.
+ *   x, u   : [batch][dim], in_dtype / out_dtype (u written).
+ *   weight, bias, silu, width: as for ssm_causal_conv1d_fwd.
+ * Chaining L calls from a window gives the same u and window as ssm_causal_conv1d_fwd
+ * over those L tokens with that initial_window.  window may not overlap x or u.
+ */
+int ssm_causal_conv1d_step(float *window, const void *x, const float *weight, const float *bias,
+                           void *u, int batch, int dim, int width, int silu,
+                           int in_dtype, int out_dtype, void *cuda_stream);
 
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char *ssm_status_string(int status);

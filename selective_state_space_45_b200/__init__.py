@@ -1,4 +1,5 @@
-"""B200 (sm_100a) selective state-space scan (S6): forward scan and decode step.
+"""B200 (sm_100a) selective state-space scan (S6): forward scan and decode step, and the
+causal depthwise convolution in front of it.
 
 The computation lives in ``libssm.so`` (C ABI in ``include/ssm.h``); this package only
 loads it and marshals torch tensors into it.
@@ -14,8 +15,11 @@ from ._lib import (  # noqa: F401
     SSM_F32,
     SSM_OK,
     SsmError,
+    causal_conv1d,
     load_library,
     selective_scan,
+    ssm_causal_conv1d_fwd,
+    ssm_causal_conv1d_step,
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_ex,
     ssm_selective_scan_fwd_noalloc,

@@ -53,6 +53,10 @@ def load_library(path: str | None = None):
         lib.ssm_selective_scan_fwd_noalloc.argtypes = list(lib.ssm_selective_scan_fwd.argtypes)
         lib.ssm_state_step.restype = i
         lib.ssm_state_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+        lib.ssm_causal_conv1d_fwd.restype = i
+        lib.ssm_causal_conv1d_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+        lib.ssm_causal_conv1d_step.restype = i
+        lib.ssm_causal_conv1d_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
         lib.ssm_status_string.restype = ctypes.c_char_p
         lib.ssm_status_string.argtypes = [i]
         lib.ssm_version.restype = i
@@ -138,6 +142,40 @@ def ssm_state_step(state, x, delta, A, B, C, D, z, y, stream=None):
     _check(load_library().ssm_state_step(
         _ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(y),
         batch, dim, N, _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, state, y)))
+
+
+def ssm_causal_conv1d_fwd(x, weight, bias, initial_window, u, final_window, silu=True,
+                          stream=None):
+    """Causal depthwise convolution + bias + SiLU (see include/ssm.h): x, u [batch, dim, L];
+    weight [dim, width] fp32; bias [dim] fp32 or None; initial_window / final_window
+    [batch, dim, width-1] fp32 or None.  Writes u (and final_window) in place."""
+    batch, dim, L = x.shape
+    width = weight.shape[1]
+    _check(load_library().ssm_causal_conv1d_fwd(
+        _ptr(x), _ptr(weight), _ptr(bias), _ptr(initial_window), _ptr(u), _ptr(final_window),
+        batch, dim, L, width, int(bool(silu)), _DTYPE_CODE[x.dtype], _DTYPE_CODE[u.dtype],
+        _stream(stream, x, u)))
+
+
+def ssm_causal_conv1d_step(window, x, weight, bias, u, silu=True, stream=None):
+    """One decode token of the convolution (see include/ssm.h): window [batch, dim, width-1]
+    fp32 updated in place (may be None for width 1); x, u [batch, dim]."""
+    batch, dim = x.shape
+    width = weight.shape[1]
+    _check(load_library().ssm_causal_conv1d_step(
+        _ptr(window), _ptr(x), _ptr(weight), _ptr(bias), _ptr(u), batch, dim, width,
+        int(bool(silu)), _DTYPE_CODE[x.dtype], _DTYPE_CODE[u.dtype], _stream(stream, x, u)))
+
+
+def causal_conv1d(x, weight, bias=None, initial_window=None, silu=True, out_dtype=None,
+                  return_final_window=False, stream=None):
+    """Allocate u (and the final window) with torch and run the convolution."""
+    batch, dim, L = x.shape
+    u = torch.empty((batch, dim, L), device=x.device, dtype=out_dtype or x.dtype)
+    fw = (torch.empty((batch, dim, weight.shape[1] - 1), device=x.device, dtype=torch.float32)
+          if return_final_window else None)
+    ssm_causal_conv1d_fwd(x, weight, bias, initial_window, u, fw, silu, stream)
+    return (u, fw) if return_final_window else u
 
 
 def selective_scan(x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,

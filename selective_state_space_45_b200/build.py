@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libssm.so")
 SOURCES = [os.path.join(CSRC, "ssm_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("common.cuh", "scan_fwd.cuh", "state_step.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("common.cuh", "conv1d.cuh", "scan_fwd.cuh", "state_step.cuh")] + [
     os.path.join(ROOT, "include", "ssm.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -11,6 +11,7 @@
 #include <type_traits>
 
 #include "../../include/ssm.h"
+#include "conv1d.cuh"
 #include "scan_fwd.cuh"
 #include "state_step.cuh"
 
@@ -23,6 +24,15 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool valid_dtype(int t) { return t == SSM_F32 || t == SSM_BF16; }
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA; }
+
+size_t dtype_size(int t) { return t == SSM_F32 ? 4 : 2; }
+
+// Do the byte ranges [p, p + pb) and [q, q + qb) share a byte?
+bool overlaps(const void *p, size_t pb, const void *q, size_t qb) {
+    if (!p || !q || pb == 0 || qb == 0) return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return a < b + qb && b < a + pb;
+}
 
 constexpr int kMinSegTokens = 4096;     // shortest segment worth a carry correction
 
@@ -159,6 +169,45 @@ int launch_step(const ssm::StepArgs &a, cudaStream_t s) {
     return launch_step_np<16, Tin, Tout>(a, s);
 }
 
+
+template <typename Tin, typename Tout, int K>
+int launch_conv_vec(const ssm::ConvArgs &a, cudaStream_t s) {
+    constexpr int CH = 2 * ssm::Vec16<Tin>::kN;
+    const long long nchunk = (a.seqlen + CH - 1) / CH;
+    const long long total = a.rows * nchunk;
+    const long long blocks = std::min<long long>((total + 255) / 256, INT_MAX);
+    ssm::causal_conv1d_vec_kernel<Tin, Tout, K>
+        <<<static_cast<unsigned>(blocks), 256, 0, s>>>(a, nchunk, total);
+    return status_of(cudaGetLastError());
+}
+
+template <typename Tin, typename Tout>
+int launch_conv(const ssm::ConvArgs &a, cudaStream_t s) {
+    // the vector path needs every row to start on a 16-byte vector of inputs
+    if (a.seqlen % ssm::Vec16<Tin>::kN == 0) {
+        switch (a.K) {
+            case 1: return launch_conv_vec<Tin, Tout, 1>(a, s);
+            case 2: return launch_conv_vec<Tin, Tout, 2>(a, s);
+            case 3: return launch_conv_vec<Tin, Tout, 3>(a, s);
+            case 4: return launch_conv_vec<Tin, Tout, 4>(a, s);
+            default: break;
+        }
+    }
+    const long long total = a.rows * a.seqlen;
+    const long long blocks = std::min<long long>((total + 255) / 256, INT_MAX);
+    ssm::causal_conv1d_any_kernel<Tin, Tout><<<static_cast<unsigned>(blocks), 256, 0, s>>>(a);
+    return status_of(cudaGetLastError());
+}
+
+template <typename Tin, typename Tout>
+int launch_conv_step(float *window, const void *x, const float *w, const float *bias, void *u,
+                     long long rows, int dim, int K, int silu, cudaStream_t s) {
+    const long long blocks = (rows + 255) / 256;
+    if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    ssm::conv1d_step_kernel<Tin, Tout><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        window, static_cast<const Tin *>(x), w, bias, static_cast<Tout *>(u), rows, dim, K, silu);
+    return status_of(cudaGetLastError());
+}
 
 // ---------------------------------------------------------------------------------
 // Allocation-free variant (ssm_selective_scan_fwd_noalloc).  The segment aggregates of
@@ -388,6 +437,75 @@ int ssm_state_step(float *state, const void *x, const void *delta, const float *
         return launch_step<__nv_bfloat16, __nv_bfloat16>(a, stream);
     if (in_dtype == SSM_BF16) return launch_step<__nv_bfloat16, float>(a, stream);
     return launch_step<float, __nv_bfloat16>(a, stream);
+}
+
+int ssm_causal_conv1d_fwd(const void *x, const float *weight, const float *bias,
+                          const float *initial_window, void *u, float *final_window,
+                          int batch, int dim, int seqlen, int width, int silu,
+                          int in_dtype, int out_dtype, void *cuda_stream) {
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return SSM_ERR_INVALID_ARG;
+    if (batch < 0 || dim < 0 || seqlen < 0 || width < 1) return SSM_ERR_INVALID_ARG;
+    if (width > ssm::kMaxConvWidth) return SSM_ERR_UNSUPPORTED;
+    const long long rows = (long long)batch * dim;
+    const int H = width - 1;
+    const bool work = rows > 0 && seqlen > 0;
+    if (work && (!x || !weight || !u)) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, weight, bias, initial_window, u, final_window};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSM_ERR_ALIGNMENT;
+    const size_t xb = size_t(rows) * seqlen * dtype_size(in_dtype);
+    const size_t ub = size_t(rows) * seqlen * dtype_size(out_dtype);
+    const size_t wb = size_t(rows) * H * sizeof(float);
+    if (overlaps(u, ub, x, xb) || overlaps(final_window, wb, initial_window, wb) ||
+        overlaps(final_window, wb, x, xb) || overlaps(final_window, wb, u, ub))
+        return SSM_ERR_INVALID_ARG;
+    if (rows == 0) return SSM_OK;
+
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (!work) {   // empty sequences: the window is the one carried in
+        if (!final_window || H == 0) return SSM_OK;
+        if (initial_window)
+            return status_of(cudaMemcpyAsync(final_window, initial_window, wb, cudaMemcpyDeviceToDevice, stream));
+        return status_of(cudaMemsetAsync(final_window, 0, wb, stream));
+    }
+
+    ssm::ConvArgs a{};
+    a.x = x; a.w = weight; a.bias = bias; a.hist = initial_window; a.u = u;
+    a.hist_out = final_window; a.rows = rows; a.dim = dim; a.seqlen = seqlen; a.K = width;
+    a.silu = silu ? 1 : 0;
+    if (in_dtype == SSM_F32 && out_dtype == SSM_F32) return launch_conv<float, float>(a, stream);
+    if (in_dtype == SSM_BF16 && out_dtype == SSM_BF16)
+        return launch_conv<__nv_bfloat16, __nv_bfloat16>(a, stream);
+    if (in_dtype == SSM_BF16) return launch_conv<__nv_bfloat16, float>(a, stream);
+    return launch_conv<float, __nv_bfloat16>(a, stream);
+}
+
+int ssm_causal_conv1d_step(float *window, const void *x, const float *weight, const float *bias,
+                           void *u, int batch, int dim, int width, int silu,
+                           int in_dtype, int out_dtype, void *cuda_stream) {
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return SSM_ERR_INVALID_ARG;
+    if (batch < 0 || dim < 0 || width < 1) return SSM_ERR_INVALID_ARG;
+    if (width > ssm::kMaxConvWidth) return SSM_ERR_UNSUPPORTED;
+    const long long rows = (long long)batch * dim;
+    const int H = width - 1;
+    if (rows > 0 && (!x || !weight || !u || (H > 0 && !window))) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {window, x, weight, bias, u};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSM_ERR_ALIGNMENT;
+    const size_t wb = size_t(rows) * H * sizeof(float);
+    if (overlaps(window, wb, x, size_t(rows) * dtype_size(in_dtype)) ||
+        overlaps(window, wb, u, size_t(rows) * dtype_size(out_dtype)))
+        return SSM_ERR_INVALID_ARG;
+    if (rows == 0) return SSM_OK;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    const int sf = silu ? 1 : 0;
+    if (in_dtype == SSM_F32 && out_dtype == SSM_F32)
+        return launch_conv_step<float, float>(window, x, weight, bias, u, rows, dim, width, sf, stream);
+    if (in_dtype == SSM_BF16 && out_dtype == SSM_BF16)
+        return launch_conv_step<__nv_bfloat16, __nv_bfloat16>(window, x, weight, bias, u, rows, dim, width, sf, stream);
+    if (in_dtype == SSM_BF16)
+        return launch_conv_step<__nv_bfloat16, float>(window, x, weight, bias, u, rows, dim, width, sf, stream);
+    return launch_conv_step<float, __nv_bfloat16>(window, x, weight, bias, u, rows, dim, width, sf, stream);
 }
 
 }  // extern "C"

@@ -1,4 +1,5 @@
-"""Seeded synthetic inputs for the selective scan and the decode step.
+"""Seeded synthetic inputs for the selective scan, the decode step and the causal
+convolution in front of the scan.
 
 This module only draws random numbers in the shapes and distributions of the
 workloads; it computes nothing of the scan itself, so the CUDA path and the fp64
@@ -17,6 +18,9 @@ mamba130m      8       2048       1536     16   bf16 (A, D, bias, state fp32)
 mamba2p8b      4       4096       5120     16   bf16
 long1m         1       1048576    1536     16   bf16
 decode         256     1 x 64     5120     16   bf16 tokens, fp32 state
+conv130m       8       2048       1536     --   bf16 x and u; width 4, fp32 taps/bias
+conv2p8b       4       4096       5120     --   bf16 x and u; width 4
+convstep       256     1 x 64     5120     --   bf16 tokens, fp32 window (width 4)
 =============  ======  =========  =======  ===  =====================================
 
 Draw order (one generator seeded once): x, delta_raw, z, B, C, D, dt.
@@ -44,6 +48,10 @@ CONFIGS = {
                    dt_dist="uniform"),
     "decode": dict(batch=256, steps=64, dim=5120, dstate=16, dtype=torch.bfloat16,
                    dt_dist="uniform"),
+    # the causal convolution in front of the scan, in the same block shapes (width 4)
+    "conv130m": dict(batch=8, seqlen=2048, dim=1536, width=4, dtype=torch.bfloat16),
+    "conv2p8b": dict(batch=4, seqlen=4096, dim=5120, width=4, dtype=torch.bfloat16),
+    "convstep": dict(batch=256, steps=64, dim=5120, width=4, dtype=torch.bfloat16),
 }
 
 DT_MIN, DT_MAX = 1e-3, 1e-1
@@ -95,6 +103,12 @@ def make_scan_inputs(batch, dim, seqlen, dstate, dtype=torch.float32, device="cp
 
 def make_config_inputs(name, device="cpu", seed=0):
     c = CONFIGS[name]
+    if name == "convstep":
+        return make_conv_step_inputs(c["batch"], c["dim"], c["steps"], c["width"], c["dtype"],
+                                     device=device, seed=seed)
+    if name.startswith("conv"):
+        return make_conv_inputs(c["batch"], c["dim"], c["seqlen"], c["width"], c["dtype"],
+                                device=device, seed=seed)
     if name == "decode":
         return make_decode_inputs(c["batch"], c["dim"], c["dstate"], c["steps"], c["dtype"],
                                   device=device, seed=seed)
@@ -123,3 +137,39 @@ def make_decode_inputs(batch, dim, dstate, steps, dtype=torch.bfloat16, device="
     delta = (dt[None, None, :] * torch.exp(0.5 * noise)).to(dtype)
     A = -torch.arange(1, dstate + 1, device=device, dtype=f32).repeat(dim, 1).contiguous()
     return dict(state=state, x=x, delta=delta, z=z, B=B, C=C, A=A, D=D)
+
+
+def make_conv_inputs(batch, dim, seqlen, width=4, dtype=torch.bfloat16, device="cpu", seed=0,
+                     with_window=False):
+    """Inputs of one causal-convolution call (the filter in front of the scan).
+
+    Keys: x ([batch, dim, seqlen], ``dtype``, N(0, 1)); weight ([dim, width] fp32) and bias
+    ([dim] fp32), both U(-1/sqrt(width), 1/sqrt(width)) -- the default initialisation of a
+    depthwise Conv1d, whose fan-in is the width; window ([batch, dim, width-1] fp32,
+    N(0, 1), the inputs before position 0) when ``with_window``.
+    Draw order: x, weight, bias, window.
+    """
+    g = _generator(device, seed)
+    f32 = torch.float32
+    bound = 1.0 / math.sqrt(width)
+    x = torch.randn(batch, dim, seqlen, generator=g, device=device, dtype=f32).to(dtype)
+    weight = (torch.rand(dim, width, generator=g, device=device, dtype=f32) * 2 - 1) * bound
+    bias = (torch.rand(dim, generator=g, device=device, dtype=f32) * 2 - 1) * bound
+    out = dict(x=x, weight=weight.contiguous(), bias=bias)
+    if with_window:
+        out["window"] = torch.randn(batch, dim, width - 1, generator=g, device=device, dtype=f32)
+    return out
+
+
+def make_conv_step_inputs(batch, dim, steps, width=4, dtype=torch.bfloat16, device="cpu", seed=0):
+    """Inputs of ``steps`` chained convolution decode calls: window ([batch, dim, width-1]
+    fp32, N(0, 1)); x ([steps, batch, dim], ``dtype``, N(0, 1)); weight, bias as in
+    ``make_conv_inputs``.  Draw order: window, x, weight, bias."""
+    g = _generator(device, seed)
+    f32 = torch.float32
+    bound = 1.0 / math.sqrt(width)
+    window = torch.randn(batch, dim, width - 1, generator=g, device=device, dtype=f32)
+    x = torch.randn(steps, batch, dim, generator=g, device=device, dtype=f32).to(dtype)
+    weight = (torch.rand(dim, width, generator=g, device=device, dtype=f32) * 2 - 1) * bound
+    bias = (torch.rand(dim, generator=g, device=device, dtype=f32) * 2 - 1) * bound
+    return dict(window=window, x=x, weight=weight.contiguous(), bias=bias)

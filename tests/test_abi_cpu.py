@@ -32,7 +32,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for expected in ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_scan_fwd_noalloc",
-                     "ssm_state_step",
+                     "ssm_state_step", "ssm_causal_conv1d_fwd", "ssm_causal_conv1d_step",
                      "ssm_status_string", "ssm_version"):
         assert expected in names
 
@@ -115,6 +115,71 @@ def test_scan_argument_checks(lib, kw, status):
 ])
 def test_step_argument_checks(lib, kw, status):
     assert step(lib, **kw) == status
+
+
+# distinct fake buffers, 1 MiB apart, for the calls that check overlaps
+X, U, W, BIAS, H0, H1 = (0x7F0000000000 + k * (1 << 20) for k in range(6))
+
+
+def conv(lib, **kw):
+    args = dict(x=X, w=W, bias=BIAS, h0=H0, u=U, h1=H1, batch=2, dim=3, L=8, K=4, silu=1,
+                din=ssm.SSM_BF16, dout=ssm.SSM_BF16)
+    args.update(kw)
+    return lib.ssm_causal_conv1d_fwd(args["x"], args["w"], args["bias"], args["h0"], args["u"],
+                                     args["h1"], args["batch"], args["dim"], args["L"], args["K"],
+                                     args["silu"], args["din"], args["dout"], None)
+
+
+def conv_step(lib, **kw):
+    args = dict(win=H0, x=X, w=W, bias=BIAS, u=U, batch=2, dim=3, K=4, silu=1,
+                din=ssm.SSM_BF16, dout=ssm.SSM_BF16)
+    args.update(kw)
+    return lib.ssm_causal_conv1d_step(args["win"], args["x"], args["w"], args["bias"], args["u"],
+                                      args["batch"], args["dim"], args["K"], args["silu"],
+                                      args["din"], args["dout"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(w=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(u=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(K=0), ssm.SSM_ERR_INVALID_ARG),
+    (dict(K=9), ssm.SSM_ERR_UNSUPPORTED),
+    (dict(L=-1), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dim=-1), ssm.SSM_ERR_INVALID_ARG),
+    (dict(din=3), ssm.SSM_ERR_INVALID_ARG),
+    (dict(x=X + 8), ssm.SSM_ERR_ALIGNMENT),
+    (dict(h1=H1 + 4), ssm.SSM_ERR_ALIGNMENT),
+    (dict(w=W + 4), ssm.SSM_ERR_ALIGNMENT),
+    # outputs overlapping inputs are refused: u over x, the new window over the old one
+    (dict(u=X), ssm.SSM_ERR_INVALID_ARG),
+    (dict(u=X + 16), ssm.SSM_ERR_INVALID_ARG),
+    (dict(h1=H0), ssm.SSM_ERR_INVALID_ARG),
+    (dict(h1=U + 32), ssm.SSM_ERR_INVALID_ARG),
+    (dict(h1=X), ssm.SSM_ERR_INVALID_ARG),
+    # x holds 2*3*8 bf16 = 96 bytes: a u that starts in its last 16 overlaps it
+    (dict(u=X + 80), ssm.SSM_ERR_INVALID_ARG),
+    (dict(batch=0), ssm.SSM_OK),
+    (dict(dim=0, x=None, u=None, w=None), ssm.SSM_OK),
+])
+def test_conv_argument_checks(lib, kw, status):
+    assert conv(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(win=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(x=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(u=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(w=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(K=0), ssm.SSM_ERR_INVALID_ARG),
+    (dict(K=9), ssm.SSM_ERR_UNSUPPORTED),
+    (dict(win=H0 + 4), ssm.SSM_ERR_ALIGNMENT),
+    (dict(win=X), ssm.SSM_ERR_INVALID_ARG),
+    (dict(u=H0), ssm.SSM_ERR_INVALID_ARG),
+    (dict(batch=0), ssm.SSM_OK),
+])
+def test_conv_step_argument_checks(lib, kw, status):
+    assert conv_step(lib, **kw) == status
 
 
 def test_python_binding_raises_on_error(lib):

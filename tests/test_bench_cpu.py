@@ -92,3 +92,28 @@ def test_dist_env_defaults(world, monkeypatch):
     for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
         monkeypatch.delenv(k, raising=False)
     assert bench.dist_env() == (0, 1, 0)
+
+
+def test_conv_counts_mamba130m():
+    c = bench.conv_counts(8, 1536, 2048, 4, 2, 2)
+    assert c["tokch"] == 8 * 1536 * 2048
+    # x in, u out (2 B each) + taps and bias + the final window (3 fp32 per row)
+    assert c["bytes"] == 8 * 1536 * 2048 * 4 + 1536 * 5 * 4 + 8 * 1536 * 3 * 4
+    assert abs(c["bytes"] / 1e6 - 100.8) < 0.1
+
+
+def test_conv_step_counts():
+    c = bench.conv_step_counts(256, 5120, 4, 2, 2)
+    assert c["tokch"] == 256 * 5120
+    assert c["bytes"] == 256 * 5120 * (24 + 4) + 5120 * 20
+
+
+def test_workload_kinds():
+    assert [bench.workload_kind(n) for n in ("mamba130m", "decode", "conv130m", "conv2p8b", "convstep")] \
+        == ["scan", "decode", "conv", "conv", "convstep"]
+
+
+@pytest.mark.parametrize("name", ["conv130m", "convstep"])
+def test_conv_oracle_rate_single_core(name):
+    r = bench.oracle_rate(name, threads=4, budget_s=0.2)
+    assert r["kind"] == "oracle" and r["cores"] == 1 and r["value"] > 0
