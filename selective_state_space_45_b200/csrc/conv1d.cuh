@@ -29,21 +29,22 @@ struct ConvArgs {
     int silu;
 };
 
-template <typename T> struct Vec16;  // one 16-byte vector of T
+// One 16-byte vector of T: kN elements, loaded raw (Raw) and widened to fp32 (unpack).
+template <typename T> struct Vec16;
 template <> struct Vec16<float> {
     static constexpr int kN = 4;
-    __device__ __forceinline__ static void load(const float *p, float *v) {
-        const float4 q = __ldg(reinterpret_cast<const float4 *>(p));
+    using Raw = float4;
+    __device__ __forceinline__ static void unpack(const float4 &q, float *v) {
         v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
     }
 };
 template <> struct Vec16<__nv_bfloat16> {
     static constexpr int kN = 8;
-    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float *v) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(p));
+    using Raw = uint4;
+    __device__ __forceinline__ static void unpack(const uint4 &q, float *v) {
         const unsigned w4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4; ++i) {   // bf16 -> fp32 is exact: the bits move up 16 places
             v[2 * i] = __uint_as_float(w4[i] << 16);
             v[2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
         }
@@ -73,68 +74,83 @@ template <int n> __device__ __forceinline__ void store_run(__nv_bfloat16 *p, con
     }
 }
 
-// Vector path: rows whose length is a multiple of one 16-byte vector and 16-byte aligned
-// tensors.  Thread g owns chunk c = g mod nchunk of row g / nchunk: CH = 2 vectors of
-// consecutive tokens (the last chunk of a row may hold one).  The K-1 inputs before the
-// chunk come from lane - 1 by shuffle (it owns chunk c-1 of the same row), from the carried
-// history when c = 0, and from global memory for lane 0.  All lanes of a warp run the
-// loop together so that the shuffles see every lane.
-template <typename Tin, typename Tout, int K>
-__global__ void __launch_bounds__(256)
-causal_conv1d_vec_kernel(ConvArgs a, long long nchunk, long long total) {
+// Vector path: rows whose length is a multiple of one 16-byte vector (V elements), widths
+// 1..4 (K-1 <= V).  Each warp owns a span of 32*U consecutive vectors of one row, laid out
+// as a copy kernel lays them out: vector v0 + 32k + lane goes to lane `lane`, load k, so
+// every load and store instruction of the warp covers 512 contiguous bytes.  The K-1
+// inputs in front of a vector are the tail of the vector before it: lane - 1's vector of
+// the same load, lane 31's vector of the previous load (for lane 0), and for the span's
+// first vector the row itself (span > 0) or the carried window (span 0).  All U loads are
+// issued before any arithmetic.
+// 6 resident blocks of 256 threads per SM (a 40-register budget); fp32 inputs with bf16
+// outputs need a few more registers to pack, and take 5.
+template <typename Tin, typename Tout, int K, int U>
+__global__ void __launch_bounds__(256, (sizeof(Tin) == 4 && sizeof(Tout) == 2) ? 5 : 6)
+causal_conv1d_vec_kernel(ConvArgs a, long long nvr, long long spans_per_row, long long total_spans) {
     constexpr int V = Vec16<Tin>::kN;
-    constexpr int CH = 2 * V;
     constexpr int H = K - 1;
-    const Tin *__restrict__ x = static_cast<const Tin *>(a.x);
-    Tout *__restrict__ u = static_cast<Tout *>(a.u);
+    static_assert(H <= V, "the window must fit in one vector");
+    using R = typename Vec16<Tin>::Raw;
     const int lane = threadIdx.x & 31;
-    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-    for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-         g - lane < total; g += stride) {
-        const bool active = g < total;
-        const long long row = active ? g / nchunk : 0;
-        const long long c = active ? g - row * nchunk : 0;
-        const long long t0 = c * CH;
-        const long long base = row * a.seqlen + t0;
-        const bool second = active && t0 + V < a.seqlen;
-        // xe[0..H) = inputs t0-H .. t0-1, xe[H..H+CH) = this chunk
-        float xe[H + CH];
+    const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (gw >= total_spans) return;   // the whole warp: the shuffles below see all lanes
+    const long long row = gw / spans_per_row;
+    const long long v0 = (gw - row * spans_per_row) * (32 * U);
+    const Tin *__restrict__ xr = static_cast<const Tin *>(a.x) + row * a.seqlen;
+    Tout *__restrict__ ur = static_cast<Tout *>(a.u) + row * a.seqlen;
+    R raw[U];
 #pragma unroll
-        for (int i = 0; i < H + CH; ++i) xe[i] = 0.f;
-        if (active) Vec16<Tin>::load(x + base, xe + H);
-        if (second) Vec16<Tin>::load(x + base + V, xe + H + V);
-        // the previous chunk is always full, so its last H values are xe[CH..CH+H) of lane - 1
+    for (int k = 0; k < U; ++k) {
+        const long long p = v0 + 32 * k + lane;
+        if (p < nvr) raw[k] = __ldg(reinterpret_cast<const R *>(xr + p * V));
+        else raw[k] = R{};
+    }
+    const int d = static_cast<int>(row % a.dim);
+    float w[K];
 #pragma unroll
-        for (int j = 0; j < H; ++j) xe[j] = __shfl_up_sync(0xffffffffu, xe[CH + j], 1);
-        if (active && c == 0) {
-            const float *hp = a.hist ? a.hist + row * H : nullptr;
+    for (int i = 0; i < K; ++i) w[i] = __ldg(a.w + static_cast<long long>(d) * K + i);
+    const float b0 = a.bias ? __ldg(a.bias + d) : 0.f;
+    float halo0[H > 0 ? H : 1];      // inputs before the span (lane 0 only)
 #pragma unroll
-            for (int j = 0; j < H; ++j) xe[j] = hp ? __ldg(hp + j) : 0.f;
-        } else if (active && lane == 0) {
+    for (int j = 0; j < H; ++j) halo0[j] = 0.f;
+    if (lane == 0) {
+        if (v0 > 0) {
 #pragma unroll
-            for (int j = 0; j < H; ++j) xe[j] = to_f32<Tin>(x[base - H + j]);
+            for (int j = 0; j < H; ++j) halo0[j] = to_f32<Tin>(xr[v0 * V - H + j]);
+        } else if (a.hist) {
+#pragma unroll
+            for (int j = 0; j < H; ++j) halo0[j] = __ldg(a.hist + row * H + j);
         }
-        if (!active) continue;
-        const int d = static_cast<int>(row % a.dim);
-        float w[K];
+    }
+    float tail[H > 0 ? H : 1];       // the last H inputs of this lane's previous vector
 #pragma unroll
-        for (int i = 0; i < K; ++i) w[i] = __ldg(a.w + static_cast<long long>(d) * K + i);
-        const float b0 = a.bias ? __ldg(a.bias + d) : 0.f;
-        float o[CH];
+    for (int j = 0; j < H; ++j) tail[j] = 0.f;
 #pragma unroll
-        for (int t = 0; t < CH; ++t) {
-            float acc = b0;
+    for (int k = 0; k < U; ++k) {
+        const long long p = v0 + 32 * k + lane;
+        float xe[H + V];             // xe[0..H) the inputs before the vector, then the vector
+        Vec16<Tin>::unpack(raw[k], xe + H);
 #pragma unroll
-            for (int i = 0; i < K; ++i) acc = fmaf(w[i], xe[t + i], acc);
-            o[t] = a.silu ? silu_f(acc) : acc;
+        for (int j = 0; j < H; ++j) {
+            const float up = __shfl_up_sync(0xffffffffu, xe[V + j], 1);
+            const float wrap = __shfl_sync(0xffffffffu, tail[j], 31);
+            xe[j] = lane > 0 ? up : (k > 0 ? wrap : halo0[j]);
+            tail[j] = xe[V + j];
         }
-        store_run<V>(u + base, o);
-        if (second) store_run<V>(u + base + V, o + V);
-        if (a.hist_out && H > 0 && t0 + CH >= a.seqlen) {
-            // the row's last chunk: the window a decode step continues from
-            // its last H inputs end the chunk's one or two vectors (V >= H)
+        if (p < nvr) {
+            float o[V];
 #pragma unroll
-            for (int j = 0; j < H; ++j) a.hist_out[row * H + j] = second ? xe[CH + j] : xe[V + j];
+            for (int t = 0; t < V; ++t) {
+                float acc = b0;
+#pragma unroll
+                for (int i = 0; i < K; ++i) acc = fmaf(w[i], xe[t + i], acc);
+                o[t] = a.silu ? silu_f(acc) : acc;
+            }
+            store_run<V>(ur + p * V, o);
+            if (a.hist_out && p == nvr - 1) {   // the row's last vector: the window to continue from
+#pragma unroll
+                for (int j = 0; j < H; ++j) a.hist_out[row * H + j] = xe[V + j];
+            }
         }
     }
 }

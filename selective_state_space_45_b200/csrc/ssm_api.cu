@@ -172,12 +172,20 @@ int launch_step(const ssm::StepArgs &a, cudaStream_t s) {
 
 template <typename Tin, typename Tout, int K>
 int launch_conv_vec(const ssm::ConvArgs &a, cudaStream_t s) {
-    constexpr int CH = 2 * ssm::Vec16<Tin>::kN;
-    const long long nchunk = (a.seqlen + CH - 1) / CH;
-    const long long total = a.rows * nchunk;
-    const long long blocks = std::min<long long>((total + 255) / 256, INT_MAX);
-    ssm::causal_conv1d_vec_kernel<Tin, Tout, K>
-        <<<static_cast<unsigned>(blocks), 256, 0, s>>>(a, nchunk, total);
+    // warp spans of 32*U vectors: U = 4 for rows of more than 64 vectors, else 1 so that
+    // short rows do not leave most lanes idle
+    const long long nvr = a.seqlen / ssm::Vec16<Tin>::kN;
+    const int U = nvr > 64 ? 4 : 1;
+    const long long spans_per_row = (nvr + 32 * U - 1) / (32 * U);
+    const long long total_spans = a.rows * spans_per_row;
+    const long long blocks = (total_spans * 32 + 255) / 256;
+    if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    if (U == 4)
+        ssm::causal_conv1d_vec_kernel<Tin, Tout, K, 4><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+            a, nvr, spans_per_row, total_spans);
+    else
+        ssm::causal_conv1d_vec_kernel<Tin, Tout, K, 1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+            a, nvr, spans_per_row, total_spans);
     return status_of(cudaGetLastError());
 }
 
