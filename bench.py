@@ -20,7 +20,6 @@ from __future__ import annotations
 
 import argparse
 import datetime
-import hashlib
 import json
 import os
 import statistics
@@ -115,14 +114,15 @@ def load_peaks():
         return dict(hbm_gbs=FALLBACK_HBM_GBS, sm_max_mhz=FALLBACK_SM_MHZ, source="fallback")
 
 
-def kernel_source_hash():
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "selective_state_space_45_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
-    return h.hexdigest()[:16]
+# translation unit of libssm.so that holds each kernel and its launch logic
+KERNEL_UNIT = {"scan_fwd_kernel": "scan_api.cu", "state_step_kernel": "step_api.cu",
+               "causal_conv1d_vec_kernel": "conv_api.cu", "conv1d_step_kernel": "conv_api.cu"}
+
+
+def kernel_source_hash(kernel):
+    """Hash of the sources (kernel, headers, launch code) a kernel is built from."""
+    from selective_state_space_45_b200.build import source_hash
+    return source_hash(KERNEL_UNIT[kernel])
 
 
 def recorded_traffic(kernel, workload):
@@ -132,7 +132,7 @@ def recorded_traffic(kernel, workload):
             rec = json.load(f).get("%s %s" % (kernel, workload))
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return float(rec["dram_bytes_per_launch"])
 
