@@ -12,6 +12,7 @@ from .oracle import (  # noqa: F401
     lti_conv,
     lti_kernel,
     scan,
+    scan_bwd,
     scan_parallel_reference,
     step,
 )

@@ -21,6 +21,9 @@ Functions and the passages they follow:
 ``scan_parallel_reference``   the whole selective scan routed through the Hillis-Steele
                               rounds over N-expanded pairs (tiny inputs only): an
                               implementation independent of the C loop.
+``scan_bwd``        gradients of the scan by reverse-mode differentiation of the same
+                    recurrence (Euler gain): the training half; xmarva lesson 10,
+                    section 6 (Mamba's kernel recomputes the states in the backward pass).
 ``causal_conv1d`` / ``conv1d_step``  the causal depthwise convolution with SiLU in front of
                               the scan, and its one-token window form: learnllm "Module 19",
                               "The Causal Convolution"; xmarva lesson 10, sections 4 and 7.
@@ -67,6 +70,9 @@ def _load():
                                         p, p, i64, i64, i64, i64, ctypes.c_int]
             lib.oracle_step.restype = None
             lib.oracle_step.argtypes = [p, p, p, p, p, p, p, p, p, i64, i64, i64]
+            lib.oracle_scan_bwd.restype = ctypes.c_int
+            lib.oracle_scan_bwd.argtypes = [p, p, p, ctypes.c_int, p, p, p, p, p, p, p, p,
+                                            p, p, p, p, p, p, p, p, p, i64, i64, i64, i64]
             lib.oracle_causal_conv1d.restype = None
             lib.oracle_causal_conv1d.argtypes = [p, p, p, p, ctypes.c_int, p, p, i64, i64, i64, i64]
             lib.oracle_conv1d_step.restype = None
@@ -144,6 +150,43 @@ def step(state, x, delta, A, B, C, D=None, z=None):
     _load().oracle_step(_ptr(st), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
                         _ptr(z), _ptr(y), batch, dim, N)
     return y, st
+
+
+def scan_bwd(dy, x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
+             h0=None, dfinal=None):
+    """Gradients of  sum(dy * y) + sum(dfinal * final_state)  of the (Euler) scan, in fp64.
+
+    Same layouts as ``scan``; dy [batch, dim, L], dfinal [batch, dim, N].  Returns a dict
+    with dx, ddelta, dz (or None), dB, dC, dA, dD (or None), ddelta_bias (or None), dh0.
+    """
+    x = _f64(x)
+    batch, dim, L = x.shape
+    A = _f64(A)
+    N = A.shape[1]
+    dy = _f64(dy, (batch, dim, L))
+    delta = _f64(delta, (batch, dim, L))
+    B = _f64(B, (batch, L, N))
+    C = _f64(C, (batch, L, N))
+    D = _f64(D, (dim,))
+    z = _f64(z, (batch, dim, L))
+    delta_bias = _f64(delta_bias, (dim,))
+    h0 = _f64(h0, (batch, dim, N))
+    dfinal = _f64(dfinal, (batch, dim, N))
+    out = dict(dx=np.empty((batch, dim, L)), ddelta=np.empty((batch, dim, L)),
+               dz=None if z is None else np.empty((batch, dim, L)),
+               dB=np.empty((batch, L, N)), dC=np.empty((batch, L, N)), dA=np.empty((dim, N)),
+               dD=None if D is None else np.empty(dim),
+               ddelta_bias=None if delta_bias is None else np.empty(dim),
+               dh0=np.empty((batch, dim, N)))
+    rc = _load().oracle_scan_bwd(
+        _ptr(x), _ptr(delta), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(A), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), _ptr(h0), _ptr(dy), _ptr(dfinal),
+        _ptr(out["dx"]), _ptr(out["ddelta"]), _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]),
+        _ptr(out["dD"]), _ptr(out["dz"]), _ptr(out["ddelta_bias"]), _ptr(out["dh0"]),
+        batch, dim, L, N)
+    if rc != 0:
+        raise ValueError("oracle.scan_bwd: unsupported sizes")
+    return out
 
 
 def causal_conv1d(x, weight, bias=None, hist=None, silu=True):

@@ -44,6 +44,7 @@
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
+#include <stdlib.h>
 #ifdef _OPENMP
 #include <omp.h>
 #endif
@@ -228,4 +229,129 @@ void oracle_conv1d_step(double *window, const double *x, const double *w, const 
             if (K > 1)
                 win[K - 2] = x[row];
         }
+}
+
+/*
+ * Backward of the scan (Euler gain): the gradients of a scalar loss
+ *     loss = sum_{b,d,t} dy[b,d,t] * y[b,d,t]  +  sum_{b,d,n} dfinal[b,d,n] * h_{L-1}[b,d,n]
+ * with respect to every input, by reverse-mode differentiation of the recurrence written
+ * above -- the training half that the xmarva lesson (section 6, the paragraph on Mamba's
+ * own kernel) describes as recomputing the states in the backward pass instead of
+ * storing them.  Here the states of one channel are stored (the oracle has memory to
+ * spare); the kernel recomputes them.
+ *
+ * With h_{-1} = h0, Delta_t, Abar_t[n] = exp(Delta_t A[n]) and y_t as in oracle_scan,
+ * going t = L-1 .. 0 with mu[n] = dfinal[n] (the adjoint flowing into h_{L-1} from later
+ * tokens):
+ *     g_t       = SiLU(z_t)                     (1 without a gate)
+ *     dypre_t   = dy_t * g_t                    (adjoint of the pre-gate output)
+ *     dz_t      = dy_t * ypre_t * SiLU'(z_t),   SiLU'(z) = s (1 + z (1 - s)), s = sigmoid(z)
+ *     lambda[n] = dypre_t C_t[n] + mu[n]        (adjoint of h_t)
+ *     dC_t[n]  += dypre_t h_t[n]                dB_t[n] += lambda[n] Delta_t x_t
+ *     dx_t      = dypre_t D + sum_n lambda[n] Delta_t B_t[n]
+ *     dDelta_t  = sum_n lambda[n] (B_t[n] x_t + h_{t-1}[n] Abar_t[n] A[n])
+ *     dA[n]    += lambda[n] h_{t-1}[n] Abar_t[n] Delta_t
+ *     mu[n]     = Abar_t[n] lambda[n]           (adjoint of h_{t-1})
+ *     ddelta_t  = dDelta_t * sigmoid(delta_t + bias)   (the softplus' slope; 1 without it)
+ *     dbias    += ddelta_t,  dD += dypre_t x_t
+ * and dh0 = mu after t = 0.  dB, dC sum over channels; dA, dD, dbias over sequences and
+ * positions.  Accumulated outputs are zeroed here first.
+ *   dy, dx, ddelta, dz : [batch][dim][seqlen];  dB, dC: [batch][seqlen][dstate]
+ *   dA: [dim][dstate];  dD, ddelta_bias: [dim];  dfinal, h0, dh0: [batch][dim][dstate]
+ * Optional (NULL): dfinal (zero), h0 (zero), D and dD, z and dz, delta_bias and
+ * ddelta_bias, dh0.  Returns 0, or -1 for sizes it cannot handle or a failed allocation.
+ */
+int oracle_scan_bwd(const double *x, const double *delta, const double *delta_bias,
+                    int delta_softplus, const double *A, const double *B, const double *C,
+                    const double *D, const double *z, const double *h0,
+                    const double *dy, const double *dfinal,
+                    double *dx, double *ddelta, double *dA, double *dB, double *dC,
+                    double *dD, double *dz, double *ddelta_bias, double *dh0,
+                    int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate)
+{
+    if (dstate < 1 || dstate > 256 || batch < 0 || dim < 0 || seqlen < 0)
+        return -1;
+    const int64_t N = dstate;
+    double *hs = (double *)malloc(sizeof(double) * (size_t)((seqlen + 1) * N + 2 * seqlen + 1));
+    if (!hs)
+        return -1;
+    double *step = hs + (seqlen + 1) * N;   /* Delta_t      */
+    double *ypre = step + seqlen;           /* y_t before the gate */
+    for (int64_t i = 0; i < dim * N; ++i) dA[i] = 0.0;
+    for (int64_t i = 0; i < batch * seqlen * N; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
+    if (dD) for (int64_t i = 0; i < dim; ++i) dD[i] = 0.0;
+    if (ddelta_bias) for (int64_t i = 0; i < dim; ++i) ddelta_bias[i] = 0.0;
+
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t row = b * dim + d;
+            const double *x_r = x + row * seqlen;
+            const double *A_d = A + d * N;
+            /* forward: keep every state, h_{t} at hs[(t+1)*N] and h_{-1} at hs[0] */
+            for (int64_t n = 0; n < N; ++n)
+                hs[n] = h0 ? h0[row * N + n] : 0.0;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                double v = delta[row * seqlen + t] + (delta_bias ? delta_bias[d] : 0.0);
+                step[t] = delta_softplus ? oracle_softplus(v) : v;
+                const double *B_t = B + (b * seqlen + t) * N;
+                const double *C_t = C + (b * seqlen + t) * N;
+                double yp = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    double h = exp(step[t] * A_d[n]) * hs[t * N + n] + step[t] * B_t[n] * x_r[t];
+                    hs[(t + 1) * N + n] = h;
+                    yp += C_t[n] * h;
+                }
+                if (D)
+                    yp += D[d] * x_r[t];
+                ypre[t] = yp;
+            }
+            /* reverse */
+            double mu[256];
+            for (int64_t n = 0; n < N; ++n)
+                mu[n] = dfinal ? dfinal[row * N + n] : 0.0;
+            for (int64_t t = seqlen - 1; t >= 0; --t) {
+                const double dy_t = dy[row * seqlen + t];
+                double g = 1.0;
+                if (z) {
+                    const double zt = z[row * seqlen + t];
+                    const double s = 1.0 / (1.0 + exp(-zt));
+                    g = zt * s;
+                    dz[row * seqlen + t] = dy_t * ypre[t] * s * (1.0 + zt * (1.0 - s));
+                }
+                const double dypre = dy_t * g;
+                const double *B_t = B + (b * seqlen + t) * N;
+                const double *C_t = C + (b * seqlen + t) * N;
+                double *dB_t = dB + (b * seqlen + t) * N;
+                double *dC_t = dC + (b * seqlen + t) * N;
+                double dxt = D ? dypre * D[d] : 0.0;
+                double dstep = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double lam = dypre * C_t[n] + mu[n];
+                    const double abar = exp(step[t] * A_d[n]);
+                    const double hprev = hs[t * N + n];
+                    dC_t[n] += dypre * hs[(t + 1) * N + n];
+                    dB_t[n] += lam * step[t] * x_r[t];
+                    dxt += lam * step[t] * B_t[n];
+                    dstep += lam * (B_t[n] * x_r[t] + hprev * abar * A_d[n]);
+                    dA[d * N + n] += lam * hprev * abar * step[t];
+                    mu[n] = abar * lam;
+                }
+                double dd = dstep;
+                if (delta_softplus) {
+                    const double v = delta[row * seqlen + t] + (delta_bias ? delta_bias[d] : 0.0);
+                    dd *= 1.0 / (1.0 + exp(-v));
+                }
+                ddelta[row * seqlen + t] = dd;
+                if (ddelta_bias)
+                    ddelta_bias[d] += dd;
+                if (dD)
+                    dD[d] += dypre * x_r[t];
+                dx[row * seqlen + t] = dxt;
+            }
+            if (dh0)
+                for (int64_t n = 0; n < N; ++n)
+                    dh0[row * N + n] = mu[n];
+        }
+    free(hs);
+    return 0;
 }

@@ -391,3 +391,98 @@ def test_conv_width_one_is_pointwise():
     u, win = oracle.causal_conv1d(x, w, bias=b, silu=False)
     np.testing.assert_allclose(u, w[None, :, :1] * x + b[None, :, None], rtol=1e-15)
     assert win.shape == (1, 3, 0)
+
+
+# ----------------------------------------------------------------------------------
+# backward of the scan (xmarva lesson 10, section 6: the training half recomputes the
+# states): pinned by central finite differences of the forward oracle and closed forms
+# ----------------------------------------------------------------------------------
+
+def _bwd_case(rng, batch, dim, L, N, softplus=True):
+    case = _random_case(rng, batch, dim, L, N)
+    case["h0"] = rng.normal(size=(batch, dim, N))
+    if not softplus:
+        case["delta"] = np.abs(case["delta"]) * 0.5 + 0.05     # positive steps as given
+        case["delta_bias"] = np.abs(case["delta_bias"]) * 0.1
+    return case
+
+
+def _loss(case, dy, dfinal, softplus):
+    y, hN = oracle.scan(delta_softplus=softplus, **case)
+    return float(np.sum(dy * y) + np.sum(dfinal * hN))
+
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_scan_bwd_matches_central_differences(softplus):
+    rng = np.random.default_rng(29 + softplus)
+    batch, dim, L, N = 2, 3, 6, 4
+    case = _bwd_case(rng, batch, dim, L, N, softplus)
+    dy = rng.normal(size=(batch, dim, L))
+    dfinal = rng.normal(size=(batch, dim, N))
+    g = oracle.scan_bwd(dy, delta_softplus=softplus, dfinal=dfinal, **case)
+    names = dict(x="dx", delta="ddelta", z="dz", A="dA", B="dB", C="dC", D="dD",
+                 delta_bias="ddelta_bias", h0="dh0")
+    eps = 1e-6
+    for key, gname in names.items():
+        base = case[key]
+        fd = np.empty_like(base)
+        for idx in np.ndindex(base.shape):
+            plus = {k: v.copy() for k, v in case.items()}
+            minus = {k: v.copy() for k, v in case.items()}
+            plus[key][idx] += eps
+            minus[key][idx] -= eps
+            fd[idx] = (_loss(plus, dy, dfinal, softplus) - _loss(minus, dy, dfinal, softplus)) / (2 * eps)
+        np.testing.assert_allclose(g[gname], fd, rtol=1e-6, atol=1e-7, err_msg=gname)
+
+
+def test_scan_bwd_no_decay_closed_form():
+    # A = 0: h_t = sum_{s<=t} Delta_s B_s x_s (a running sum).  Loss = y_{L-1} alone, so
+    # every earlier token reaches it with weight C_{L-1}.
+    rng = np.random.default_rng(31)
+    L = 5
+    x, step, B, C = (rng.normal(size=L), rng.uniform(0.1, 0.9, size=L), rng.normal(size=L),
+                     rng.normal(size=L))
+    dy = np.zeros((1, 1, L))
+    dy[0, 0, -1] = 1.0
+    g = oracle.scan_bwd(dy, x.reshape(1, 1, L), step.reshape(1, 1, L), np.zeros((1, 1)),
+                        B.reshape(1, L, 1), C.reshape(1, L, 1))
+    cL = C[-1]
+    np.testing.assert_allclose(g["dx"][0, 0], cL * step * B, rtol=1e-14)
+    np.testing.assert_allclose(g["ddelta"][0, 0], cL * B * x, rtol=1e-14)
+    np.testing.assert_allclose(g["dB"][0, :, 0], cL * step * x, rtol=1e-14)
+    h = np.cumsum(step * B * x)
+    expect_dC = np.zeros(L)
+    expect_dC[-1] = h[-1]
+    np.testing.assert_allclose(g["dC"][0, :, 0], expect_dC, rtol=1e-14, atol=0)
+    hprev = np.concatenate([[0.0], h[:-1]])
+    np.testing.assert_allclose(g["dA"][0, 0], cL * np.sum(hprev * step), rtol=1e-13)
+
+
+def test_scan_bwd_initial_state_gradient_is_the_decay_product():
+    # one state, loss = y_{L-1}: dh0 = C_{L-1} prod_t exp(Delta_t a)
+    rng = np.random.default_rng(37)
+    L, a = 6, -0.7
+    step = rng.uniform(0.05, 0.5, size=L)
+    C = rng.normal(size=L)
+    dy = np.zeros((1, 1, L))
+    dy[0, 0, -1] = 1.0
+    g = oracle.scan_bwd(dy, rng.normal(size=(1, 1, L)), step.reshape(1, 1, L), np.array([[a]]),
+                        rng.normal(size=(1, L, 1)), C.reshape(1, L, 1), h0=np.ones((1, 1, 1)))
+    assert abs(g["dh0"][0, 0, 0] - C[-1] * math.exp(a * step.sum())) < 1e-14
+
+
+def test_scan_bwd_gate_and_skip_closed_form():
+    # C = 0, D = 1: y = x SiLU(z); SiLU'(0) = 1/2, SiLU'(z) = s (1 + z (1 - s))
+    zs = np.array([0.0, math.log(3.0), -math.log(3.0)])
+    x = np.array([2.0, -1.0, 0.5])
+    dy = np.array([1.0, 2.0, -1.0])
+    L = 3
+    g = oracle.scan_bwd(dy.reshape(1, 1, L), x.reshape(1, 1, L), np.full((1, 1, L), 0.3),
+                        np.array([[-1.0]]), np.ones((1, L, 1)), np.zeros((1, L, 1)),
+                        D=np.array([1.0]), z=zs.reshape(1, 1, L))
+    s = np.array([0.5, 0.75, 0.25])
+    np.testing.assert_allclose(g["dz"][0, 0], dy * x * s * (1 + zs * (1 - s)), rtol=1e-14)
+    assert abs(g["dz"][0, 0, 0] - 0.5 * dy[0] * x[0]) < 1e-15
+    # the state never reaches y, so x's gradient is the skip's alone
+    np.testing.assert_allclose(g["dx"][0, 0], dy * zs * s, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(g["dD"], [np.sum(dy * zs * s * x)], rtol=1e-14)
