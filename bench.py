@@ -3,7 +3,8 @@
 
 One JSON line on rank 0.  A step is one pass of the whole hot path over one batch:
 for the scan workloads one ``ssm_selective_scan_fwd`` call (discretise, recurrence,
-readout, skip, gate, final state), for the decode workload one ``ssm_state_step`` call;
+readout, skip, gate, final state), for the decode workload one ``ssm_state_step`` call,
+for bwd130m one ``ssm_selective_scan_bwd`` call (all gradients of the scan);
 the conv workloads time the causal convolution in front of the scan
 (``ssm_causal_conv1d_fwd`` with its final window, or one ``ssm_causal_conv1d_step``).
 
@@ -11,8 +12,8 @@ the conv workloads time the causal convolution in front of the scan
   python bench.py --impl reference ...        # the fp64 CPU oracle, timed on host cores
 
 Workloads (selective_state_space_45_b200.inputs.CONFIGS): mamba130m (default: batch 8,
-L 2048, d_inner 1536, N 16, bf16 in/out, fp32 state), mamba2p8b, long1m, decode, and the
-convolution's conv130m, conv2p8b, convstep.
+L 2048, d_inner 1536, N 16, bf16 in/out, fp32 state), mamba2p8b, long1m, decode, the
+backward's bwd130m, and the convolution's conv130m, conv2p8b, convstep.
 Multi-GPU: every rank runs its own replica (channels are independent; the path has no
 exchange step), timing is the max over ranks, value counts all ranks' work.
 """
@@ -51,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba130m",
                     choices=["mamba130m", "mamba2p8b", "long1m", "decode", "tiny",
-                             "conv130m", "conv2p8b", "convstep"])
+                             "conv130m", "conv2p8b", "convstep", "bwd130m"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0,
@@ -116,6 +117,7 @@ def load_peaks():
 
 # translation unit of libssm.so that holds each kernel and its launch logic
 KERNEL_UNIT = {"scan_fwd_kernel": "scan_api.cu", "state_step_kernel": "step_api.cu",
+               "scan_bwd_kernel": "bwd_api.cu",
                "causal_conv1d_vec_kernel": "conv_api.cu", "conv1d_step_kernel": "conv_api.cu"}
 
 
@@ -212,7 +214,20 @@ def conv_step_counts(batch, dim, K, in_size, out_size):
     return dict(bytes=window + streams + params, exps=batch * dim, tokch=batch * dim)
 
 
+def bwd_counts(batch, dim, L, N, in_size, g_size):
+    """Backward: inputs read once (x, delta, z, B, C, dy, parameters), gradients written
+    once.  Work: 2 ex2 per (t, d, n) -- the states recomputed forward and the decay again
+    in the reverse walk, the least a backward that keeps no N-expanded tensor in HBM
+    needs."""
+    streams = batch * dim * L * (3 * in_size + g_size + 3 * g_size)   # x, delta, z, dy in; dx, ddelta, dz out
+    bc = 2 * batch * L * N * (in_size + g_size)                       # B, C in; dB, dC out
+    params = 2 * (dim * N * 4 + 2 * dim * 4)                          # A, D, bias in; dA, dD, dbias out
+    return dict(bytes=streams + bc + params, exps=2 * batch * L * dim * N, tokch=batch * L * dim)
+
+
 def workload_kind(name):
+    if name.startswith("bwd"):
+        return "bwd"
     if name == "decode":
         return "decode"
     if name == "convstep":
@@ -245,6 +260,8 @@ class Workload:
         esz = torch.tensor([], dtype=dt).element_size()
         if self.kind == "scan":
             self.counts = scan_counts(c["batch"], c["dim"], c["seqlen"], c["dstate"], esz, esz)
+        elif self.kind == "bwd":
+            self.counts = bwd_counts(c["batch"], c["dim"], c["seqlen"], c["dstate"], esz, esz)
         elif self.kind == "decode":
             self.counts = step_counts(c["batch"], c["dim"], c["dstate"], esz, esz)
         elif self.kind == "conv":
@@ -259,6 +276,14 @@ class Workload:
             if self.kind == "scan":
                 inp["y"] = torch.empty(inp["x"].shape, device=device, dtype=dt)
                 inp["fs"] = torch.empty(c["batch"], c["dim"], c["dstate"], device=device)
+            elif self.kind == "bwd":
+                for k in ("dx", "ddelta", "dz"):
+                    inp[k] = torch.empty(inp["x"].shape, device=device, dtype=dt)
+                for k in ("dB", "dC"):
+                    inp[k] = torch.empty(inp["B"].shape, device=device, dtype=dt)
+                inp["dA"] = torch.empty(inp["A"].shape, device=device)
+                inp["dD"] = torch.empty(c["dim"], device=device)
+                inp["dbias"] = torch.empty(c["dim"], device=device)
             elif self.kind == "conv":
                 inp["u"] = torch.empty(inp["x"].shape, device=device, dtype=dt)
                 inp["fw"] = torch.empty(c["batch"], c["dim"], c["width"] - 1, device=device)
@@ -273,6 +298,10 @@ class Workload:
         if self.kind == "scan":
             ssm.ssm_selective_scan_fwd(s["x"], s["delta"], s["delta_bias"], True, s["A"], s["B"],
                                        s["C"], s["D"], s["z"], s["y"], s["fs"], stream)
+        elif self.kind == "bwd":
+            ssm.ssm_selective_scan_bwd(s["x"], s["delta"], s["delta_bias"], True, s["A"], s["B"], s["C"],
+                                       s["D"], s["z"], None, s["dy"], None, s["dx"], s["ddelta"], s["dA"],
+                                       s["dB"], s["dC"], s["dD"], s["dz"], s["dbias"], None, stream)
         elif self.kind == "decode":
             t = (i // self.nsets) % s["x"].shape[0]
             ssm.ssm_state_step(s["state"], s["x"][t], s["delta"][t], s["A"], s["B"][t], s["C"][t],
@@ -295,6 +324,10 @@ class Workload:
         if self.kind == "convstep":
             return ("decode conv1d step: batch %d, d_inner %d, width %d, fp32 window in place, one %s "
                     "token per sequence" % (c["batch"], c["dim"], c["width"], io))
+        if self.kind == "bwd":
+            return ("%s-shaped selective scan backward (states recomputed): batch %d, L %d, d_inner %d, "
+                    "N %d, %s inputs, dy and gradients, fp32 A/D/bias gradients"
+                    % (self.name[3:], c["batch"], c["seqlen"], c["dim"], c["dstate"], io))
         if self.kind == "scan":
             return ("%s-shaped selective scan: batch %d, L %d, d_inner %d, N %d, %s x/delta/z/B/C "
                     "and y, fp32 A/D/bias/state" % (self.name, c["batch"], c["seqlen"], c["dim"],
@@ -305,7 +338,7 @@ class Workload:
 
 def kernel_name(kind):
     return dict(scan="scan_fwd_kernel", decode="state_step_kernel", conv="causal_conv1d_vec_kernel",
-                convstep="conv1d_step_kernel")[kind]
+                convstep="conv1d_step_kernel", bwd="scan_bwd_kernel")[kind]
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -338,6 +371,18 @@ def _oracle_sample(name, n_target_tokch, seed=0):
                                       seed=seed)
         return kind, inp, per_channel * k, "%d sequences x %d of %d channels, all %d tokens" % (
             c["batch"], k, c["dim"], c["seqlen"])
+    if kind == "bwd":
+        per_channel = c["batch"] * c["seqlen"]
+        k = int(max(1, min(c["dim"], n_target_tokch // per_channel)))
+        L = c["seqlen"]
+        if k == 1 and n_target_tokch < per_channel:  # one channel of one sequence, shortened
+            L = int(max(64, min(L, n_target_tokch)))
+            inp = inputs.make_scan_bwd_inputs(1, 1, L, c["dstate"], c["dtype"], device="cpu", seed=seed)
+            return kind, inp, L, "1 channel of 1 sequence, first %d of %d tokens" % (L, c["seqlen"])
+        inp = inputs.make_scan_bwd_inputs(c["batch"], k, L, c["dstate"], c["dtype"], device="cpu",
+                                          seed=seed)
+        return kind, inp, per_channel * k, "%d sequences x %d of %d channels, all %d tokens" % (
+            c["batch"], k, c["dim"], L)
     if name == "decode":
         k = int(max(1, min(c["dim"], n_target_tokch // c["batch"])))
         inp = inputs.make_decode_inputs(c["batch"], k, c["dstate"], 1, c["dtype"], device="cpu",
@@ -365,6 +410,9 @@ def _oracle_call(kind, inp, threads):
     if kind == "scan":
         oracle.scan(x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], D=inp["D"],
                     z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True, nthreads=threads)
+    elif kind == "bwd":
+        oracle.scan_bwd(inp["dy"], inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                        z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True)
     elif kind == "conv":
         oracle.causal_conv1d(inp["x"], inp["weight"], bias=inp["bias"])
     elif kind == "convstep":
@@ -454,6 +502,8 @@ def time_e2e(wl, steps, stream):
     per_token = {"decode": ("x", "delta", "z", "B", "C"), "convstep": ("x",)}.get(wl.kind, ())
     names_in, names_out = dict(
         scan=(["x", "delta", "z", "B", "C", "A", "D", "delta_bias"], ["y", "fs"]),
+        bwd=(["x", "delta", "z", "B", "C", "A", "D", "delta_bias", "dy"],
+             ["dx", "ddelta", "dz", "dB", "dC", "dA", "dD", "dbias"]),
         decode=(["state", "x", "delta", "z", "B", "C", "A", "D"], ["y", "state"]),
         conv=(["x", "weight", "bias"], ["u", "fw"]),
         convstep=(["window", "x", "weight", "bias"], ["u", "window"]))[wl.kind]
@@ -476,6 +526,11 @@ def time_e2e(wl, steps, stream):
         if wl.kind == "scan":
             ssm.ssm_selective_scan_fwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"],
                                        dev["B"], dev["C"], dev["D"], dev["z"], dev["y"], dev["fs"])
+        elif wl.kind == "bwd":
+            ssm.ssm_selective_scan_bwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"], dev["B"],
+                                       dev["C"], dev["D"], dev["z"], None, dev["dy"], None, dev["dx"],
+                                       dev["ddelta"], dev["dA"], dev["dB"], dev["dC"], dev["dD"], dev["dz"],
+                                       dev["dbias"], None)
         elif wl.kind == "decode":
             ssm.ssm_state_step(dev["state"], dev["x"][0], dev["delta"][0], dev["A"], dev["B"][0],
                                dev["C"][0], dev["D"], dev["z"][0], dev["y"])
@@ -558,7 +613,7 @@ def run_ours(args):
     peaks = load_peaks()
     kern_s = kern_ms / 1e3
     gbs = wl.counts["bytes"] / kern_s / 1e9
-    if wl.kind == "scan":
+    if wl.kind in ("scan", "bwd"):
         peak_gexp = N_SM * MUFU_EX2_PER_CLK_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e9
         achieved = wl.counts["exps"] / kern_s / 1e9
         roof = dict(bound="alu", achieved=achieved, peak=peak_gexp, unit="Gexp/s",

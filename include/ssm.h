@@ -5,7 +5,8 @@
  *   ssm_selective_scan_fwd  the selective scan (S6) over a whole sequence;
  *   ssm_state_step          one decode token on a carried state, updated in place;
  *   ssm_causal_conv1d_fwd   the causal depthwise convolution + SiLU that feeds the scan;
- *   ssm_causal_conv1d_step  its one-token form on a carried window, updated in place.
+ *   ssm_causal_conv1d_step  its one-token form on a carried window, updated in place;
+ *   ssm_selective_scan_bwd  the gradients of the scan (training), states recomputed.
  *
  * The scan and the state step compute, per sequence b and channel d, with an N-wide fp32 state h:
  *     Delta_t = softplus(delta[b,d,t] + delta_bias[d])   (bias and softplus optional)
@@ -23,7 +24,8 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library keeps
  *    no state between calls.  ssm_selective_scan_fwd may take a temporary scratch
  *    buffer with cudaMallocAsync / cudaFreeAsync on cuda_stream (long sequences with
- *    few channels, see below); every other call allocates nothing.
+ *    few channels, see below), and so does ssm_selective_scan_bwd; every other call
+ *    allocates nothing.
  *  - Every pointer must be 16-byte aligned (SSM_ERR_ALIGNMENT otherwise).
  *  - The call is asynchronous on `cuda_stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and never synchronises.  Argument errors are returned before
@@ -193,6 +195,45 @@ int ssm_causal_conv1d_fwd(const void *x, const float *weight, const float *bias,
 int ssm_causal_conv1d_step(float *window, const void *x, const float *weight, const float *bias,
                            void *u, int batch, int dim, int width, int silu,
                            int in_dtype, int out_dtype, void *cuda_stream);
+
+/*
+ * Backward of the scan (Euler gain): the gradients of
+ *     loss = sum dy[b,d,t] * y[b,d,t] + sum dfinal_state[b,d,n] * final_state[b,d,n]
+ * with respect to every input of ssm_selective_scan_fwd_ex (zoh_exact = 0), for the
+ * training half that "Beyond attention with Mamba, state space models and hybrids"
+ * (xmarva lesson 10, section 6) describes: the states are recomputed in the backward pass,
+ * never stored.  Reverse-mode differentiation of the recurrence: with mu the adjoint
+ * flowing into h_t, lambda_n = dypre_t C_t[n] + mu_n, dC_t[n] += dypre_t h_t[n],
+ * dB_t[n] += lambda_n Delta_t x_t, dx_t = dypre_t D + sum_n lambda_n Delta_t B_t[n],
+ * dDelta_t = sum_n lambda_n (B_t[n] x_t + h_{t-1}[n] Abar_t[n] A[n]), dA[n] +=
+ * lambda_n h_{t-1}[n] Abar_t[n] Delta_t, mu_n <- Abar_t[n] lambda_n, where dypre_t =
+ * dy_t SiLU(z_t) and dz_t = dy_t ypre_t SiLU'(z_t).
+ *
+ *   inputs     : as ssm_selective_scan_fwd_ex (x, delta, z, B, C in in_dtype; A, D,
+ *                delta_bias, initial_state fp32; z, D, delta_bias, initial_state optional).
+ *   dy         : [batch][dim][seqlen], grad_dtype.
+ *   dfinal_state: [batch][dim][dstate] fp32 or NULL (zero).
+ *   dx, ddelta : [batch][dim][seqlen], grad_dtype, written (ddelta is the gradient of the
+ *                raw delta, through the bias and softplus).
+ *   dz         : [batch][dim][seqlen], grad_dtype, or NULL (requires z when given).
+ *   dB, dC     : [batch][seqlen][dstate], grad_dtype, written.
+ *   dA         : [dim][dstate] fp32, written.   dD, ddelta_bias: [dim] fp32 or NULL.
+ *   dinitial_state: [batch][dim][dstate] fp32 or NULL: the gradient of the start state.
+ * Sums over channels (dB, dC) and over sequences and positions (dA, dD, ddelta_bias) are
+ * formed from per-CTA partial sums added in a fixed order: results are deterministic.
+ * Takes a stream-ordered scratch buffer of about batch*dim'*(64*ceil(seqlen/32) + 4*seqlen
+ * + 72) bytes, dim' = dim rounded up to 32 (cudaMallocAsync / cudaFreeAsync on cuda_stream).
+ * dstate must be 1..16; zoh_exact has no backward here.
+ * seqlen = 0 writes zero parameter gradients and dinitial_state = dfinal_state.
+ */
+int ssm_selective_scan_bwd(const void *x, const void *delta, const float *delta_bias,
+                           int delta_softplus, const float *A, const void *B, const void *C,
+                           const float *D, const void *z, const float *initial_state,
+                           const void *dy, const float *dfinal_state,
+                           void *dx, void *ddelta, float *dA, void *dB, void *dC, float *dD,
+                           void *dz, float *ddelta_bias, float *dinitial_state,
+                           int batch, int dim, int seqlen, int dstate,
+                           int in_dtype, int grad_dtype, void *cuda_stream);
 
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char *ssm_status_string(int status);

@@ -57,6 +57,10 @@ def load_library(path: str | None = None):
         lib.ssm_causal_conv1d_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
         lib.ssm_causal_conv1d_step.restype = i
         lib.ssm_causal_conv1d_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+        lib.ssm_selective_scan_bwd.restype = i
+        lib.ssm_selective_scan_bwd.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, vp,
+                                               vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                               i, i, i, i, i, i, vp]
         lib.ssm_status_string.restype = ctypes.c_char_p
         lib.ssm_status_string.argtypes = [i]
         lib.ssm_version.restype = i
@@ -142,6 +146,46 @@ def ssm_state_step(state, x, delta, A, B, C, D, z, y, stream=None):
     _check(load_library().ssm_state_step(
         _ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(y),
         batch, dim, N, _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, state, y)))
+
+
+def ssm_selective_scan_bwd(x, delta, delta_bias, delta_softplus, A, B, C, D, z, initial_state,
+                           dy, dfinal_state, dx, ddelta, dA, dB, dC, dD, dz, ddelta_bias,
+                           dinitial_state, stream=None):
+    """Backward of the scan (see include/ssm.h).  Gradient tensors share dy's dtype
+    (dx, ddelta, dz, dB, dC); dA, dD, ddelta_bias, dinitial_state are fp32.  Optional
+    arguments are None.  Writes the gradients in place."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    _check(load_library().ssm_selective_scan_bwd(
+        _ptr(x), _ptr(delta), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(A), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), _ptr(initial_state), _ptr(dy), _ptr(dfinal_state),
+        _ptr(dx), _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz),
+        _ptr(ddelta_bias), _ptr(dinitial_state), batch, dim, L, N,
+        _DTYPE_CODE[x.dtype], _DTYPE_CODE[dy.dtype], _stream(stream, x, dy)))
+
+
+def selective_scan_bwd(dy, x, delta, A, B, C, D=None, z=None, delta_bias=None,
+                       delta_softplus=False, initial_state=None, dfinal_state=None, stream=None):
+    """Allocate the gradients with torch (dy's dtype for the tensor gradients) and run the
+    backward; returns a dict dx, ddelta, dz, dA, dB, dC, dD, ddelta_bias, dinitial_state
+    (None where the input was absent)."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    dev, gd, f32 = x.device, dy.dtype, torch.float32
+    g = dict(dx=torch.empty((batch, dim, L), device=dev, dtype=gd),
+             ddelta=torch.empty((batch, dim, L), device=dev, dtype=gd),
+             dz=None if z is None else torch.empty((batch, dim, L), device=dev, dtype=gd),
+             dA=torch.empty((dim, N), device=dev, dtype=f32),
+             dB=torch.empty((batch, L, N), device=dev, dtype=gd),
+             dC=torch.empty((batch, L, N), device=dev, dtype=gd),
+             dD=None if D is None else torch.empty(dim, device=dev, dtype=f32),
+             ddelta_bias=None if delta_bias is None else torch.empty(dim, device=dev, dtype=f32),
+             dinitial_state=None if initial_state is None else
+             torch.empty((batch, dim, N), device=dev, dtype=f32))
+    ssm_selective_scan_bwd(x, delta, delta_bias, delta_softplus, A, B, C, D, z, initial_state,
+                           dy, dfinal_state, g["dx"], g["ddelta"], g["dA"], g["dB"], g["dC"],
+                           g["dD"], g["dz"], g["ddelta_bias"], g["dinitial_state"], stream)
+    return g
 
 
 def ssm_causal_conv1d_fwd(x, weight, bias, initial_window, u, final_window, silu=True,

@@ -1,4 +1,4 @@
-// common.cuh -- small device helpers shared by the scan and decode kernels.
+// common.cuh -- small device helpers shared by the scan, decode and convolution kernels.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -75,6 +75,40 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
+// 8 consecutive values of a staged row as fp32 (16-byte aligned source).
+template <typename T> __device__ __forceinline__ void load8(const T *src, float (&v)[8]);
+template <> __device__ __forceinline__ void load8<float>(const float *src, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(src);
+    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <> __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *src, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(src);
+    const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {            // bf16 -> fp32 is a 16-bit left shift
+        v[2 * k] = __uint_as_float(w[k] << 16);
+        v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+}
+
+// 8 fp32 values stored as 8 values of T (16-byte aligned destination).
+template <typename T> __device__ __forceinline__ void store8(T *dst, const float (&v)[8]);
+template <> __device__ __forceinline__ void store8<float>(float *dst, const float (&v)[8]) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <> __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16 *dst, const float (&v)[8]) {
+    unsigned w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<const unsigned *>(&p);
+    }
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // 16-byte asynchronous global -> shared copy (bypasses L1), grouped with commit/wait.
 __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gmem_src) {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
@@ -87,37 +121,5 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N> __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
-
-// Sum of per-lane partials over the G lanes that share one channel (G consecutive lanes),
-// "transposed": on entry each lane holds partial sums p[0..G) for G consecutive
-// timesteps; on exit lane r of the group holds the full sum for timestep r.  Costs
-// G-1 shuffles per G timesteps instead of G*log2(G) for G separate butterflies.
-template <int G> struct GroupReduceScatter;
-
-template <> struct GroupReduceScatter<1> {
-    __device__ __forceinline__ static float run(const float *p, int) { return p[0]; }
-};
-
-template <> struct GroupReduceScatter<2> {
-    __device__ __forceinline__ static float run(const float *p, int r) {
-        const float send = (r & 1) ? p[0] : p[1];
-        const float keep = (r & 1) ? p[1] : p[0];
-        return keep + __shfl_xor_sync(0xffffffffu, send, 1);
-    }
-};
-
-template <> struct GroupReduceScatter<4> {
-    __device__ __forceinline__ static float run(const float *p, int r) {
-        const bool hi = (r & 2) != 0;
-        const float s0 = hi ? p[0] : p[2], s1 = hi ? p[1] : p[3];
-        const float k0 = hi ? p[2] : p[0], k1 = hi ? p[3] : p[1];
-        const float q0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 2);
-        const float q1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 2);
-        const bool lo = (r & 1) != 0;
-        const float send = lo ? q0 : q1;
-        const float keep = lo ? q1 : q0;
-        return keep + __shfl_xor_sync(0xffffffffu, send, 1);
-    }
-};
 
 }  // namespace ssm

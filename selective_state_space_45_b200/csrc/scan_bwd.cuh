@@ -1,0 +1,604 @@
+// scan_bwd.cuh -- backward of the selective scan (S6, Euler gain) for sm_100a.
+//
+// Gradients of  loss = sum dy * y + sum dfinal * h_last  with respect to x, delta, z, A,
+// B, C, D, delta_bias and the start state, by reverse-mode differentiation of the
+// recurrence (forward: scan_fwd.cuh).  With mu the adjoint flowing into h_t from later
+// tokens, going t = L-1 .. 0:
+//     dypre_t  = dy_t * SiLU(z_t);   dz_t = dy_t * ypre_t * SiLU'(z_t)
+//     lambda_n = dypre_t C_t[n] + mu_n                      (adjoint of h_t[n])
+//     dC_t[n] += dypre_t h_t[n];     dB_t[n] += lambda_n Delta_t x_t
+//     dx_t     = dypre_t D + sum_n lambda_n Delta_t B_t[n]
+//     dDelta_t = sum_n lambda_n (B_t[n] x_t + h_{t-1}[n] Abar_t[n] A[n])
+//     dA[n]   += lambda_n h_{t-1}[n] Abar_t[n] Delta_t;     mu_n = Abar_t[n] lambda_n
+// and ddelta_t = dDelta_t * sigmoid(delta_t + bias) under softplus.
+// Source: the states are recomputed in the backward pass rather than stored, as Mamba's own
+// kernel does ("Beyond attention with Mamba, state space models and hybrids", xmarva
+// lesson 10, section 6); the recurrence is the one of sections 3-4 of that lesson.
+//
+// Layout of the work (one CTA = 32 channels x 16 states of one sequence, 4 warps, one
+// channel per lane and one state quad per warp, as in the forward kernel):
+//   phase F   the forward recurrence over the whole sequence, keeping only the state at
+//             every tile start (a global scratch array, mostly L2-resident);
+//   phase R   tiles in reverse.  Per tile: (R1) recompute the tile forward from its
+//             checkpoint, keeping the state before every 4th token in registers and the
+//             per-quad readout in shared memory; (R2) per (t, d): the pre-gate output,
+//             dy * SiLU(z) and dz; (R3) sub-chunks of 4 tokens in reverse: recompute their
+//             states from the register checkpoint, then walk them backwards carrying mu;
+//             the dB / dC terms of the 32 channels are summed through a per-warp shared
+//             transpose and written as per-CTA partial sums; (R4) per (t, d): the quads'
+//             dx and dDelta partials summed, the softplus slope, 16-byte row stores.
+//   Partial sums over channel groups (dB, dC) and over sequences (dA, dD, dbias) are
+//   added up by reduce_partials_kernel in a fixed order: the gradients are deterministic.
+#pragma once
+
+#include "common.cuh"
+
+namespace ssm {
+
+// sigmoid(v) = 1 / (1 + e^-v) with the SFU exponential and reciprocal (0 for v -> -inf).
+__device__ __forceinline__ float sigmoid_f(float v) {
+    return rcp_approx(1.f + ex2_approx(-v * kLog2e));
+}
+
+struct BwdArgs {
+    const void *x;
+    const void *delta;
+    const float *delta_bias;
+    const float *A;
+    const void *B;
+    const void *C;
+    const float *D;
+    const void *z;
+    const float *h0;      // [batch][dim][dstate] or null (zero start)
+    const void *dy;       // [batch][dim][L], gradient dtype
+    const float *dfinal;  // [batch][dim][dstate] or null
+    void *dx;
+    void *ddelta;
+    void *dz;             // written when given (z must be given too)
+    float *dh0;           // [batch][dim][dstate] or null
+    float *ck;            // [ctas][ntiles][4][32] float4: state at every tile start
+    float *part_bc;       // [2][ctas][L][16]: per-CTA channel sums of the dB and dC terms
+    float *part_a;        // [batch][dim][16]: per-sequence dA
+    float *part_dd;       // [2][batch][dim]: per-sequence dD and ddelta_bias
+    int batch, dim, seqlen, dstate;
+    int softplus;
+    int groups_per_seq;
+    int ntiles;
+};
+
+template <typename Tin_, typename Tg_, bool VEC_>
+struct BwdCfg {
+    using Tin = Tin_;
+    using Tg = Tg_;
+    static constexpr int NP = 16, Q = 4, CH = 32, T = 32, NSTAGE = 2, NT = 128;
+    static constexpr bool VEC = VEC_;
+    static constexpr int EIN = 16 / sizeof(Tin);
+    static constexpr int EG = 16 / sizeof(Tg);
+    static constexpr int RAW_ROW = T + EIN;     // staged rows: 16 B past a multiple of 16 B
+    static constexpr int G_ROW = T + EG;
+    static constexpr int P_ROW = T + 4;         // per-quad partial rows (floats)
+    static constexpr int X_ROW = 36;            // transpose rows: conflict-free both ways
+    static constexpr int T8 = T / 8;
+    static_assert(CH * T8 == NT, "one (channel, 8-token chunk) task per thread");
+
+    static constexpr size_t al(size_t v) { return (v + 15) & ~size_t(15); }
+    static constexpr size_t RAW_ARR = al(size_t(CH) * RAW_ROW * sizeof(Tin));
+    static constexpr size_t G_ARR = al(size_t(CH) * G_ROW * sizeof(Tg));
+    static constexpr size_t RAW_BC = al(size_t(T) * NP * sizeof(Tin));
+    static constexpr size_t STAGE_BYTES = 3 * RAW_ARR + G_ARR + 2 * RAW_BC;
+    static constexpr size_t OFF_RAW = 0;
+    static constexpr size_t OFF_PREP = OFF_RAW + NSTAGE * STAGE_BYTES;   // float4 [T][CH]
+    static constexpr size_t OFF_BF = OFF_PREP + al(size_t(T) * CH * sizeof(float4));
+    static constexpr size_t OFF_CF = OFF_BF + al(size_t(T) * NP * sizeof(float));
+    static constexpr size_t PART_ARR = al(size_t(Q) * CH * P_ROW * sizeof(float));
+    static constexpr size_t OFF_PART = OFF_CF + al(size_t(T) * NP * sizeof(float));
+    static constexpr size_t OFF_XP = OFF_PART + 2 * PART_ARR;
+    static constexpr size_t SMEM_BYTES = OFF_XP + al(size_t(Q) * 32 * X_ROW * sizeof(float));
+    // the staged dx / ddelta / dz rows reuse the partial arrays once they are summed
+    static_assert(3 * CH * G_ROW * sizeof(Tg) <= 2 * PART_ARR, "output staging must fit");
+};
+
+// Views of one ring stage: x, delta, z rows [CH][RAW_ROW], dy rows [CH][G_ROW], B, C [T][N].
+template <class Cfg> struct BwdStage {
+    typename Cfg::Tin *xs, *ds, *zs, *bs, *cs;
+    typename Cfg::Tg *gs;
+    __device__ __forceinline__ BwdStage(unsigned char *smem, int s) {
+        unsigned char *base = smem + Cfg::OFF_RAW + size_t(s) * Cfg::STAGE_BYTES;
+        xs = reinterpret_cast<typename Cfg::Tin *>(base);
+        ds = reinterpret_cast<typename Cfg::Tin *>(base + Cfg::RAW_ARR);
+        zs = reinterpret_cast<typename Cfg::Tin *>(base + 2 * Cfg::RAW_ARR);
+        gs = reinterpret_cast<typename Cfg::Tg *>(base + 3 * Cfg::RAW_ARR);
+        bs = reinterpret_cast<typename Cfg::Tin *>(base + 3 * Cfg::RAW_ARR + Cfg::G_ARR);
+        cs = reinterpret_cast<typename Cfg::Tin *>(base + 3 * Cfg::RAW_ARR + Cfg::G_ARR + Cfg::RAW_BC);
+    }
+};
+
+// Stage tile [t0, t0 + T): x, delta and B always; z, dy and C when `full` (phase R).
+// VEC: 16-byte cp.async chunks, each wholly inside or outside [0, L) (L is a multiple of
+// both chunk widths); else guarded scalar copies.
+template <class Cfg>
+__device__ __forceinline__ void bwd_load_tile(const BwdArgs &p, unsigned char *smem, int st, int t0,
+                                              size_t row0, size_t bc0, int nch, bool full) {
+    using Tin = typename Cfg::Tin;
+    using Tg = typename Cfg::Tg;
+    constexpr int CH = Cfg::CH, T = Cfg::T, NT = Cfg::NT, EIN = Cfg::EIN, EG = Cfg::EG, NP = Cfg::NP;
+    BwdStage<Cfg> s(smem, st);
+    const int L = p.seqlen, N = p.dstate;
+    const Tin *gx = static_cast<const Tin *>(p.x) + row0;
+    const Tin *gd = static_cast<const Tin *>(p.delta) + row0;
+    const Tin *gz = p.z ? static_cast<const Tin *>(p.z) + row0 : gx;
+    const Tg *gg = static_cast<const Tg *>(p.dy) + row0;
+    const int narr = full ? (p.z ? 3 : 2) : 2;
+    const int nbc = full ? 2 : 1;
+    const Tin *gb = static_cast<const Tin *>(p.B) + bc0 + size_t(t0) * N;
+    const Tin *gc = static_cast<const Tin *>(p.C) + bc0 + size_t(t0) * N;
+    if constexpr (Cfg::VEC) {
+        constexpr int CPR = T / EIN;
+        constexpr int ROWC = 3 * CH * CPR;
+#pragma unroll
+        for (int k = 0; k < (ROWC + NT - 1) / NT; ++k) {
+            const int i = tid_x() + k * NT;
+            const int a = i / (CH * CPR);
+            const int rem = i % (CH * CPR);
+            const int cc = rem / CPR, qq = rem % CPR;
+            if (i < ROWC && a < narr && cc < nch && t0 + qq * EIN < L) {
+                const Tin *src = (a == 0 ? gx : a == 1 ? gd : gz) + size_t(cc) * L + t0 + qq * EIN;
+                Tin *dst = (a == 0 ? s.xs : a == 1 ? s.ds : s.zs) + cc * Cfg::RAW_ROW + qq * EIN;
+                cp_async_16(dst, src);
+            }
+        }
+        if (full) {
+            constexpr int CPRG = T / EG;
+#pragma unroll
+            for (int k = 0; k < (CH * CPRG + NT - 1) / NT; ++k) {
+                const int i = tid_x() + k * NT;
+                const int cc = i / CPRG, qq = i % CPRG;
+                if (i < CH * CPRG && cc < nch && t0 + qq * EG < L)
+                    cp_async_16(s.gs + cc * Cfg::G_ROW + qq * EG, gg + size_t(cc) * L + t0 + qq * EG);
+            }
+        }
+        if (N == NP) {
+            constexpr int BCC = T * NP / EIN;
+#pragma unroll
+            for (int k = 0; k < (2 * BCC + NT - 1) / NT; ++k) {
+                const int i = tid_x() + k * NT;
+                const int which = i / BCC, qq = i % BCC;
+                if (i < 2 * BCC && which < nbc && t0 + (qq * EIN) / NP < L)
+                    cp_async_16((which ? s.cs : s.bs) + qq * EIN, (which ? gc : gb) + qq * EIN);
+            }
+        } else {
+            const int valid_t = min(T, L - t0);
+            const int bc_chunks = (valid_t * N * int(sizeof(Tin))) / 16;
+            for (int i = tid_x(); i < nbc * bc_chunks; i += NT) {
+                const int which = i >= bc_chunks;
+                const int qq = i - which * bc_chunks;
+                cp_async_16((which ? s.cs : s.bs) + qq * EIN, (which ? gc : gb) + qq * EIN);
+            }
+        }
+    } else {
+        constexpr int NEL = 3 * CH * T;
+#pragma unroll 4
+        for (int k = 0; k < (NEL + NT - 1) / NT; ++k) {
+            const int i = tid_x() + k * NT;
+            const int a = i / (CH * T);
+            const int rem = i % (CH * T);
+            const int cc = rem / T, tt = rem % T;
+            if (i < NEL && a < narr && cc < nch && t0 + tt < L) {
+                const Tin *src = (a == 0 ? gx : a == 1 ? gd : gz) + size_t(cc) * L + t0 + tt;
+                Tin *dst = (a == 0 ? s.xs : a == 1 ? s.ds : s.zs) + cc * Cfg::RAW_ROW + tt;
+                *dst = *src;
+            }
+        }
+        if (full) {
+            for (int i = tid_x(); i < CH * T; i += NT) {
+                const int cc = i / T, tt = i % T;
+                if (cc < nch && t0 + tt < L) s.gs[cc * Cfg::G_ROW + tt] = gg[size_t(cc) * L + t0 + tt];
+            }
+        }
+        const int nel = min(T, L - t0) * N;
+        for (int i = tid_x(); i < nbc * nel; i += NT) {
+            const int which = i >= nel;
+            const int qq = i - which * nel;
+            (which ? s.cs : s.bs)[qq] = (which ? gc : gb)[qq];
+        }
+    }
+}
+
+
+// Per-(t, d) task of this thread: channel cc, tokens 8*t8 .. 8*t8+7 of the tile.  Writes
+// prep[t][cc] = (Delta_t, x_t, 0, 0); tokens past L and channels past dim become no-op
+// tokens (Delta = 0, x = 0: the state passes through unchanged, no gradient arises).
+template <class Cfg>
+__device__ __forceinline__ void bwd_prep(const BwdArgs &p, const BwdStage<Cfg> &sv, float4 *prep,
+                                         int cc, int t8, bool cvalid, float bias, int t0) {
+    using Tin = typename Cfg::Tin;
+    constexpr int CH = Cfg::CH;
+    float dr[8], xr[8];
+    load8<Tin>(sv.ds + cc * Cfg::RAW_ROW + 8 * t8, dr);
+    load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        float dl = dr[u] + bias;
+        if (p.softplus) dl = softplus_f(dl);
+        const bool ok = cvalid && t0 + 8 * t8 + u < p.seqlen;
+        prep[(8 * t8 + u) * CH + cc] = make_float4(ok ? dl : 0.f, ok ? xr[u] : 0.f, 0.f, 0.f);
+    }
+}
+
+// B (and C when `both`) of the tile widened to fp32 [T][NP], zero past dstate and past L.
+template <class Cfg>
+__device__ __forceinline__ void bwd_widen_bc(const BwdArgs &p, const BwdStage<Cfg> &sv, float *Bf,
+                                             float *Cf, int t0, bool both) {
+    constexpr int T = Cfg::T, NP = Cfg::NP, NT = Cfg::NT;
+    const int L = p.seqlen, N = p.dstate;
+#pragma unroll
+    for (int k = 0; k < (T * NP + NT - 1) / NT; ++k) {
+        const int i = tid_x() + k * NT;
+        if (i < T * NP) {
+            const int tt = i / NP, n = i % NP;
+            const bool ok = n < N && t0 + tt < L;
+            Bf[i] = ok ? to_f32(sv.bs[tt * N + n]) : 0.f;
+            if (both) Cf[i] = ok ? to_f32(sv.cs[tt * N + n]) : 0.f;
+        }
+    }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
+    using Tin = typename Cfg::Tin;
+    using Tg = typename Cfg::Tg;
+    constexpr int NP = Cfg::NP, Q = Cfg::Q, CH = Cfg::CH, T = Cfg::T, NT = Cfg::NT;
+    extern __shared__ __align__(16) unsigned char smem[];
+
+    const int tid = threadIdx.x;
+    const int q = tid >> 5, lane = tid & 31, c = lane;
+    const int cta = blockIdx.x;
+    const int ctas = gridDim.x;
+    const int b = cta / p.groups_per_seq;
+    const int d0 = (cta - b * p.groups_per_seq) * CH;
+    const int L = p.seqlen, N = p.dstate, dim = p.dim, ntiles = p.ntiles;
+    const int nch = min(CH, dim - d0);
+    const bool dvalid = c < nch;
+
+    float4 *prep = reinterpret_cast<float4 *>(smem + Cfg::OFF_PREP);
+    float *Bf = reinterpret_cast<float *>(smem + Cfg::OFF_BF);
+    float *Cf = reinterpret_cast<float *>(smem + Cfg::OFF_CF);
+    float *part0 = reinterpret_cast<float *>(smem + Cfg::OFF_PART);
+    float *part1 = part0 + Cfg::PART_ARR / sizeof(float);
+    float *xp = reinterpret_cast<float *>(smem + Cfg::OFF_XP) + q * 32 * Cfg::X_ROW;
+
+    float Af[4], A2[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const int n = 4 * q + s;
+        Af[s] = (dvalid && n < N) ? p.A[size_t(d0 + c) * N + n] : 0.f;
+        A2[s] = Af[s] * kLog2e;
+    }
+    // this thread's (t, d) task: channel cc, 8-token chunk t8 of every tile
+    const int cc = tid % CH, t8 = tid / CH;
+    const bool cvalid = cc < nch;
+    const float tbias = (p.delta_bias != nullptr && cvalid) ? p.delta_bias[d0 + cc] : 0.f;
+    const float tD = (p.D != nullptr && cvalid) ? p.D[d0 + cc] : 0.f;
+
+    const size_t row0 = (size_t(b) * dim + d0) * size_t(L);
+    const size_t bc0 = size_t(b) * L * size_t(N);
+    const size_t chrow = size_t(b) * dim + d0 + c;
+    float4 *ck = reinterpret_cast<float4 *>(p.ck) + (size_t(cta) * ntiles * Q + q) * 32 + lane;
+
+    // ---------------- phase F: forward, keeping the state at every tile start ----------------
+    float h[4] = {0.f, 0.f, 0.f, 0.f};
+    if (p.h0 != nullptr && dvalid) {
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            if (4 * q + s < N) h[s] = p.h0[chrow * N + 4 * q + s];
+    }
+    bwd_load_tile<Cfg>(p, smem, 0, 0, row0, bc0, nch, false);
+    cp_async_commit();
+    for (int tile = 0; tile < ntiles; ++tile) {
+        const int t0 = tile * T;
+        ck[size_t(tile) * Q * 32] = make_float4(h[0], h[1], h[2], h[3]);
+        cp_async_wait<0>();
+        __syncthreads();
+        if (tile + 1 < ntiles) bwd_load_tile<Cfg>(p, smem, (tile + 1) & 1, t0 + T, row0, bc0, nch, false);
+        cp_async_commit();
+        const BwdStage<Cfg> sv(smem, tile & 1);
+        bwd_prep<Cfg>(p, sv, prep, cc, t8, cvalid, tbias, t0);
+        bwd_widen_bc<Cfg>(p, sv, Bf, Cf, t0, false);
+        __syncthreads();
+#pragma unroll 8
+        for (int t = 0; t < T; ++t) {
+            const float4 pv = prep[t * CH + c];
+            const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
+            const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+            const float dx = pv.x * pv.y;
+#pragma unroll
+            for (int s = 0; s < 4; ++s) h[s] = fmaf(ex2_approx(pv.x * A2[s]), h[s], dx * bb[s]);
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // ---------------- phase R: tiles in reverse ----------------
+    float mu[4] = {0.f, 0.f, 0.f, 0.f};
+    if (p.dfinal != nullptr && dvalid) {
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            if (4 * q + s < N) mu[s] = p.dfinal[chrow * N + 4 * q + s];
+    }
+    float dA_acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float dD_acc = 0.f, db_acc = 0.f;          // this thread's task channel, over its chunks
+    float *dxp = part0 + (q * CH + c) * Cfg::P_ROW;    // per-quad partials of this lane
+    float *ddp = part1 + (q * CH + c) * Cfg::P_ROW;
+    float *xrow = xp + lane * Cfg::X_ROW;
+    const size_t bc_stride = size_t(ctas) * L * NP;    // dB block -> dC block of part_bc
+    float *pbc = p.part_bc + size_t(cta) * L * NP;
+
+    bwd_load_tile<Cfg>(p, smem, 0, (ntiles - 1) * T, row0, bc0, nch, true);
+    cp_async_commit();
+    for (int r = 0; r < ntiles; ++r) {
+        const int tile = ntiles - 1 - r;
+        const int t0 = tile * T;
+        cp_async_wait<0>();
+        __syncthreads();
+        if (tile > 0) bwd_load_tile<Cfg>(p, smem, (r + 1) & 1, t0 - T, row0, bc0, nch, true);
+        cp_async_commit();
+        const BwdStage<Cfg> sv(smem, r & 1);
+        bwd_prep<Cfg>(p, sv, prep, cc, t8, cvalid, tbias, t0);
+        bwd_widen_bc<Cfg>(p, sv, Bf, Cf, t0, true);
+        __syncthreads();
+
+        // R1: the tile forward again from its checkpoint; the state before every 4th token
+        // stays in registers, the per-quad readout goes to part0
+        float sub[T / 4][4];
+        {
+            const float4 hv = ck[size_t(tile) * Q * 32];
+            float hh[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+            for (int g = 0; g < T / 4; ++g) {
+#pragma unroll
+                for (int s = 0; s < 4; ++s) sub[g][s] = hh[s];
+                float out[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int t = 4 * g + u;
+                    const float4 pv = prep[t * CH + c];
+                    const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
+                    const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
+                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+                    const float cb[4] = {cq.x, cq.y, cq.z, cq.w};
+                    const float dx = pv.x * pv.y;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        hh[s] = fmaf(ex2_approx(pv.x * A2[s]), hh[s], dx * bb[s]);
+                        acc = fmaf(cb[s], hh[s], acc);
+                    }
+                    out[u] = acc;
+                }
+                *reinterpret_cast<float4 *>(dxp + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
+            }
+        }
+        __syncthreads();
+
+        // R2: per (t, d): pre-gate output, dypre = dy * SiLU(z), dz -> prep[t][cc].zw
+        {
+            float acc[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < Q; ++qq) {
+                const float *src = part0 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
+                const float4 a0 = *reinterpret_cast<const float4 *>(src);
+                const float4 a1 = *reinterpret_cast<const float4 *>(src + 4);
+                acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
+                acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
+            }
+            float xr[8], gr[8], zr[8];
+            load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+            load8<Tg>(sv.gs + cc * Cfg::G_ROW + 8 * t8, gr);
+            if (p.z != nullptr) load8<Tin>(sv.zs + cc * Cfg::RAW_ROW + 8 * t8, zr);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool ok = cvalid && t0 + 8 * t8 + u < L;
+                const float ypre = fmaf(tD, xr[u], acc[u]);
+                float dyp = gr[u], dzv = 0.f;
+                if (p.z != nullptr) {
+                    const float sg = sigmoid_f(zr[u]);
+                    dzv = gr[u] * ypre * sg * fmaf(zr[u], 1.f - sg, 1.f);
+                    dyp = gr[u] * zr[u] * sg;
+                }
+                *reinterpret_cast<float2 *>(reinterpret_cast<float *>(prep + (8 * t8 + u) * CH + cc) + 2) =
+                    make_float2(ok ? dyp : 0.f, ok ? dzv : 0.f);
+            }
+        }
+        __syncthreads();
+
+        // R3: sub-chunks of 4 tokens, last first: recompute their states, walk them back
+#pragma unroll 1
+        for (int j = T / 4 - 1; j >= 0; --j) {
+            float hs[5][4], a[4][4], dl[4], xv[4], dyp[4];
+#pragma unroll
+            for (int s = 0; s < 4; ++s) hs[0][s] = sub[j][s];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int t = 4 * j + u;
+                const float4 pv = prep[t * CH + c];
+                dl[u] = pv.x; xv[u] = pv.y; dyp[u] = pv.z;
+                const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
+                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+                const float dx = dl[u] * xv[u];
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    a[u][s] = ex2_approx(dl[u] * A2[s]);
+                    hs[u + 1][s] = fmaf(a[u][s], hs[u][s], dx * bb[s]);
+                }
+            }
+            float dxo[4], ddo[4];
+#pragma unroll
+            for (int u = 3; u >= 0; --u) {
+                const int t = 4 * j + u;
+                const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
+                const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
+                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+                const float cb[4] = {cq.x, cq.y, cq.z, cq.w};
+                const float dlx = dl[u] * xv[u];
+                float dxa = 0.f, dda = 0.f, vb[4], vc[4];
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const float lam = fmaf(dyp[u], cb[s], mu[s]);
+                    const float ha = hs[u][s] * a[u][s];         // h_{t-1} * Abar_t
+                    vb[s] = lam * dlx;                           // dB term
+                    vc[s] = dyp[u] * hs[u + 1][s];               // dC term
+                    dxa = fmaf(lam, bb[s], dxa);
+                    dda = fmaf(lam, fmaf(bb[s], xv[u], ha * Af[s]), dda);
+                    dA_acc[s] = fmaf(lam * ha, dl[u], dA_acc[s]);
+                    mu[s] = a[u][s] * lam;
+                }
+                dxo[u] = dxa * dl[u];
+                ddo[u] = dda;
+                *reinterpret_cast<float4 *>(xrow + 8 * u) = make_float4(vb[0], vb[1], vb[2], vb[3]);
+                *reinterpret_cast<float4 *>(xrow + 8 * u + 4) = make_float4(vc[0], vc[1], vc[2], vc[3]);
+            }
+            *reinterpret_cast<float4 *>(dxp + 4 * j) = make_float4(dxo[0], dxo[1], dxo[2], dxo[3]);
+            *reinterpret_cast<float4 *>(ddp + 4 * j) = make_float4(ddo[0], ddo[1], ddo[2], ddo[3]);
+            __syncwarp();
+            // column `lane` of the warp's transpose: value (token u, B or C, state s) summed
+            // over the 32 channels
+            float sum = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) sum += xp[rr * Cfg::X_ROW + lane];
+            __syncwarp();
+            const int u = lane >> 3, which = (lane >> 2) & 1, st = lane & 3;
+            const int tok = t0 + 4 * j + u;
+            if (tok < L && 4 * q + st < N)
+                pbc[which * bc_stride + size_t(tok) * NP + 4 * q + st] = sum;
+        }
+        __syncthreads();
+
+        // R4: per (t, d): sum the quads' dx and dDelta partials, skip term, softplus slope
+        {
+            float dxs[8], dds[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) { dxs[u] = 0.f; dds[u] = 0.f; }
+#pragma unroll
+            for (int qq = 0; qq < Q; ++qq) {
+                const float *s0 = part0 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
+                const float *s1 = part1 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
+                const float4 a0 = *reinterpret_cast<const float4 *>(s0);
+                const float4 a1 = *reinterpret_cast<const float4 *>(s0 + 4);
+                const float4 b0 = *reinterpret_cast<const float4 *>(s1);
+                const float4 b1 = *reinterpret_cast<const float4 *>(s1 + 4);
+                dxs[0] += a0.x; dxs[1] += a0.y; dxs[2] += a0.z; dxs[3] += a0.w;
+                dxs[4] += a1.x; dxs[5] += a1.y; dxs[6] += a1.z; dxs[7] += a1.w;
+                dds[0] += b0.x; dds[1] += b0.y; dds[2] += b0.z; dds[3] += b0.w;
+                dds[4] += b1.x; dds[5] += b1.y; dds[6] += b1.z; dds[7] += b1.w;
+            }
+            float xr[8], dr[8], dzv[8];
+            load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+            load8<Tin>(sv.ds + cc * Cfg::RAW_ROW + 8 * t8, dr);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float4 pv = prep[(8 * t8 + u) * CH + cc];
+                const bool ok = cvalid && t0 + 8 * t8 + u < L;
+                dxs[u] = fmaf(pv.z, tD, dxs[u]);
+                if (p.softplus) dds[u] *= sigmoid_f(dr[u] + tbias);
+                dds[u] = ok ? dds[u] : 0.f;          // no-op tokens carry no step gradient
+                dzv[u] = pv.w;
+                dD_acc = fmaf(pv.z, ok ? xr[u] : 0.f, dD_acc);
+                db_acc += dds[u];
+            }
+            __syncthreads();                         // the partials are read: reuse as staging
+            Tg *ox = reinterpret_cast<Tg *>(part0);
+            Tg *od = ox + CH * Cfg::G_ROW;
+            Tg *oz = od + CH * Cfg::G_ROW;
+            store8<Tg>(ox + cc * Cfg::G_ROW + 8 * t8, dxs);
+            store8<Tg>(od + cc * Cfg::G_ROW + 8 * t8, dds);
+            if (p.z != nullptr) store8<Tg>(oz + cc * Cfg::G_ROW + 8 * t8, dzv);
+        }
+        __syncthreads();
+
+        // dx, ddelta, dz rows of the tile back to global memory (coalesced)
+        {
+            const Tg *ox = reinterpret_cast<const Tg *>(part0);
+            const int narr = p.dz != nullptr ? 3 : 2;
+            if constexpr (Cfg::VEC) {
+                constexpr int CPR = T / Cfg::EG;
+#pragma unroll
+                for (int k = 0; k < (3 * CH * CPR + NT - 1) / NT; ++k) {
+                    const int i = tid + k * NT;
+                    const int a = i / (CH * CPR);
+                    const int rem = i % (CH * CPR);
+                    const int ch = rem / CPR, qq = rem % CPR;
+                    const int tg = t0 + qq * Cfg::EG;
+                    if (i < 3 * CH * CPR && a < narr && ch < nch && tg < L) {
+                        Tg *dst = static_cast<Tg *>(a == 0 ? p.dx : a == 1 ? p.ddelta : p.dz) + row0 +
+                                  size_t(ch) * L + tg;
+                        *reinterpret_cast<uint4 *>(dst) =
+                            *reinterpret_cast<const uint4 *>(ox + (a * CH + ch) * Cfg::G_ROW + qq * Cfg::EG);
+                    }
+                }
+            } else {
+                for (int i = tid; i < narr * CH * T; i += NT) {
+                    const int a = i / (CH * T);
+                    const int rem = i % (CH * T);
+                    const int ch = rem / T, tt = rem % T;
+                    if (ch < nch && t0 + tt < L) {
+                        Tg *dst = static_cast<Tg *>(a == 0 ? p.dx : a == 1 ? p.ddelta : p.dz) + row0 +
+                                  size_t(ch) * L + t0 + tt;
+                        *dst = ox[(a * CH + ch) * Cfg::G_ROW + tt];
+                    }
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+
+    // per-sequence partials: dA of this lane's states; dD and ddelta_bias of the channels
+    if (dvalid) {
+        *reinterpret_cast<float4 *>(p.part_a + chrow * NP + 4 * q) =
+            make_float4(dA_acc[0], dA_acc[1], dA_acc[2], dA_acc[3]);
+        if (p.dh0 != nullptr) {
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                if (4 * q + s < N) p.dh0[chrow * N + 4 * q + s] = mu[s];
+        }
+    }
+    __syncthreads();
+    float *red = reinterpret_cast<float *>(prep);   // [2][T8][CH]
+    red[t8 * CH + cc] = dD_acc;
+    red[(Cfg::T8 + t8) * CH + cc] = db_acc;
+    __syncthreads();
+    if (tid < nch) {
+        float sd = 0.f, sb = 0.f;
+#pragma unroll
+        for (int k = 0; k < Cfg::T8; ++k) {
+            sd += red[k * CH + tid];
+            sb += red[(Cfg::T8 + k) * CH + tid];
+        }
+        const size_t bd = size_t(b) * dim + d0 + tid;
+        p.part_dd[bd] = sd;
+        p.part_dd[size_t(p.batch) * dim + bd] = sb;
+    }
+}
+
+// out[(i*R + r)*Nout + n] = sum_{k<K} in[((i*K + k)*R + r)*NPin + n] for n < Nout, summed
+// in k order (deterministic).  One thread per output element.
+template <typename To>
+__global__ void __launch_bounds__(256)
+reduce_partials_kernel(const float *__restrict__ in, To *__restrict__ out, long long outer, int K,
+                       long long R, int NPin, int Nout) {
+    const long long total = outer * R * Nout;
+    for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+         e += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long n = e % Nout;
+        const long long ir = e / Nout;                 // i * R + r
+        const long long i = ir / R, r = ir - i * R;
+        const float *src = in + ((i * K) * R + r) * NPin + n;
+        float acc = 0.f;
+        for (int k = 0; k < K; ++k) acc += src[static_cast<long long>(k) * R * NPin];
+        out[e] = from_f32<To>(acc);
+    }
+}
+
+
+}  // namespace ssm

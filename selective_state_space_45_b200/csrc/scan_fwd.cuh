@@ -119,40 +119,6 @@ template <class Cfg> struct Stage {
     }
 };
 
-// 8 consecutive values of a staged row as fp32 (16-byte aligned source).
-template <typename T> __device__ __forceinline__ void load8(const T *src, float (&v)[8]);
-template <> __device__ __forceinline__ void load8<float>(const float *src, float (&v)[8]) {
-    const float4 a = *reinterpret_cast<const float4 *>(src);
-    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-template <> __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *src, float (&v)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(src);
-    const unsigned w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {            // bf16 -> fp32 is a 16-bit left shift
-        v[2 * k] = __uint_as_float(w[k] << 16);
-        v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-    }
-}
-
-// 8 fp32 values stored as 8 values of T (16-byte aligned destination).
-template <typename T> __device__ __forceinline__ void store8(T *dst, const float (&v)[8]);
-template <> __device__ __forceinline__ void store8<float>(float *dst, const float (&v)[8]) {
-    *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4 *>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
-}
-template <> __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16 *dst, const float (&v)[8]) {
-    unsigned w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-        w[k] = *reinterpret_cast<const unsigned *>(&p);
-    }
-    *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 // Stage tile [t0, t0 + T) of x, delta, z (rows of nch channels) and of B, C into ring stage
 // st, with every index split by compile-time divisors.  VEC: 16-byte cp.async chunks, each
 // wholly inside or wholly outside [0, L) because L is a multiple of the chunk width.

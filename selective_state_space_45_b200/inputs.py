@@ -18,6 +18,7 @@ mamba130m      8       2048       1536     16   bf16 (A, D, bias, state fp32)
 mamba2p8b      4       4096       5120     16   bf16
 long1m         1       1048576    1536     16   bf16
 decode         256     1 x 64     5120     16   bf16 tokens, fp32 state
+bwd130m        8       2048       1536     16   bf16 inputs, dy and gradients (backward)
 conv130m       8       2048       1536     --   bf16 x and u; width 4, fp32 taps/bias
 conv2p8b       4       4096       5120     --   bf16 x and u; width 4
 convstep       256     1 x 64     5120     --   bf16 tokens, fp32 window (width 4)
@@ -48,6 +49,9 @@ CONFIGS = {
                    dt_dist="uniform"),
     "decode": dict(batch=256, steps=64, dim=5120, dstate=16, dtype=torch.bfloat16,
                    dt_dist="uniform"),
+    # the backward of the mamba130m-shaped scan (training), bf16 inputs and gradients
+    "bwd130m": dict(batch=8, seqlen=2048, dim=1536, dstate=16, dtype=torch.bfloat16,
+                    dt_dist="uniform"),
     # the causal convolution in front of the scan, in the same block shapes (width 4)
     "conv130m": dict(batch=8, seqlen=2048, dim=1536, width=4, dtype=torch.bfloat16),
     "conv2p8b": dict(batch=4, seqlen=4096, dim=5120, width=4, dtype=torch.bfloat16),
@@ -101,11 +105,27 @@ def make_scan_inputs(batch, dim, seqlen, dstate, dtype=torch.float32, device="cp
     return dict(x=x, delta=delta, z=z, B=B, C=C, A=A, D=D, delta_bias=delta_bias)
 
 
+def make_scan_bwd_inputs(batch, dim, seqlen, dstate, dtype=torch.bfloat16, device="cpu", seed=0,
+                         dt_dist="uniform"):
+    """Inputs of one backward call: those of ``make_scan_inputs`` (same seed) plus the
+    output gradient dy ([batch, dim, seqlen], ``dtype``, N(0, 1)) from a second generator
+    seeded seed + 1."""
+    inp = make_scan_inputs(batch, dim, seqlen, dstate, dtype, device=device, seed=seed,
+                           dt_dist=dt_dist)
+    g = _generator(device, seed + 1)
+    inp["dy"] = torch.randn(batch, dim, seqlen, generator=g, device=device,
+                            dtype=torch.float32).to(dtype)
+    return inp
+
+
 def make_config_inputs(name, device="cpu", seed=0):
     c = CONFIGS[name]
     if name == "convstep":
         return make_conv_step_inputs(c["batch"], c["dim"], c["steps"], c["width"], c["dtype"],
                                      device=device, seed=seed)
+    if name.startswith("bwd"):
+        return make_scan_bwd_inputs(c["batch"], c["dim"], c["seqlen"], c["dstate"], c["dtype"],
+                                    device=device, seed=seed, dt_dist=c["dt_dist"])
     if name.startswith("conv"):
         return make_conv_inputs(c["batch"], c["dim"], c["seqlen"], c["width"], c["dtype"],
                                 device=device, seed=seed)

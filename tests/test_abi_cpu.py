@@ -33,6 +33,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for expected in ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_scan_fwd_noalloc",
                      "ssm_state_step", "ssm_causal_conv1d_fwd", "ssm_causal_conv1d_step",
+                     "ssm_selective_scan_bwd",
                      "ssm_status_string", "ssm_version"):
         assert expected in names
 
@@ -180,6 +181,40 @@ def test_conv_argument_checks(lib, kw, status):
 ])
 def test_conv_step_argument_checks(lib, kw, status):
     assert conv_step(lib, **kw) == status
+
+
+def bwd(lib, **kw):
+    args = dict(x=P, delta=P, bias=None, sp=1, A=P, B=P, C=P, D=P, z=P, h0=None, dy=P, dfin=None,
+                dx=P, ddelta=P, dA=P, dB=P, dC=P, dD=P, dz=P, dbias=None, dh0=None,
+                batch=2, dim=3, L=8, N=16, din=ssm.SSM_BF16, dg=ssm.SSM_F32)
+    args.update(kw)
+    return lib.ssm_selective_scan_bwd(
+        args["x"], args["delta"], args["bias"], args["sp"], args["A"], args["B"], args["C"],
+        args["D"], args["z"], args["h0"], args["dy"], args["dfin"], args["dx"], args["ddelta"],
+        args["dA"], args["dB"], args["dC"], args["dD"], args["dz"], args["dbias"], args["dh0"],
+        args["batch"], args["dim"], args["L"], args["N"], args["din"], args["dg"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dy=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dx=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(ddelta=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dA=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dB=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dC=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(z=None), ssm.SSM_ERR_INVALID_ARG),         # dz requested without a gate
+    (dict(N=0), ssm.SSM_ERR_INVALID_ARG),
+    (dict(N=17), ssm.SSM_ERR_UNSUPPORTED),
+    (dict(L=-3), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dg=5), ssm.SSM_ERR_INVALID_ARG),
+    (dict(dy=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(dA=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(dh0=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(dim=0), ssm.SSM_OK),
+])
+def test_bwd_argument_checks(lib, kw, status):
+    assert bwd(lib, **kw) == status
 
 
 def test_python_binding_raises_on_error(lib):

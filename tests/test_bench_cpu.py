@@ -117,3 +117,17 @@ def test_workload_kinds():
 def test_conv_oracle_rate_single_core(name):
     r = bench.oracle_rate(name, threads=4, budget_s=0.2)
     assert r["kind"] == "oracle" and r["cores"] == 1 and r["value"] > 0
+
+
+def test_bwd_counts_mamba130m():
+    c = bench.bwd_counts(8, 1536, 2048, 16, 2, 2)
+    assert c["tokch"] == 8 * 2048 * 1536 and c["exps"] == 2 * 8 * 2048 * 1536 * 16
+    # x, delta, z, dy in and dx, ddelta, dz out (2 B each) + B, C in and dB, dC out + params
+    expect = 8 * 1536 * 2048 * 14 + 2 * 8 * 2048 * 16 * 4 + 2 * (1536 * 16 * 4 + 2 * 1536 * 4)
+    assert c["bytes"] == expect
+    assert bench.workload_kind("bwd130m") == "bwd"
+
+
+def test_bwd_oracle_rate_single_core():
+    r = bench.oracle_rate("bwd130m", threads=4, budget_s=0.2)
+    assert r["kind"] == "oracle" and r["cores"] == 1 and r["value"] > 0
