@@ -221,8 +221,10 @@ int ssm_causal_conv1d_step(float *window, const void *x, const float *weight, co
  *   dinitial_state: [batch][dim][dstate] fp32 or NULL: the gradient of the start state.
  * Sums over channels (dB, dC) and over sequences and positions (dA, dD, ddelta_bias) are
  * formed from per-CTA partial sums added in a fixed order: results are deterministic.
- * Takes a stream-ordered scratch buffer of about batch*dim'*(64*ceil(seqlen/32) + 4*seqlen
- * + 72) bytes, dim' = dim rounded up to 32 (cudaMallocAsync / cudaFreeAsync on cuda_stream).
+ * Takes a stream-ordered scratch buffer of about batch*dim'*(20*L' + 72) bytes, dim' = dim
+ * rounded up to 32 and L' = seqlen rounded up to 16 (the state before every 4th token,
+ * 16*L' bytes per channel, and per-CTA partial sums), with cudaMallocAsync / cudaFreeAsync
+ * on cuda_stream.
  * dstate must be 1..16; zoh_exact has no backward here.
  * seqlen = 0 writes zero parameter gradients and dinitial_state = dfinal_state.
  */

@@ -32,7 +32,7 @@ int run_bwd(ssm::BwdArgs a, void *dB, void *dC, float *dA, float *dD, float *dde
     if (ctas > INT_MAX || groups > INT_MAX) return SSM_ERR_UNSUPPORTED;
     a.groups_per_seq = int(groups);
     a.ntiles = (a.seqlen + Cfg::T - 1) / Cfg::T;
-    const size_t ck_floats = size_t(ctas) * a.ntiles * Cfg::NP * 32;
+    const size_t ck_floats = size_t(ctas) * a.ntiles * (Cfg::T / 4) * Cfg::NP * 32;
     const size_t bc_floats = 2 * size_t(ctas) * a.seqlen * Cfg::NP;
     const size_t pa_floats = size_t(a.batch) * a.dim * Cfg::NP;
     const size_t pd_floats = 2 * size_t(a.batch) * a.dim;

@@ -17,16 +17,15 @@
 //
 // Layout of the work (one CTA = 32 channels x 16 states of one sequence, 4 warps, one
 // channel per lane and one state quad per warp, as in the forward kernel):
-//   phase F   the forward recurrence over the whole sequence, keeping only the state at
-//             every tile start (a global scratch array, mostly L2-resident);
-//   phase R   tiles in reverse.  Per tile: (R1) recompute the tile forward from its
-//             checkpoint, keeping the state before every 4th token in registers and the
-//             per-quad readout in shared memory; (R2) per (t, d): the pre-gate output,
-//             dy * SiLU(z) and dz; (R3) sub-chunks of 4 tokens in reverse: recompute their
-//             states from the register checkpoint, then walk them backwards carrying mu;
-//             the dB / dC terms of the 32 channels are summed through a per-warp shared
-//             transpose and written as per-CTA partial sums; (R4) per (t, d): the quads'
-//             dx and dDelta partials summed, the softplus slope, 16-byte row stores.
+//   phase F   the forward recurrence over the whole sequence, keeping only the state
+//             before every 4th token (a global scratch array);
+//   phase R   16-token tiles in reverse.  Per tile: per (t, d) the step Delta and
+//             dypre = dy * SiLU(z); then sub-chunks of 4 tokens, last first: the states
+//             of the sub-chunk recomputed from its checkpoint (with the readout, for dz),
+//             then walked backwards carrying mu; the dB / dC terms of the 32 channels are
+//             summed through a per-warp shared transpose and written as per-CTA partial
+//             sums; finally per (t, d) the quads' dx, dDelta and readout partials summed,
+//             the softplus slope and dz, 16-byte row stores.
 //   Partial sums over channel groups (dB, dC) and over sequences (dA, dD, dbias) are
 //   added up by reduce_partials_kernel in a fixed order: the gradients are deterministic.
 #pragma once
@@ -56,7 +55,7 @@ struct BwdArgs {
     void *ddelta;
     void *dz;             // written when given (z must be given too)
     float *dh0;           // [batch][dim][dstate] or null
-    float *ck;            // [ctas][ntiles][4][32] float4: state at every tile start
+    float *ck;            // [ctas][ntiles*T/4][4][32] float4: state before every 4th token
     float *part_bc;       // [2][ctas][L][16]: per-CTA channel sums of the dB and dC terms
     float *part_a;        // [batch][dim][16]: per-sequence dA
     float *part_dd;       // [2][batch][dim]: per-sequence dD and ddelta_bias
@@ -70,7 +69,7 @@ template <typename Tin_, typename Tg_, bool VEC_>
 struct BwdCfg {
     using Tin = Tin_;
     using Tg = Tg_;
-    static constexpr int NP = 16, Q = 4, CH = 32, T = 32, NSTAGE = 2, NT = 128;
+    static constexpr int NP = 16, Q = 4, CH = 32, T = 16, NSTAGE = 2, NT = 128;
     static constexpr bool VEC = VEC_;
     static constexpr int EIN = 16 / sizeof(Tin);
     static constexpr int EG = 16 / sizeof(Tg);
@@ -79,7 +78,8 @@ struct BwdCfg {
     static constexpr int P_ROW = T + 4;         // per-quad partial rows (floats)
     static constexpr int X_ROW = 36;            // transpose rows: conflict-free both ways
     static constexpr int T8 = T / 8;
-    static_assert(CH * T8 == NT, "one (channel, 8-token chunk) task per thread");
+    static constexpr int NTASK = CH * T8;       // (channel, 8-token chunk) tasks per tile
+    static_assert(NTASK <= NT, "at most one task per thread");
 
     static constexpr size_t al(size_t v) { return (v + 15) & ~size_t(15); }
     static constexpr size_t RAW_ARR = al(size_t(CH) * RAW_ROW * sizeof(Tin));
@@ -92,10 +92,10 @@ struct BwdCfg {
     static constexpr size_t OFF_CF = OFF_BF + al(size_t(T) * NP * sizeof(float));
     static constexpr size_t PART_ARR = al(size_t(Q) * CH * P_ROW * sizeof(float));
     static constexpr size_t OFF_PART = OFF_CF + al(size_t(T) * NP * sizeof(float));
-    static constexpr size_t OFF_XP = OFF_PART + 2 * PART_ARR;
+    static constexpr size_t OFF_XP = OFF_PART + 3 * PART_ARR;
     static constexpr size_t SMEM_BYTES = OFF_XP + al(size_t(Q) * 32 * X_ROW * sizeof(float));
     // the staged dx / ddelta / dz rows reuse the partial arrays once they are summed
-    static_assert(3 * CH * G_ROW * sizeof(Tg) <= 2 * PART_ARR, "output staging must fit");
+    static_assert(3 * CH * G_ROW * sizeof(Tg) <= 3 * PART_ARR, "output staging must fit");
 };
 
 // Views of one ring stage: x, delta, z rows [CH][RAW_ROW], dy rows [CH][G_ROW], B, C [T][N].
@@ -206,22 +206,30 @@ __device__ __forceinline__ void bwd_load_tile(const BwdArgs &p, unsigned char *s
 
 
 // Per-(t, d) task of this thread: channel cc, tokens 8*t8 .. 8*t8+7 of the tile.  Writes
-// prep[t][cc] = (Delta_t, x_t, 0, 0); tokens past L and channels past dim become no-op
-// tokens (Delta = 0, x = 0: the state passes through unchanged, no gradient arises).
+// prep[t][cc] = (Delta_t, x_t, dypre_t, 0) with dypre = dy * SiLU(z) (dy alone without a
+// gate) when `full`, else (Delta_t, x_t, 0, 0).  Tokens past L and channels past dim become
+// no-op tokens (Delta = 0, x = 0, dypre = 0: the state passes through, no gradient arises).
 template <class Cfg>
 __device__ __forceinline__ void bwd_prep(const BwdArgs &p, const BwdStage<Cfg> &sv, float4 *prep,
-                                         int cc, int t8, bool cvalid, float bias, int t0) {
+                                         int cc, int t8, bool cvalid, float bias, int t0, bool full) {
     using Tin = typename Cfg::Tin;
+    using Tg = typename Cfg::Tg;
     constexpr int CH = Cfg::CH;
-    float dr[8], xr[8];
+    float dr[8], xr[8], gr[8], zr[8];
     load8<Tin>(sv.ds + cc * Cfg::RAW_ROW + 8 * t8, dr);
     load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+    if (full) {
+        load8<Tg>(sv.gs + cc * Cfg::G_ROW + 8 * t8, gr);
+        if (p.z != nullptr) load8<Tin>(sv.zs + cc * Cfg::RAW_ROW + 8 * t8, zr);
+    }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         float dl = dr[u] + bias;
         if (p.softplus) dl = softplus_f(dl);
         const bool ok = cvalid && t0 + 8 * t8 + u < p.seqlen;
-        prep[(8 * t8 + u) * CH + cc] = make_float4(ok ? dl : 0.f, ok ? xr[u] : 0.f, 0.f, 0.f);
+        float dyp = 0.f;
+        if (full) dyp = p.z != nullptr ? gr[u] * (zr[u] * sigmoid_f(zr[u])) : gr[u];
+        prep[(8 * t8 + u) * CH + cc] = make_float4(ok ? dl : 0.f, ok ? xr[u] : 0.f, ok ? dyp : 0.f, 0.f);
     }
 }
 
@@ -244,7 +252,7 @@ __device__ __forceinline__ void bwd_widen_bc(const BwdArgs &p, const BwdStage<Cf
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
+__global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
     using Tin = typename Cfg::Tin;
     using Tg = typename Cfg::Tg;
     constexpr int NP = Cfg::NP, Q = Cfg::Q, CH = Cfg::CH, T = Cfg::T, NT = Cfg::NT;
@@ -274,18 +282,21 @@ __global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
         Af[s] = (dvalid && n < N) ? p.A[size_t(d0 + c) * N + n] : 0.f;
         A2[s] = Af[s] * kLog2e;
     }
-    // this thread's (t, d) task: channel cc, 8-token chunk t8 of every tile
-    const int cc = tid % CH, t8 = tid / CH;
-    const bool cvalid = cc < nch;
+    // this thread's (t, d) task, if it has one: channel cc, 8-token chunk t8 of every tile
+    const bool has_task = tid < Cfg::NTASK;
+    const int cc = tid % CH, t8 = has_task ? tid / CH : 0;
+    const bool cvalid = has_task && cc < nch;
     const float tbias = (p.delta_bias != nullptr && cvalid) ? p.delta_bias[d0 + cc] : 0.f;
     const float tD = (p.D != nullptr && cvalid) ? p.D[d0 + cc] : 0.f;
 
     const size_t row0 = (size_t(b) * dim + d0) * size_t(L);
     const size_t bc0 = size_t(b) * L * size_t(N);
     const size_t chrow = size_t(b) * dim + d0 + c;
-    float4 *ck = reinterpret_cast<float4 *>(p.ck) + (size_t(cta) * ntiles * Q + q) * 32 + lane;
+    // checkpoint k of this CTA (the state before token 4k) for this lane: float4 at ck(k)
+    float4 *ckb = reinterpret_cast<float4 *>(p.ck) + (size_t(cta) * ntiles * (T / 4) * Q + q) * 32 + lane;
+    auto ck = [&](int k) { return ckb + size_t(k) * Q * 32; };
 
-    // ---------------- phase F: forward, keeping the state at every tile start ----------------
+    // ---------------- phase F: forward, keeping the state before every 4th token ----------------
     float h[4] = {0.f, 0.f, 0.f, 0.f};
     if (p.h0 != nullptr && dvalid) {
 #pragma unroll
@@ -296,17 +307,17 @@ __global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
     cp_async_commit();
     for (int tile = 0; tile < ntiles; ++tile) {
         const int t0 = tile * T;
-        ck[size_t(tile) * Q * 32] = make_float4(h[0], h[1], h[2], h[3]);
         cp_async_wait<0>();
         __syncthreads();
         if (tile + 1 < ntiles) bwd_load_tile<Cfg>(p, smem, (tile + 1) & 1, t0 + T, row0, bc0, nch, false);
         cp_async_commit();
         const BwdStage<Cfg> sv(smem, tile & 1);
-        bwd_prep<Cfg>(p, sv, prep, cc, t8, cvalid, tbias, t0);
+        if (has_task) bwd_prep<Cfg>(p, sv, prep, cc, t8, cvalid, tbias, t0, false);
         bwd_widen_bc<Cfg>(p, sv, Bf, Cf, t0, false);
         __syncthreads();
-#pragma unroll 8
+#pragma unroll
         for (int t = 0; t < T; ++t) {
+            if (t % 4 == 0) *ck(tile * (T / 4) + t / 4) = make_float4(h[0], h[1], h[2], h[3]);
             const float4 pv = prep[t * CH + c];
             const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
             const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
@@ -327,11 +338,18 @@ __global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
     }
     float dA_acc[4] = {0.f, 0.f, 0.f, 0.f};
     float dD_acc = 0.f, db_acc = 0.f;          // this thread's task channel, over its chunks
-    float *dxp = part0 + (q * CH + c) * Cfg::P_ROW;    // per-quad partials of this lane
-    float *ddp = part1 + (q * CH + c) * Cfg::P_ROW;
+    float *part2 = part1 + Cfg::PART_ARR / sizeof(float);
+    float *dxp = part0 + (q * CH + c) * Cfg::P_ROW;    // per-quad partials of this lane:
+    float *ddp = part1 + (q * CH + c) * Cfg::P_ROW;    //   sum_n lambda B, the dDelta terms,
+    float *ypp = part2 + (q * CH + c) * Cfg::P_ROW;    //   and the readout sum_n C h
     float *xrow = xp + lane * Cfg::X_ROW;
     const size_t bc_stride = size_t(ctas) * L * NP;    // dB block -> dC block of part_bc
     float *pbc = p.part_bc + size_t(cta) * L * NP;
+    // checkpoints are read two sub-chunks ahead of their use (they come from HBM)
+    const int nck = ntiles * (T / 4);
+    float4 ck1 = *ck(nck - 1);
+    float4 ck2 = nck >= 2 ? *ck(nck - 2) : make_float4(0.f, 0.f, 0.f, 0.f);
+    int knext = nck - 3;
 
     bwd_load_tile<Cfg>(p, smem, 0, (ntiles - 1) * T, row0, bc0, nch, true);
     cp_async_commit();
@@ -343,96 +361,40 @@ __global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
         if (tile > 0) bwd_load_tile<Cfg>(p, smem, (r + 1) & 1, t0 - T, row0, bc0, nch, true);
         cp_async_commit();
         const BwdStage<Cfg> sv(smem, r & 1);
-        bwd_prep<Cfg>(p, sv, prep, cc, t8, cvalid, tbias, t0);
+        if (has_task) bwd_prep<Cfg>(p, sv, prep, cc, t8, cvalid, tbias, t0, true);
         bwd_widen_bc<Cfg>(p, sv, Bf, Cf, t0, true);
         __syncthreads();
 
-        // R1: the tile forward again from its checkpoint; the state before every 4th token
-        // stays in registers, the per-quad readout goes to part0
-        float sub[T / 4][4];
-        {
-            const float4 hv = ck[size_t(tile) * Q * 32];
-            float hh[4] = {hv.x, hv.y, hv.z, hv.w};
-#pragma unroll
-            for (int g = 0; g < T / 4; ++g) {
-#pragma unroll
-                for (int s = 0; s < 4; ++s) sub[g][s] = hh[s];
-                float out[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int t = 4 * g + u;
-                    const float4 pv = prep[t * CH + c];
-                    const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
-                    const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
-                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-                    const float cb[4] = {cq.x, cq.y, cq.z, cq.w};
-                    const float dx = pv.x * pv.y;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        hh[s] = fmaf(ex2_approx(pv.x * A2[s]), hh[s], dx * bb[s]);
-                        acc = fmaf(cb[s], hh[s], acc);
-                    }
-                    out[u] = acc;
-                }
-                *reinterpret_cast<float4 *>(dxp + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
-            }
-        }
-        __syncthreads();
-
-        // R2: per (t, d): pre-gate output, dypre = dy * SiLU(z), dz -> prep[t][cc].zw
-        {
-            float acc[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-#pragma unroll
-            for (int qq = 0; qq < Q; ++qq) {
-                const float *src = part0 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
-                const float4 a0 = *reinterpret_cast<const float4 *>(src);
-                const float4 a1 = *reinterpret_cast<const float4 *>(src + 4);
-                acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
-                acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
-            }
-            float xr[8], gr[8], zr[8];
-            load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
-            load8<Tg>(sv.gs + cc * Cfg::G_ROW + 8 * t8, gr);
-            if (p.z != nullptr) load8<Tin>(sv.zs + cc * Cfg::RAW_ROW + 8 * t8, zr);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const bool ok = cvalid && t0 + 8 * t8 + u < L;
-                const float ypre = fmaf(tD, xr[u], acc[u]);
-                float dyp = gr[u], dzv = 0.f;
-                if (p.z != nullptr) {
-                    const float sg = sigmoid_f(zr[u]);
-                    dzv = gr[u] * ypre * sg * fmaf(zr[u], 1.f - sg, 1.f);
-                    dyp = gr[u] * zr[u] * sg;
-                }
-                *reinterpret_cast<float2 *>(reinterpret_cast<float *>(prep + (8 * t8 + u) * CH + cc) + 2) =
-                    make_float2(ok ? dyp : 0.f, ok ? dzv : 0.f);
-            }
-        }
-        __syncthreads();
-
-        // R3: sub-chunks of 4 tokens, last first: recompute their states, walk them back
+        // sub-chunks of 4 tokens, last first: recompute their states from the checkpoint,
+        // keep the readout, then walk them backwards carrying mu
 #pragma unroll 1
         for (int j = T / 4 - 1; j >= 0; --j) {
-            float hs[5][4], a[4][4], dl[4], xv[4], dyp[4];
-#pragma unroll
-            for (int s = 0; s < 4; ++s) hs[0][s] = sub[j][s];
+            const float4 hv = ck1;
+            ck1 = ck2;
+            if (knext >= 0) ck2 = *ck(knext);
+            --knext;
+            float hs[5][4], a[4][4], dl[4], xv[4], dyp[4], yo[4];
+            hs[0][0] = hv.x; hs[0][1] = hv.y; hs[0][2] = hv.z; hs[0][3] = hv.w;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int t = 4 * j + u;
                 const float4 pv = prep[t * CH + c];
                 dl[u] = pv.x; xv[u] = pv.y; dyp[u] = pv.z;
                 const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
+                const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
                 const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+                const float cb[4] = {cq.x, cq.y, cq.z, cq.w};
                 const float dx = dl[u] * xv[u];
+                float acc = 0.f;
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
                     a[u][s] = ex2_approx(dl[u] * A2[s]);
                     hs[u + 1][s] = fmaf(a[u][s], hs[u][s], dx * bb[s]);
+                    acc = fmaf(cb[s], hs[u + 1][s], acc);
                 }
+                yo[u] = acc;
             }
+            *reinterpret_cast<float4 *>(ypp + 4 * j) = make_float4(yo[0], yo[1], yo[2], yo[3]);
             float dxo[4], ddo[4];
 #pragma unroll
             for (int u = 3; u >= 0; --u) {
@@ -442,20 +404,22 @@ __global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
                 const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
                 const float cb[4] = {cq.x, cq.y, cq.z, cq.w};
                 const float dlx = dl[u] * xv[u];
-                float dxa = 0.f, dda = 0.f, vb[4], vc[4];
+                // sum_n lambda B_n gives both dx (times Delta) and, times x, the B part of
+                // dDelta; the decay part of dDelta and dA share lambda h_{t-1} Abar
+                float lb = 0.f, s2 = 0.f, vb[4], vc[4];
 #pragma unroll
                 for (int s = 0; s < 4; ++s) {
                     const float lam = fmaf(dyp[u], cb[s], mu[s]);
-                    const float ha = hs[u][s] * a[u][s];         // h_{t-1} * Abar_t
+                    const float lha = lam * (hs[u][s] * a[u][s]);
                     vb[s] = lam * dlx;                           // dB term
                     vc[s] = dyp[u] * hs[u + 1][s];               // dC term
-                    dxa = fmaf(lam, bb[s], dxa);
-                    dda = fmaf(lam, fmaf(bb[s], xv[u], ha * Af[s]), dda);
-                    dA_acc[s] = fmaf(lam * ha, dl[u], dA_acc[s]);
+                    lb = fmaf(lam, bb[s], lb);
+                    s2 = fmaf(lha, Af[s], s2);
+                    dA_acc[s] = fmaf(lha, dl[u], dA_acc[s]);
                     mu[s] = a[u][s] * lam;
                 }
-                dxo[u] = dxa * dl[u];
-                ddo[u] = dda;
+                dxo[u] = lb * dl[u];
+                ddo[u] = fmaf(lb, xv[u], s2);
                 *reinterpret_cast<float4 *>(xrow + 8 * u) = make_float4(vb[0], vb[1], vb[2], vb[3]);
                 *reinterpret_cast<float4 *>(xrow + 8 * u + 4) = make_float4(vc[0], vc[1], vc[2], vc[3]);
             }
@@ -475,45 +439,54 @@ __global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
         }
         __syncthreads();
 
-        // R4: per (t, d): sum the quads' dx and dDelta partials, skip term, softplus slope
+        // per (t, d): the quads' partials summed; dx with the skip, dDelta through the
+        // softplus slope, dz from the pre-gate output
         {
-            float dxs[8], dds[8];
+            float dxs[8], dds[8], yps[8], dzv[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) { dxs[u] = 0.f; dds[u] = 0.f; }
+            for (int u = 0; u < 8; ++u) { dxs[u] = 0.f; dds[u] = 0.f; yps[u] = 0.f; }
 #pragma unroll
             for (int qq = 0; qq < Q; ++qq) {
                 const float *s0 = part0 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
                 const float *s1 = part1 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
-                const float4 a0 = *reinterpret_cast<const float4 *>(s0);
-                const float4 a1 = *reinterpret_cast<const float4 *>(s0 + 4);
-                const float4 b0 = *reinterpret_cast<const float4 *>(s1);
-                const float4 b1 = *reinterpret_cast<const float4 *>(s1 + 4);
-                dxs[0] += a0.x; dxs[1] += a0.y; dxs[2] += a0.z; dxs[3] += a0.w;
-                dxs[4] += a1.x; dxs[5] += a1.y; dxs[6] += a1.z; dxs[7] += a1.w;
-                dds[0] += b0.x; dds[1] += b0.y; dds[2] += b0.z; dds[3] += b0.w;
-                dds[4] += b1.x; dds[5] += b1.y; dds[6] += b1.z; dds[7] += b1.w;
+                const float *s2 = part2 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
+                float v0[8], v1[8], v2[8];
+                load8<float>(s0, v0);
+                load8<float>(s1, v1);
+                load8<float>(s2, v2);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) { dxs[u] += v0[u]; dds[u] += v1[u]; yps[u] += v2[u]; }
             }
-            float xr[8], dr[8], dzv[8];
+            float xr[8], dr[8], gr[8], zr[8];
             load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
             load8<Tin>(sv.ds + cc * Cfg::RAW_ROW + 8 * t8, dr);
+            load8<Tg>(sv.gs + cc * Cfg::G_ROW + 8 * t8, gr);
+            if (p.z != nullptr) load8<Tin>(sv.zs + cc * Cfg::RAW_ROW + 8 * t8, zr);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const float4 pv = prep[(8 * t8 + u) * CH + cc];
+                const float dyp = prep[(8 * t8 + u) * CH + cc].z;
                 const bool ok = cvalid && t0 + 8 * t8 + u < L;
-                dxs[u] = fmaf(pv.z, tD, dxs[u]);
+                dxs[u] = fmaf(dyp, tD, dxs[u]);
                 if (p.softplus) dds[u] *= sigmoid_f(dr[u] + tbias);
                 dds[u] = ok ? dds[u] : 0.f;          // no-op tokens carry no step gradient
-                dzv[u] = pv.w;
-                dD_acc = fmaf(pv.z, ok ? xr[u] : 0.f, dD_acc);
+                dzv[u] = 0.f;
+                if (p.z != nullptr) {
+                    const float ypre = fmaf(tD, xr[u], yps[u]);
+                    const float sg = sigmoid_f(zr[u]);
+                    dzv[u] = ok ? gr[u] * ypre * sg * fmaf(zr[u], 1.f - sg, 1.f) : 0.f;
+                }
+                dD_acc = fmaf(dyp, ok ? xr[u] : 0.f, dD_acc);
                 db_acc += dds[u];
             }
             __syncthreads();                         // the partials are read: reuse as staging
-            Tg *ox = reinterpret_cast<Tg *>(part0);
-            Tg *od = ox + CH * Cfg::G_ROW;
-            Tg *oz = od + CH * Cfg::G_ROW;
-            store8<Tg>(ox + cc * Cfg::G_ROW + 8 * t8, dxs);
-            store8<Tg>(od + cc * Cfg::G_ROW + 8 * t8, dds);
-            if (p.z != nullptr) store8<Tg>(oz + cc * Cfg::G_ROW + 8 * t8, dzv);
+            if (has_task) {
+                Tg *ox = reinterpret_cast<Tg *>(part0);
+                Tg *od = ox + CH * Cfg::G_ROW;
+                Tg *oz = od + CH * Cfg::G_ROW;
+                store8<Tg>(ox + cc * Cfg::G_ROW + 8 * t8, dxs);
+                store8<Tg>(od + cc * Cfg::G_ROW + 8 * t8, dds);
+                if (p.z != nullptr) store8<Tg>(oz + cc * Cfg::G_ROW + 8 * t8, dzv);
+            }
         }
         __syncthreads();
 
@@ -565,8 +538,10 @@ __global__ void __launch_bounds__(Cfg::NT, 2) scan_bwd_kernel(const BwdArgs p) {
     }
     __syncthreads();
     float *red = reinterpret_cast<float *>(prep);   // [2][T8][CH]
-    red[t8 * CH + cc] = dD_acc;
-    red[(Cfg::T8 + t8) * CH + cc] = db_acc;
+    if (has_task) {
+        red[t8 * CH + cc] = dD_acc;
+        red[(Cfg::T8 + t8) * CH + cc] = db_acc;
+    }
     __syncthreads();
     if (tid < nch) {
         float sd = 0.f, sb = 0.f;
