@@ -63,6 +63,13 @@ __device__ __forceinline__ float silu_f(float z) {
     return z * rcp_approx(1.f + ex2_approx(-z * kLog2e));
 }
 
+// Packed FP32 pairs (sm_100: one instruction does two FP32 FMAs / products, each rounded
+// as fmaf / a plain product would be).  Used where independent states pair up.
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 ex2_pair(float2 v) { return f2(ex2_approx(v.x), ex2_approx(v.y)); }
+
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {

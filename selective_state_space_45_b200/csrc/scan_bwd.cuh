@@ -32,7 +32,18 @@
 
 #include "common.cuh"
 
+// Build-time tuning: independent partial sums in the column reduction of the dB / dC
+// transpose, and how many 4-token sub-chunks the reverse loop unrolls.
+#ifndef SSM_BWD_COLSUM_ACC
+#define SSM_BWD_COLSUM_ACC 4
+#endif
+#ifndef SSM_BWD_UNROLL_J
+#define SSM_BWD_UNROLL_J 1
+#endif
+
 namespace ssm {
+
+constexpr int kBwdUnrollJ = SSM_BWD_UNROLL_J;
 
 // sigmoid(v) = 1 / (1 + e^-v) with the SFU exponential and reciprocal (0 for v -> -inf).
 __device__ __forceinline__ float sigmoid_f(float v) {
@@ -275,12 +286,19 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
     float *part1 = part0 + Cfg::PART_ARR / sizeof(float);
     float *xp = reinterpret_cast<float *>(smem + Cfg::OFF_XP) + q * 32 * Cfg::X_ROW;
 
-    float Af[4], A2[4];
+    // this lane's 4 states as two pairs (0,1), (2,3) for the packed FP32 instructions
+    float2 Af[2], A2[2];
+    {
+        float av[4];
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        const int n = 4 * q + s;
-        Af[s] = (dvalid && n < N) ? p.A[size_t(d0 + c) * N + n] : 0.f;
-        A2[s] = Af[s] * kLog2e;
+        for (int s = 0; s < 4; ++s) {
+            const int n = 4 * q + s;
+            av[s] = (dvalid && n < N) ? p.A[size_t(d0 + c) * N + n] : 0.f;
+        }
+        Af[0] = f2(av[0], av[1]);
+        Af[1] = f2(av[2], av[3]);
+        A2[0] = fmul2(Af[0], f2(kLog2e, kLog2e));
+        A2[1] = fmul2(Af[1], f2(kLog2e, kLog2e));
     }
     // this thread's (t, d) task, if it has one: channel cc, 8-token chunk t8 of every tile
     const bool has_task = tid < Cfg::NTASK;
@@ -297,11 +315,14 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
     auto ck = [&](int k) { return ckb + size_t(k) * Q * 32; };
 
     // ---------------- phase F: forward, keeping the state before every 4th token ----------------
-    float h[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 h[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
     if (p.h0 != nullptr && dvalid) {
+        float hv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-            if (4 * q + s < N) h[s] = p.h0[chrow * N + 4 * q + s];
+            if (4 * q + s < N) hv[s] = p.h0[chrow * N + 4 * q + s];
+        h[0] = f2(hv[0], hv[1]);
+        h[1] = f2(hv[2], hv[3]);
     }
     bwd_load_tile<Cfg>(p, smem, 0, 0, row0, bc0, nch, false);
     cp_async_commit();
@@ -317,26 +338,32 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
         __syncthreads();
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-            if (t % 4 == 0) *ck(tile * (T / 4) + t / 4) = make_float4(h[0], h[1], h[2], h[3]);
+            if (t % 4 == 0) *ck(tile * (T / 4) + t / 4) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
             const float4 pv = prep[t * CH + c];
             const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
-            const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+            const float2 bb[2] = {f2(bq.x, bq.y), f2(bq.z, bq.w)};
+            const float2 dl2 = f2(pv.x, pv.x);
             const float dx = pv.x * pv.y;
+            const float2 dx2 = f2(dx, dx);
 #pragma unroll
-            for (int s = 0; s < 4; ++s) h[s] = fmaf(ex2_approx(pv.x * A2[s]), h[s], dx * bb[s]);
+            for (int k = 0; k < 2; ++k)
+                h[k] = ffma2(ex2_pair(fmul2(dl2, A2[k])), h[k], fmul2(dx2, bb[k]));
         }
     }
     cp_async_wait<0>();
     __syncthreads();
 
     // ---------------- phase R: tiles in reverse ----------------
-    float mu[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 mu[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
     if (p.dfinal != nullptr && dvalid) {
+        float mv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-            if (4 * q + s < N) mu[s] = p.dfinal[chrow * N + 4 * q + s];
+            if (4 * q + s < N) mv[s] = p.dfinal[chrow * N + 4 * q + s];
+        mu[0] = f2(mv[0], mv[1]);
+        mu[1] = f2(mv[2], mv[3]);
     }
-    float dA_acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 dA_acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
     float dD_acc = 0.f, db_acc = 0.f;          // this thread's task channel, over its chunks
     float *part2 = part1 + Cfg::PART_ARR / sizeof(float);
     float *dxp = part0 + (q * CH + c) * Cfg::P_ROW;    // per-quad partials of this lane:
@@ -367,14 +394,16 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
 
         // sub-chunks of 4 tokens, last first: recompute their states from the checkpoint,
         // keep the readout, then walk them backwards carrying mu
-#pragma unroll 1
+#pragma unroll kBwdUnrollJ
         for (int j = T / 4 - 1; j >= 0; --j) {
             const float4 hv = ck1;
             ck1 = ck2;
             if (knext >= 0) ck2 = *ck(knext);
             --knext;
-            float hs[5][4], a[4][4], dl[4], xv[4], dyp[4], yo[4];
-            hs[0][0] = hv.x; hs[0][1] = hv.y; hs[0][2] = hv.z; hs[0][3] = hv.w;
+            float2 hs[5][2], a[4][2];
+            float dl[4], xv[4], dyp[4], yo[4];
+            hs[0][0] = f2(hv.x, hv.y);
+            hs[0][1] = f2(hv.z, hv.w);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int t = 4 * j + u;
@@ -382,17 +411,19 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
                 dl[u] = pv.x; xv[u] = pv.y; dyp[u] = pv.z;
                 const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
                 const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
-                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-                const float cb[4] = {cq.x, cq.y, cq.z, cq.w};
+                const float2 bb[2] = {f2(bq.x, bq.y), f2(bq.z, bq.w)};
+                const float2 cb[2] = {f2(cq.x, cq.y), f2(cq.z, cq.w)};
+                const float2 dl2 = f2(dl[u], dl[u]);
                 const float dx = dl[u] * xv[u];
-                float acc = 0.f;
+                const float2 dx2 = f2(dx, dx);
+                float2 acc = f2(0.f, 0.f);
 #pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    a[u][s] = ex2_approx(dl[u] * A2[s]);
-                    hs[u + 1][s] = fmaf(a[u][s], hs[u][s], dx * bb[s]);
-                    acc = fmaf(cb[s], hs[u + 1][s], acc);
+                for (int k = 0; k < 2; ++k) {
+                    a[u][k] = ex2_pair(fmul2(dl2, A2[k]));
+                    hs[u + 1][k] = ffma2(a[u][k], hs[u][k], fmul2(dx2, bb[k]));
+                    acc = ffma2(cb[k], hs[u + 1][k], acc);
                 }
-                yo[u] = acc;
+                yo[u] = acc.x + acc.y;
             }
             *reinterpret_cast<float4 *>(ypp + 4 * j) = make_float4(yo[0], yo[1], yo[2], yo[3]);
             float dxo[4], ddo[4];
@@ -401,36 +432,43 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
                 const int t = 4 * j + u;
                 const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
                 const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
-                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-                const float cb[4] = {cq.x, cq.y, cq.z, cq.w};
+                const float2 bb[2] = {f2(bq.x, bq.y), f2(bq.z, bq.w)};
+                const float2 cb[2] = {f2(cq.x, cq.y), f2(cq.z, cq.w)};
                 const float dlx = dl[u] * xv[u];
+                const float2 dyp2 = f2(dyp[u], dyp[u]), dlx2 = f2(dlx, dlx), dl2 = f2(dl[u], dl[u]);
                 // sum_n lambda B_n gives both dx (times Delta) and, times x, the B part of
                 // dDelta; the decay part of dDelta and dA share lambda h_{t-1} Abar
-                float lb = 0.f, s2 = 0.f, vb[4], vc[4];
+                float2 lb = f2(0.f, 0.f), s2 = f2(0.f, 0.f), vb[2], vc[2];
 #pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const float lam = fmaf(dyp[u], cb[s], mu[s]);
-                    const float lha = lam * (hs[u][s] * a[u][s]);
-                    vb[s] = lam * dlx;                           // dB term
-                    vc[s] = dyp[u] * hs[u + 1][s];               // dC term
-                    lb = fmaf(lam, bb[s], lb);
-                    s2 = fmaf(lha, Af[s], s2);
-                    dA_acc[s] = fmaf(lha, dl[u], dA_acc[s]);
-                    mu[s] = a[u][s] * lam;
+                for (int k = 0; k < 2; ++k) {
+                    const float2 lam = ffma2(dyp2, cb[k], mu[k]);
+                    const float2 lha = fmul2(lam, fmul2(hs[u][k], a[u][k]));
+                    vb[k] = fmul2(lam, dlx2);                    // dB terms
+                    vc[k] = fmul2(dyp2, hs[u + 1][k]);           // dC terms
+                    lb = ffma2(lam, bb[k], lb);
+                    s2 = ffma2(lha, Af[k], s2);
+                    dA_acc[k] = ffma2(lha, dl2, dA_acc[k]);
+                    mu[k] = fmul2(a[u][k], lam);
                 }
-                dxo[u] = lb * dl[u];
-                ddo[u] = fmaf(lb, xv[u], s2);
-                *reinterpret_cast<float4 *>(xrow + 8 * u) = make_float4(vb[0], vb[1], vb[2], vb[3]);
-                *reinterpret_cast<float4 *>(xrow + 8 * u + 4) = make_float4(vc[0], vc[1], vc[2], vc[3]);
+                const float lbs = lb.x + lb.y;
+                dxo[u] = lbs * dl[u];
+                ddo[u] = fmaf(lbs, xv[u], s2.x + s2.y);
+                *reinterpret_cast<float4 *>(xrow + 8 * u) = make_float4(vb[0].x, vb[0].y, vb[1].x, vb[1].y);
+                *reinterpret_cast<float4 *>(xrow + 8 * u + 4) = make_float4(vc[0].x, vc[0].y, vc[1].x, vc[1].y);
             }
             *reinterpret_cast<float4 *>(dxp + 4 * j) = make_float4(dxo[0], dxo[1], dxo[2], dxo[3]);
             *reinterpret_cast<float4 *>(ddp + 4 * j) = make_float4(ddo[0], ddo[1], ddo[2], ddo[3]);
             __syncwarp();
             // column `lane` of the warp's transpose: value (token u, B or C, state s) summed
             // over the 32 channels
-            float sum = 0.f;
+            float part[SSM_BWD_COLSUM_ACC];
 #pragma unroll
-            for (int rr = 0; rr < 32; ++rr) sum += xp[rr * Cfg::X_ROW + lane];
+            for (int k = 0; k < SSM_BWD_COLSUM_ACC; ++k) part[k] = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) part[rr % SSM_BWD_COLSUM_ACC] += xp[rr * Cfg::X_ROW + lane];
+            float sum = part[0];
+#pragma unroll
+            for (int k = 1; k < SSM_BWD_COLSUM_ACC; ++k) sum += part[k];
             __syncwarp();
             const int u = lane >> 3, which = (lane >> 2) & 1, st = lane & 3;
             const int tok = t0 + 4 * j + u;
@@ -529,11 +567,12 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
     // per-sequence partials: dA of this lane's states; dD and ddelta_bias of the channels
     if (dvalid) {
         *reinterpret_cast<float4 *>(p.part_a + chrow * NP + 4 * q) =
-            make_float4(dA_acc[0], dA_acc[1], dA_acc[2], dA_acc[3]);
+            make_float4(dA_acc[0].x, dA_acc[0].y, dA_acc[1].x, dA_acc[1].y);
         if (p.dh0 != nullptr) {
+            const float mv[4] = {mu[0].x, mu[0].y, mu[1].x, mu[1].y};
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                if (4 * q + s < N) p.dh0[chrow * N + 4 * q + s] = mu[s];
+                if (4 * q + s < N) p.dh0[chrow * N + 4 * q + s] = mv[s];
         }
     }
     __syncthreads();

@@ -298,6 +298,9 @@ scan_fwd_kernel(const ScanArgs p) {
         }
     }
 
+    // the state in the recurrence: pairs (0,1), (2,3) for the packed FP32 instructions
+    float2 hp[2] = {f2(h[0], h[1]), f2(h[2], h[3])};
+    const float2 A2p[2] = {f2(A2[0], A2[1]), f2(A2[2], A2[3])};
     for (int tile = 0; tile < ntiles; ++tile) {
         const int st = tile % Cfg::NSTAGE;
         const int t0 = tbeg + tile * T;
@@ -384,8 +387,9 @@ scan_fwd_kernel(const ScanArgs p) {
         {
             const float4 *pp = prep + c;
             float *ypr = yp + (q * CH + c) * Cfg::YP_ROW;
-            // decays a = exp(Delta*A) and writes w = Delta*x*B of the 4 tokens of group g
-            auto decay_write = [&](int g, float (&a)[4][4], float (&w)[4][4]) {
+            // decays a = exp(Delta*A) and writes w = Delta*x*B of the 4 tokens of group g, as
+            // state pairs (0,1), (2,3) for the packed FP32 instructions
+            auto decay_write = [&](int g, float2 (&a)[4][2], float2 (&w)[4][2]) {
                 const float4 d01 = pp[(2 * g) * CH];   // (Delta, Delta*x or x) of tokens 4g, 4g+1
                 const float4 d23 = pp[(2 * g + 1) * CH];
                 const float dl[4] = {d01.x, d01.z, d23.x, d23.z};
@@ -394,51 +398,59 @@ scan_fwd_kernel(const ScanArgs p) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const float4 bq = *reinterpret_cast<const float4 *>(Bf + (4 * g + u) * NP + 4 * q);
-                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+                    const float2 bb[2] = {f2(bq.x, bq.y), f2(bq.z, bq.w)};
+                    const float2 dl2 = f2(dl[u], dl[u]);
 #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        a[u][s] = ex2_approx(dl[u] * A2[s]);
+                    for (int k = 0; k < 2; ++k) {
+                        a[u][k] = ex2_pair(fmul2(dl2, A2p[k]));
                         if constexpr (ZOH) {   // dx holds x here; gain = expm1(Delta a) / a
-                            const float v = dl[u] * A2[s] * (1.f / kLog2e);
-                            const float em1 = fabsf(v) < 0.1f ? expm1_small(v) : a[u][s] - 1.f;
-                            const float gain = invA[s] != 0.f ? em1 * invA[s] : dl[u];
-                            w[u][s] = gain * dx[u] * bb[s];
+                            float gw[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int s = 2 * k + e;
+                                const float av = e ? a[u][k].y : a[u][k].x;
+                                const float v = dl[u] * A2[s] * (1.f / kLog2e);
+                                const float em1 = fabsf(v) < 0.1f ? expm1_small(v) : av - 1.f;
+                                const float gain = invA[s] != 0.f ? em1 * invA[s] : dl[u];
+                                gw[e] = gain * dx[u] * (e ? bb[k].y : bb[k].x);
+                            }
+                            w[u][k] = f2(gw[0], gw[1]);
                         } else {
-                            w[u][s] = dx[u] * bb[s];
+                            w[u][k] = fmul2(f2(dx[u], dx[u]), bb[k]);
                         }
                     }
                 }
             };
-            auto recur_read = [&](int g, const float (&a)[4][4], const float (&w)[4][4]) {
+            auto recur_read = [&](int g, const float2 (&a)[4][2], const float2 (&w)[4][2]) {
                 float out[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const float4 cq = *reinterpret_cast<const float4 *>(Cf + (4 * g + u) * NP + 4 * q);
-                    const float cc4[4] = {cq.x, cq.y, cq.z, cq.w};
-                    float acc = 0.f;
+                    const float2 cc2[2] = {f2(cq.x, cq.y), f2(cq.z, cq.w)};
+                    float2 acc = f2(0.f, 0.f);
 #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        h[s] = fmaf(a[u][s], h[s], w[u][s]);
-                        acc = fmaf(cc4[s], h[s], acc);
+                    for (int k = 0; k < 2; ++k) {
+                        hp[k] = ffma2(a[u][k], hp[k], w[u][k]);
+                        acc = ffma2(cc2[k], hp[k], acc);
                     }
-                    out[u] = acc;
+                    out[u] = acc.x + acc.y;
                 }
                 *reinterpret_cast<float4 *>(ypr + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
             };
             // decays and writes of the next 4 tokens are computed before the recurrence
             // of the current 4, so the SFU work overlaps the FFMA chain
-            float a0[4][4], w0[4][4];
+            float2 a0[4][2], w0[4][2];
             decay_write(0, a0, w0);
 #pragma unroll
             for (int g = 0; g < T / 4; ++g) {
-                float a1[4][4], w1[4][4];
+                float2 a1[4][2], w1[4][2];
                 if (g + 1 < T / 4) decay_write(g + 1, a1, w1);
                 recur_read(g, a0, w0);
                 if (g + 1 < T / 4) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
 #pragma unroll
-                        for (int s = 0; s < 4; ++s) { a0[u][s] = a1[u][s]; w0[u][s] = w1[u][s]; }
+                        for (int k = 0; k < 2; ++k) { a0[u][k] = a1[u][k]; w0[u][k] = w1[u][k]; }
                 }
             }
         }
@@ -501,6 +513,7 @@ scan_fwd_kernel(const ScanArgs p) {
         }
     }
     cp_async_wait<0>();
+    h[0] = hp[0].x; h[1] = hp[0].y; h[2] = hp[1].x; h[3] = hp[1].y;
 
     if (SEG && p.pass == 1) {           // segment aggregates for pass 2
         if (dvalid) {
