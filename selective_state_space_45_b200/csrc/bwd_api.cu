@@ -18,6 +18,13 @@ int launch_reduce(const float *in, To *out, long long outer, int K, long long R,
                   cudaStream_t s) {
     const long long total = outer * R * Nout;
     if (total == 0) return SSM_OK;
+    if (NPin == Nout && Nout % 4 == 0) {   // whole 16-byte rows: the vectorised form
+        const long long groups = total / 4;
+        const long long blocks = std::min<long long>((groups + 255) / 256, 148LL * 16);
+        ssm::reduce_partials_vec4_kernel<To><<<unsigned(blocks), 256, 0, s>>>(in, out, outer, K,
+                                                                              R * Nout / 4);
+        return status_of(cudaGetLastError());
+    }
     const long long blocks = std::min<long long>((total + 255) / 256, 148LL * 16);
     ssm::reduce_partials_kernel<To><<<unsigned(blocks), 256, 0, s>>>(in, out, outer, K, R, NPin, Nout);
     return status_of(cudaGetLastError());

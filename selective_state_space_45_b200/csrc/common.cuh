@@ -116,6 +116,48 @@ template <> __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16 
     *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Store n (4 or 8) consecutive outputs with the widest aligned vectors: n * sizeof(T)
+// bytes, so the destination must be aligned to that (16 bytes, or 8 for 4 bf16).
+template <int n> __device__ __forceinline__ void store_run(float *p, const float *v) {
+#pragma unroll
+    for (int k = 0; k < n; k += 4)
+        *reinterpret_cast<float4 *>(p + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+}
+__device__ __forceinline__ unsigned pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const unsigned *>(&h);
+}
+template <int n> __device__ __forceinline__ void store_run(__nv_bfloat16 *p, const float *v) {
+    if constexpr (n == 4) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+    } else {
+#pragma unroll
+        for (int k = 0; k < n; k += 8)
+            *reinterpret_cast<uint4 *>(p + k) =
+                make_uint4(pack_bf16x2(v[k], v[k + 1]), pack_bf16x2(v[k + 2], v[k + 3]),
+                           pack_bf16x2(v[k + 4], v[k + 5]), pack_bf16x2(v[k + 6], v[k + 7]));
+    }
+}
+
+// n = 4 or 8 consecutive values of a staged row as fp32 / stored from fp32 (the source or
+// destination aligned to n * sizeof(T) bytes).
+template <int n, typename T> __device__ __forceinline__ void loadn(const T *src, float (&v)[n]) {
+    if constexpr (n == 8) {
+        load8<T>(src, v);
+    } else if constexpr (sizeof(T) == 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(src);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else {
+        const uint2 u = *reinterpret_cast<const uint2 *>(src);
+        v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
+        v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
+    }
+}
+template <int n, typename T> __device__ __forceinline__ void storen(T *dst, const float (&v)[n]) {
+    if constexpr (n == 8) store8<T>(dst, v);
+    else store_run<4>(dst, v);
+}
+
 // 16-byte asynchronous global -> shared copy (bypasses L1), grouped with commit/wait.
 __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gmem_src) {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));

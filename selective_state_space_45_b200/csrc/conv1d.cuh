@@ -51,29 +51,6 @@ template <> struct Vec16<__nv_bfloat16> {
     }
 };
 
-// Store n (4 or 8) consecutive outputs with the widest aligned vectors: n * sizeof(T)
-// bytes, so the destination must be aligned to that (16 bytes, or 8 for 4 bf16).
-template <int n> __device__ __forceinline__ void store_run(float *p, const float *v) {
-#pragma unroll
-    for (int k = 0; k < n; k += 4)
-        *reinterpret_cast<float4 *>(p + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-}
-__device__ __forceinline__ unsigned pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const unsigned *>(&h);
-}
-template <int n> __device__ __forceinline__ void store_run(__nv_bfloat16 *p, const float *v) {
-    if constexpr (n == 4) {
-        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
-    } else {
-#pragma unroll
-        for (int k = 0; k < n; k += 8)
-            *reinterpret_cast<uint4 *>(p + k) =
-                make_uint4(pack_bf16x2(v[k], v[k + 1]), pack_bf16x2(v[k + 2], v[k + 3]),
-                           pack_bf16x2(v[k + 4], v[k + 5]), pack_bf16x2(v[k + 6], v[k + 7]));
-    }
-}
-
 // Vector path: rows whose length is a multiple of one 16-byte vector (V elements), widths
 // 1..4 (K-1 <= V).  Each warp owns a span of 32*U consecutive vectors of one row, laid out
 // as a copy kernel lays them out: vector v0 + 32k + lane goes to lane `lane`, load k, so

@@ -88,8 +88,9 @@ struct BwdCfg {
     static constexpr int G_ROW = T + EG;
     static constexpr int P_ROW = T + 4;         // per-quad partial rows (floats)
     static constexpr int X_ROW = 36;            // transpose rows: conflict-free both ways
-    static constexpr int T8 = T / 8;
-    static constexpr int NTASK = CH * T8;       // (channel, 8-token chunk) tasks per tile
+    static constexpr int TW = 4;                // tokens per (t, d) task
+    static constexpr int NTW = T / TW;          // task chunks per row
+    static constexpr int NTASK = CH * NTW;      // (channel, token chunk) tasks per tile
     static_assert(NTASK <= NT, "at most one task per thread");
 
     static constexpr size_t al(size_t v) { return (v + 15) & ~size_t(15); }
@@ -216,31 +217,32 @@ __device__ __forceinline__ void bwd_load_tile(const BwdArgs &p, unsigned char *s
 }
 
 
-// Per-(t, d) task of this thread: channel cc, tokens 8*t8 .. 8*t8+7 of the tile.  Writes
+// Per-(t, d) task of this thread: channel cc, tokens TW*tk .. TW*tk+TW-1 of the tile.  Writes
 // prep[t][cc] = (Delta_t, x_t, dypre_t, 0) with dypre = dy * SiLU(z) (dy alone without a
 // gate) when `full`, else (Delta_t, x_t, 0, 0).  Tokens past L and channels past dim become
 // no-op tokens (Delta = 0, x = 0, dypre = 0: the state passes through, no gradient arises).
 template <class Cfg>
 __device__ __forceinline__ void bwd_prep(const BwdArgs &p, const BwdStage<Cfg> &sv, float4 *prep,
-                                         int cc, int t8, bool cvalid, float bias, int t0, bool full) {
+                                         int cc, int tk, bool cvalid, float bias, int t0, bool full) {
     using Tin = typename Cfg::Tin;
     using Tg = typename Cfg::Tg;
     constexpr int CH = Cfg::CH;
-    float dr[8], xr[8], gr[8], zr[8];
-    load8<Tin>(sv.ds + cc * Cfg::RAW_ROW + 8 * t8, dr);
-    load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+    constexpr int TW = Cfg::TW;
+    float dr[TW], xr[TW], gr[TW], zr[TW];
+    loadn<TW, Tin>(sv.ds + cc * Cfg::RAW_ROW + TW * tk, dr);
+    loadn<TW, Tin>(sv.xs + cc * Cfg::RAW_ROW + TW * tk, xr);
     if (full) {
-        load8<Tg>(sv.gs + cc * Cfg::G_ROW + 8 * t8, gr);
-        if (p.z != nullptr) load8<Tin>(sv.zs + cc * Cfg::RAW_ROW + 8 * t8, zr);
+        loadn<TW, Tg>(sv.gs + cc * Cfg::G_ROW + TW * tk, gr);
+        if (p.z != nullptr) loadn<TW, Tin>(sv.zs + cc * Cfg::RAW_ROW + TW * tk, zr);
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < TW; ++u) {
         float dl = dr[u] + bias;
         if (p.softplus) dl = softplus_f(dl);
-        const bool ok = cvalid && t0 + 8 * t8 + u < p.seqlen;
+        const bool ok = cvalid && t0 + TW * tk + u < p.seqlen;
         float dyp = 0.f;
         if (full) dyp = p.z != nullptr ? gr[u] * (zr[u] * sigmoid_f(zr[u])) : gr[u];
-        prep[(8 * t8 + u) * CH + cc] = make_float4(ok ? dl : 0.f, ok ? xr[u] : 0.f, ok ? dyp : 0.f, 0.f);
+        prep[(TW * tk + u) * CH + cc] = make_float4(ok ? dl : 0.f, ok ? xr[u] : 0.f, ok ? dyp : 0.f, 0.f);
     }
 }
 
@@ -300,9 +302,10 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
         A2[0] = fmul2(Af[0], f2(kLog2e, kLog2e));
         A2[1] = fmul2(Af[1], f2(kLog2e, kLog2e));
     }
-    // this thread's (t, d) task, if it has one: channel cc, 8-token chunk t8 of every tile
+    // this thread's (t, d) task, if it has one: channel cc, token chunk tk of every tile
+    constexpr int TW = Cfg::TW;
     const bool has_task = tid < Cfg::NTASK;
-    const int cc = tid % CH, t8 = has_task ? tid / CH : 0;
+    const int cc = tid % CH, tk = has_task ? tid / CH : 0;
     const bool cvalid = has_task && cc < nch;
     const float tbias = (p.delta_bias != nullptr && cvalid) ? p.delta_bias[d0 + cc] : 0.f;
     const float tD = (p.D != nullptr && cvalid) ? p.D[d0 + cc] : 0.f;
@@ -333,7 +336,7 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
         if (tile + 1 < ntiles) bwd_load_tile<Cfg>(p, smem, (tile + 1) & 1, t0 + T, row0, bc0, nch, false);
         cp_async_commit();
         const BwdStage<Cfg> sv(smem, tile & 1);
-        if (has_task) bwd_prep<Cfg>(p, sv, prep, cc, t8, cvalid, tbias, t0, false);
+        if (has_task) bwd_prep<Cfg>(p, sv, prep, cc, tk, cvalid, tbias, t0, false);
         bwd_widen_bc<Cfg>(p, sv, Bf, Cf, t0, false);
         __syncthreads();
 #pragma unroll
@@ -388,7 +391,7 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
         if (tile > 0) bwd_load_tile<Cfg>(p, smem, (r + 1) & 1, t0 - T, row0, bc0, nch, true);
         cp_async_commit();
         const BwdStage<Cfg> sv(smem, r & 1);
-        if (has_task) bwd_prep<Cfg>(p, sv, prep, cc, t8, cvalid, tbias, t0, true);
+        if (has_task) bwd_prep<Cfg>(p, sv, prep, cc, tk, cvalid, tbias, t0, true);
         bwd_widen_bc<Cfg>(p, sv, Bf, Cf, t0, true);
         __syncthreads();
 
@@ -480,30 +483,30 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
         // per (t, d): the quads' partials summed; dx with the skip, dDelta through the
         // softplus slope, dz from the pre-gate output
         {
-            float dxs[8], dds[8], yps[8], dzv[8];
+            float dxs[TW], dds[TW], yps[TW], dzv[TW];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) { dxs[u] = 0.f; dds[u] = 0.f; yps[u] = 0.f; }
+            for (int u = 0; u < TW; ++u) { dxs[u] = 0.f; dds[u] = 0.f; yps[u] = 0.f; }
 #pragma unroll
             for (int qq = 0; qq < Q; ++qq) {
-                const float *s0 = part0 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
-                const float *s1 = part1 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
-                const float *s2 = part2 + (qq * CH + cc) * Cfg::P_ROW + 8 * t8;
-                float v0[8], v1[8], v2[8];
-                load8<float>(s0, v0);
-                load8<float>(s1, v1);
-                load8<float>(s2, v2);
+                const float *s0 = part0 + (qq * CH + cc) * Cfg::P_ROW + TW * tk;
+                const float *s1 = part1 + (qq * CH + cc) * Cfg::P_ROW + TW * tk;
+                const float *s2 = part2 + (qq * CH + cc) * Cfg::P_ROW + TW * tk;
+                float v0[TW], v1[TW], v2[TW];
+                loadn<TW, float>(s0, v0);
+                loadn<TW, float>(s1, v1);
+                loadn<TW, float>(s2, v2);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) { dxs[u] += v0[u]; dds[u] += v1[u]; yps[u] += v2[u]; }
+                for (int u = 0; u < TW; ++u) { dxs[u] += v0[u]; dds[u] += v1[u]; yps[u] += v2[u]; }
             }
-            float xr[8], dr[8], gr[8], zr[8];
-            load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
-            load8<Tin>(sv.ds + cc * Cfg::RAW_ROW + 8 * t8, dr);
-            load8<Tg>(sv.gs + cc * Cfg::G_ROW + 8 * t8, gr);
-            if (p.z != nullptr) load8<Tin>(sv.zs + cc * Cfg::RAW_ROW + 8 * t8, zr);
+            float xr[TW], dr[TW], gr[TW], zr[TW];
+            loadn<TW, Tin>(sv.xs + cc * Cfg::RAW_ROW + TW * tk, xr);
+            loadn<TW, Tin>(sv.ds + cc * Cfg::RAW_ROW + TW * tk, dr);
+            loadn<TW, Tg>(sv.gs + cc * Cfg::G_ROW + TW * tk, gr);
+            if (p.z != nullptr) loadn<TW, Tin>(sv.zs + cc * Cfg::RAW_ROW + TW * tk, zr);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float dyp = prep[(8 * t8 + u) * CH + cc].z;
-                const bool ok = cvalid && t0 + 8 * t8 + u < L;
+            for (int u = 0; u < TW; ++u) {
+                const float dyp = prep[(TW * tk + u) * CH + cc].z;
+                const bool ok = cvalid && t0 + TW * tk + u < L;
                 dxs[u] = fmaf(dyp, tD, dxs[u]);
                 if (p.softplus) dds[u] *= sigmoid_f(dr[u] + tbias);
                 dds[u] = ok ? dds[u] : 0.f;          // no-op tokens carry no step gradient
@@ -521,9 +524,9 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
                 Tg *ox = reinterpret_cast<Tg *>(part0);
                 Tg *od = ox + CH * Cfg::G_ROW;
                 Tg *oz = od + CH * Cfg::G_ROW;
-                store8<Tg>(ox + cc * Cfg::G_ROW + 8 * t8, dxs);
-                store8<Tg>(od + cc * Cfg::G_ROW + 8 * t8, dds);
-                if (p.z != nullptr) store8<Tg>(oz + cc * Cfg::G_ROW + 8 * t8, dzv);
+                storen<TW, Tg>(ox + cc * Cfg::G_ROW + TW * tk, dxs);
+                storen<TW, Tg>(od + cc * Cfg::G_ROW + TW * tk, dds);
+                if (p.z != nullptr) storen<TW, Tg>(oz + cc * Cfg::G_ROW + TW * tk, dzv);
             }
         }
         __syncthreads();
@@ -576,22 +579,57 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
         }
     }
     __syncthreads();
-    float *red = reinterpret_cast<float *>(prep);   // [2][T8][CH]
+    float *red = reinterpret_cast<float *>(prep);   // [2][NTW][CH]
     if (has_task) {
-        red[t8 * CH + cc] = dD_acc;
-        red[(Cfg::T8 + t8) * CH + cc] = db_acc;
+        red[tk * CH + cc] = dD_acc;
+        red[(Cfg::NTW + tk) * CH + cc] = db_acc;
     }
     __syncthreads();
     if (tid < nch) {
         float sd = 0.f, sb = 0.f;
 #pragma unroll
-        for (int k = 0; k < Cfg::T8; ++k) {
+        for (int k = 0; k < Cfg::NTW; ++k) {
             sd += red[k * CH + tid];
-            sb += red[(Cfg::T8 + k) * CH + tid];
+            sb += red[(Cfg::NTW + k) * CH + tid];
         }
         const size_t bd = size_t(b) * dim + d0 + tid;
         p.part_dd[bd] = sd;
         p.part_dd[size_t(p.batch) * dim + bd] = sb;
+    }
+}
+
+// The same sum when every row is whole (NPin == Nout, a multiple of 4): four consecutive
+// outputs per thread with 16-byte loads, eight loads in flight, summed in k order in two
+// interleaved halves (even k, odd k) that are added at the end -- a fixed order, so the
+// result is deterministic.
+template <typename To>
+__global__ void __launch_bounds__(256)
+reduce_partials_vec4_kernel(const float *__restrict__ in, To *__restrict__ out, long long outer,
+                            int K, long long R4) {
+    const long long total = outer * R4;               // float4 groups of the output
+    for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+         e += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long i = e / R4, r = e - i * R4;
+        const float4 *src = reinterpret_cast<const float4 *>(in) + (i * K) * R4 + r;
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+        int k = 0;
+        for (; k + 8 <= K; k += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __ldg(src + static_cast<long long>(k + u) * R4);
+#pragma unroll
+            for (int u = 0; u < 8; u += 2) {
+                a0.x += v[u].x; a0.y += v[u].y; a0.z += v[u].z; a0.w += v[u].w;
+                a1.x += v[u + 1].x; a1.y += v[u + 1].y; a1.z += v[u + 1].z; a1.w += v[u + 1].w;
+            }
+        }
+        for (; k < K; ++k) {
+            const float4 v = __ldg(src + static_cast<long long>(k) * R4);
+            if (k & 1) { a1.x += v.x; a1.y += v.y; a1.z += v.z; a1.w += v.w; }
+            else       { a0.x += v.x; a0.y += v.y; a0.z += v.z; a0.w += v.w; }
+        }
+        const float o[4] = {a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w};
+        store_run<4>(out + 4 * e, o);
     }
 }
 
