@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba130m",
                     choices=["mamba130m", "mamba2p8b", "long1m", "decode", "tiny",
-                             "conv130m", "conv2p8b", "convstep", "bwd130m"])
+                             "conv130m", "conv2p8b", "convstep", "bwd130m", "decode4"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0,
@@ -117,6 +117,7 @@ def load_peaks():
 
 # translation unit of libssm.so that holds each kernel and its launch logic
 KERNEL_UNIT = {"scan_fwd_kernel": "scan_api.cu", "state_step_kernel": "step_api.cu",
+               "state_steps_kernel": "step_api.cu",
                "scan_bwd_kernel": "bwd_api.cu",
                "causal_conv1d_vec_kernel": "conv_api.cu", "conv1d_step_kernel": "conv_api.cu"}
 
@@ -228,6 +229,8 @@ def bwd_counts(batch, dim, L, N, in_size, g_size):
 def workload_kind(name):
     if name.startswith("bwd"):
         return "bwd"
+    if name == "decode4":
+        return "decodemulti"
     if name == "decode":
         return "decode"
     if name == "convstep":
@@ -235,6 +238,15 @@ def workload_kind(name):
     if name.startswith("conv"):
         return "conv"
     return "scan"
+
+
+def steps_counts(ntok, batch, dim, N, in_size, out_size):
+    """ntok decode tokens in one call: the state read and written once."""
+    c = step_counts(batch, dim, N, in_size, out_size)
+    state = 2 * batch * dim * N * 4
+    per_tok = c["bytes"] - state - (dim * N * 4 + dim * 4)
+    return dict(bytes=state + ntok * per_tok + dim * N * 4 + dim * 4, exps=ntok * c["exps"],
+                tokch=ntok * c["tokch"])
 
 
 def step_counts(batch, dim, N, in_size, out_size):
@@ -264,6 +276,8 @@ class Workload:
             self.counts = bwd_counts(c["batch"], c["dim"], c["seqlen"], c["dstate"], esz, esz)
         elif self.kind == "decode":
             self.counts = step_counts(c["batch"], c["dim"], c["dstate"], esz, esz)
+        elif self.kind == "decodemulti":
+            self.counts = steps_counts(c["ntok"], c["batch"], c["dim"], c["dstate"], esz, esz)
         elif self.kind == "conv":
             self.counts = conv_counts(c["batch"], c["dim"], c["seqlen"], c["width"], esz, esz)
         else:
@@ -287,6 +301,8 @@ class Workload:
             elif self.kind == "conv":
                 inp["u"] = torch.empty(inp["x"].shape, device=device, dtype=dt)
                 inp["fw"] = torch.empty(c["batch"], c["dim"], c["width"] - 1, device=device)
+            elif self.kind == "decodemulti":
+                inp["y"] = torch.empty(c["ntok"], c["batch"], c["dim"], device=device, dtype=dt)
             else:
                 inp["y" if self.kind == "decode" else "u"] = torch.empty(
                     c["batch"], c["dim"], device=device, dtype=dt)
@@ -298,6 +314,12 @@ class Workload:
         if self.kind == "scan":
             ssm.ssm_selective_scan_fwd(s["x"], s["delta"], s["delta_bias"], True, s["A"], s["B"],
                                        s["C"], s["D"], s["z"], s["y"], s["fs"], stream)
+        elif self.kind == "decodemulti":
+            k = self.cfg["ntok"]
+            t = ((i // self.nsets) % (s["x"].shape[0] // k)) * k
+            ssm.ssm_state_step_multi(s["state"], s["x"][t:t + k], s["delta"][t:t + k], s["A"],
+                                     s["B"][t:t + k], s["C"][t:t + k], s["D"], s["z"][t:t + k],
+                                     s["y"], stream)
         elif self.kind == "bwd":
             ssm.ssm_selective_scan_bwd(s["x"], s["delta"], s["delta_bias"], True, s["A"], s["B"], s["C"],
                                        s["D"], s["z"], None, s["dy"], None, s["dx"], s["ddelta"], s["dA"],
@@ -324,6 +346,9 @@ class Workload:
         if self.kind == "convstep":
             return ("decode conv1d step: batch %d, d_inner %d, width %d, fp32 window in place, one %s "
                     "token per sequence" % (c["batch"], c["dim"], c["width"], io))
+        if self.kind == "decodemulti":
+            return ("decode, %d tokens per call on the carried state: batch %d, d_inner %d, N %d, "
+                    "fp32 state in place, %s tokens" % (c["ntok"], c["batch"], c["dim"], c["dstate"], io))
         if self.kind == "bwd":
             return ("%s-shaped selective scan backward (states recomputed): batch %d, L %d, d_inner %d, "
                     "N %d, %s inputs, dy and gradients, fp32 A/D/bias gradients"
@@ -338,7 +363,8 @@ class Workload:
 
 def kernel_name(kind):
     return dict(scan="scan_fwd_kernel", decode="state_step_kernel", conv="causal_conv1d_vec_kernel",
-                convstep="conv1d_step_kernel", bwd="scan_bwd_kernel")[kind]
+                convstep="conv1d_step_kernel", bwd="scan_bwd_kernel",
+                decodemulti="state_steps_kernel")[kind]
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -383,6 +409,12 @@ def _oracle_sample(name, n_target_tokch, seed=0):
                                           seed=seed)
         return kind, inp, per_channel * k, "%d sequences x %d of %d channels, all %d tokens" % (
             c["batch"], k, c["dim"], L)
+    if kind == "decodemulti":
+        k = int(max(1, min(c["dim"], n_target_tokch // (c["batch"] * c["ntok"]))))
+        inp = inputs.make_decode_inputs(c["batch"], k, c["dstate"], c["ntok"], c["dtype"], device="cpu",
+                                        seed=seed)
+        return kind, inp, c["ntok"] * c["batch"] * k, "%d sequences x %d of %d channels, %d tokens" % (
+            c["batch"], k, c["dim"], c["ntok"])
     if name == "decode":
         k = int(max(1, min(c["dim"], n_target_tokch // c["batch"])))
         inp = inputs.make_decode_inputs(c["batch"], k, c["dstate"], 1, c["dtype"], device="cpu",
@@ -410,6 +442,11 @@ def _oracle_call(kind, inp, threads):
     if kind == "scan":
         oracle.scan(x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], D=inp["D"],
                     z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True, nthreads=threads)
+    elif kind == "decodemulti":
+        h = inp["state"]
+        for t in range(inp["x"].shape[0]):
+            _, h = oracle.step(h, inp["x"][t], inp["delta"][t], inp["A"], inp["B"][t], inp["C"][t],
+                               D=inp["D"], z=inp["z"][t])
     elif kind == "bwd":
         oracle.scan_bwd(inp["dy"], inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
                         z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True)
@@ -499,17 +536,22 @@ def time_e2e(wl, steps, stream):
     import selective_state_space_45_b200 as ssm
     dev = wl.sets[0]
     # per-token inputs of the decode kinds are [steps, ...]: one token's slice travels
-    per_token = {"decode": ("x", "delta", "z", "B", "C"), "convstep": ("x",)}.get(wl.kind, ())
+    per_token = {"decode": ("x", "delta", "z", "B", "C"), "convstep": ("x",),
+                 "decodemulti": ("x", "delta", "z", "B", "C")}.get(wl.kind, ())
+    ntok = wl.cfg.get("ntok", 1)
     names_in, names_out = dict(
         scan=(["x", "delta", "z", "B", "C", "A", "D", "delta_bias"], ["y", "fs"]),
         bwd=(["x", "delta", "z", "B", "C", "A", "D", "delta_bias", "dy"],
              ["dx", "ddelta", "dz", "dB", "dC", "dA", "dD", "dbias"]),
         decode=(["state", "x", "delta", "z", "B", "C", "A", "D"], ["y", "state"]),
+        decodemulti=(["state", "x", "delta", "z", "B", "C", "A", "D"], ["y", "state"]),
         conv=(["x", "weight", "bias"], ["u", "fw"]),
         convstep=(["window", "x", "weight", "bias"], ["u", "window"]))[wl.kind]
 
     def dev_view(n):
-        return dev[n][0] if n in per_token else dev[n]
+        if n not in per_token:
+            return dev[n]
+        return dev[n][0:ntok] if wl.kind == "decodemulti" else dev[n][0]
 
     host = {}
     for n in names_in:
@@ -526,6 +568,9 @@ def time_e2e(wl, steps, stream):
         if wl.kind == "scan":
             ssm.ssm_selective_scan_fwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"],
                                        dev["B"], dev["C"], dev["D"], dev["z"], dev["y"], dev["fs"])
+        elif wl.kind == "decodemulti":
+            ssm.ssm_state_step_multi(dev["state"], dev_view("x"), dev_view("delta"), dev["A"],
+                                     dev_view("B"), dev_view("C"), dev["D"], dev_view("z"), dev["y"])
         elif wl.kind == "bwd":
             ssm.ssm_selective_scan_bwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"], dev["B"],
                                        dev["C"], dev["D"], dev["z"], None, dev["dy"], None, dev["dx"],

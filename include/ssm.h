@@ -4,6 +4,7 @@
  * Operations:
  *   ssm_selective_scan_fwd  the selective scan (S6) over a whole sequence;
  *   ssm_state_step          one decode token on a carried state, updated in place;
+ *   ssm_state_step_multi    several decode tokens on a carried state in one call;
  *   ssm_causal_conv1d_fwd   the causal depthwise convolution + SiLU that feeds the scan;
  *   ssm_causal_conv1d_step  its one-token form on a carried window, updated in place;
  *   ssm_selective_scan_bwd  the gradients of the scan (training), states recomputed.
@@ -236,6 +237,23 @@ int ssm_selective_scan_bwd(const void *x, const void *delta, const float *delta_
                            void *dz, float *ddelta_bias, float *dinitial_state,
                            int batch, int dim, int seqlen, int dstate,
                            int in_dtype, int grad_dtype, void *cuda_stream);
+
+/*
+ * Several decode tokens on a carried state in one call (speculative or chunked decoding):
+ * ntok chained ssm_state_step calls, with the state read and written once.
+ *
+ *   state       : [batch][dim][dstate] fp32, read and overwritten with the state after
+ *                 the last token.
+ *   x, delta, z : [ntok][batch][dim], in_dtype (delta already positive; z may be NULL).
+ *   B, C        : [ntok][batch][dstate], in_dtype.   A, D: as for ssm_state_step.
+ *   y           : [ntok][batch][dim], out_dtype, written.
+ * Per token the arithmetic is that of ssm_state_step in the same order: the results are
+ * bit-identical to ntok chained calls.  ntok = 0 does nothing.
+ */
+int ssm_state_step_multi(float *state, const void *x, const void *delta, const float *A,
+                         const void *B, const void *C, const float *D, const void *z, void *y,
+                         int ntok, int batch, int dim, int dstate, int in_dtype, int out_dtype,
+                         void *cuda_stream);
 
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char *ssm_status_string(int status);

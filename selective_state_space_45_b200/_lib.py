@@ -57,6 +57,8 @@ def load_library(path: str | None = None):
         lib.ssm_causal_conv1d_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
         lib.ssm_causal_conv1d_step.restype = i
         lib.ssm_causal_conv1d_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+        lib.ssm_state_step_multi.restype = i
+        lib.ssm_state_step_multi.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
         lib.ssm_selective_scan_bwd.restype = i
         lib.ssm_selective_scan_bwd.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, vp,
                                                vp, vp, vp, vp, vp, vp, vp, vp, vp,
@@ -146,6 +148,16 @@ def ssm_state_step(state, x, delta, A, B, C, D, z, y, stream=None):
     _check(load_library().ssm_state_step(
         _ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(y),
         batch, dim, N, _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, state, y)))
+
+
+def ssm_state_step_multi(state, x, delta, A, B, C, D, z, y, stream=None):
+    """Several decode tokens on the carried state (see include/ssm.h): state [batch, dim, N]
+    fp32 updated in place; x, delta, z, y [ntok, batch, dim]; B, C [ntok, batch, N]."""
+    batch, dim, N = state.shape
+    ntok = x.shape[0]
+    _check(load_library().ssm_state_step_multi(
+        _ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(y),
+        ntok, batch, dim, N, _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, state, y)))
 
 
 def ssm_selective_scan_bwd(x, delta, delta_bias, delta_softplus, A, B, C, D, z, initial_state,

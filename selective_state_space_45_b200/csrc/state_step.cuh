@@ -27,6 +27,8 @@ struct StepArgs {
     const void *z;
     void *y;
     int batch, dim, dstate;
+    int ntok;             // tokens per call (state_steps_kernel): x, delta, z, y are
+                          // [ntok][batch][dim], B, C [ntok][batch][dstate]
 };
 
 // 4 consecutive input values (8 or 16 bytes, aligned) as fp32.
@@ -126,6 +128,96 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
             if (p.z != nullptr) yv *= silu_f(zv[j]);
             static_cast<Tout *>(p.y)[chs[j]] = from_f32<Tout>(yv);
         }
+    }
+}
+
+// Several decode tokens per call (speculative or chunked decoding): the state of a
+// channel-quad is loaded once, carried through the ntok tokens in registers and stored
+// once, so the state traffic is that of one step whatever ntok is.  Per token the
+// arithmetic is the one-step kernel's, in the same order: ntok chained one-token calls
+// give bit-identical results.
+template <int NP, typename Tin, typename Tout, bool VEC4>
+__global__ void __launch_bounds__(256) state_steps_kernel(const StepArgs p) {
+    constexpr int G = NP / 4;
+    const long long nquad = (long long)p.batch * p.dim * G;
+    const long long chans = (long long)p.batch * p.dim;
+    const int N = p.dstate;
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool act = g < nquad;
+    const long long q = act ? g : 0;          // inactive lanes still join the shuffles
+    const long long ch = q / G;
+    const int r = int(q - ch * G);
+    const int b = int(ch / p.dim);
+    const int d = int(ch - (long long)b * p.dim);
+    const int n0 = 4 * r;
+    float *hp = p.state + (size_t)ch * N + n0;
+    const float *Ap = p.A + (size_t)d * N + n0;
+    float h[4], a4[4];
+    if constexpr (VEC4) {
+        if (act && n0 < N) {
+            const float4 hv = *reinterpret_cast<const float4 *>(hp);
+            const float4 av = __ldg(reinterpret_cast<const float4 *>(Ap));
+            h[0] = hv.x; h[1] = hv.y; h[2] = hv.z; h[3] = hv.w;
+            a4[0] = av.x; a4[1] = av.y; a4[2] = av.z; a4[3] = av.w;
+        } else {
+#pragma unroll
+            for (int s = 0; s < 4; ++s) h[s] = a4[s] = 0.f;
+        }
+    } else {
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const bool ok = act && n0 + s < N;
+            h[s] = ok ? hp[s] : 0.f;
+            a4[s] = ok ? Ap[s] : 0.f;
+        }
+    }
+    const float Dv = p.D != nullptr ? p.D[d] : 0.f;
+    for (int t = 0; t < p.ntok; ++t) {
+        const size_t tc = (size_t)t * chans + ch;                  // [t][b][d]
+        const size_t tb = ((size_t)t * p.batch + b) * N + n0;      // [t][b][n]
+        const Tin *Bb = static_cast<const Tin *>(p.B) + tb;
+        const Tin *Cb = static_cast<const Tin *>(p.C) + tb;
+        float bb[4], cc[4];
+        if constexpr (VEC4) {
+            if (act && n0 < N) {
+                load4_nc<Tin>(Bb, bb);
+                load4_nc<Tin>(Cb, cc);
+            } else {
+#pragma unroll
+                for (int s = 0; s < 4; ++s) bb[s] = cc[s] = 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const bool ok = act && n0 + s < N;
+                bb[s] = ok ? to_f32(Bb[s]) : 0.f;
+                cc[s] = ok ? to_f32(Cb[s]) : 0.f;
+            }
+        }
+        const float dl = to_f32(static_cast<const Tin *>(p.delta)[tc]);
+        const float xv = to_f32(static_cast<const Tin *>(p.x)[tc]);
+        const float zv = p.z != nullptr ? to_f32(static_cast<const Tin *>(p.z)[tc]) : 0.f;
+        const float dx = dl * xv;
+        float acc = 0.f;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            h[s] = fmaf(ex2_approx(dl * a4[s] * kLog2e), h[s], dx * bb[s]);
+            acc = fmaf(cc[s], h[s], acc);
+        }
+#pragma unroll
+        for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (act && r == 0) {
+            float yv = fmaf(Dv, xv, acc);
+            if (p.z != nullptr) yv *= silu_f(zv);
+            static_cast<Tout *>(p.y)[tc] = from_f32<Tout>(yv);
+        }
+    }
+    if constexpr (VEC4) {
+        if (act && n0 < N) *reinterpret_cast<float4 *>(hp) = make_float4(h[0], h[1], h[2], h[3]);
+    } else {
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            if (act && n0 + s < N) hp[s] = h[s];
     }
 }
 

@@ -18,6 +18,7 @@ mamba130m      8       2048       1536     16   bf16 (A, D, bias, state fp32)
 mamba2p8b      4       4096       5120     16   bf16
 long1m         1       1048576    1536     16   bf16
 decode         256     1 x 64     5120     16   bf16 tokens, fp32 state
+decode4        256     4 x 16     5120     16   as decode, 4 tokens per call
 bwd130m        8       2048       1536     16   bf16 inputs, dy and gradients (backward)
 conv130m       8       2048       1536     --   bf16 x and u; width 4, fp32 taps/bias
 conv2p8b       4       4096       5120     --   bf16 x and u; width 4
@@ -49,6 +50,9 @@ CONFIGS = {
                    dt_dist="uniform"),
     "decode": dict(batch=256, steps=64, dim=5120, dstate=16, dtype=torch.bfloat16,
                    dt_dist="uniform"),
+    # the decode workload with 4 tokens per call on the carried state (speculative decoding)
+    "decode4": dict(batch=256, steps=64, dim=5120, dstate=16, dtype=torch.bfloat16,
+                    dt_dist="uniform", ntok=4),
     # the backward of the mamba130m-shaped scan (training), bf16 inputs and gradients
     "bwd130m": dict(batch=8, seqlen=2048, dim=1536, dstate=16, dtype=torch.bfloat16,
                     dt_dist="uniform"),
@@ -129,7 +133,7 @@ def make_config_inputs(name, device="cpu", seed=0):
     if name.startswith("conv"):
         return make_conv_inputs(c["batch"], c["dim"], c["seqlen"], c["width"], c["dtype"],
                                 device=device, seed=seed)
-    if name == "decode":
+    if name in ("decode", "decode4"):
         return make_decode_inputs(c["batch"], c["dim"], c["dstate"], c["steps"], c["dtype"],
                                   device=device, seed=seed)
     return make_scan_inputs(c["batch"], c["dim"], c["seqlen"], c["dstate"], c["dtype"],

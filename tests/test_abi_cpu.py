@@ -33,7 +33,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for expected in ("ssm_selective_scan_fwd", "ssm_selective_scan_fwd_ex", "ssm_selective_scan_fwd_noalloc",
                      "ssm_state_step", "ssm_causal_conv1d_fwd", "ssm_causal_conv1d_step",
-                     "ssm_selective_scan_bwd",
+                     "ssm_selective_scan_bwd", "ssm_state_step_multi",
                      "ssm_status_string", "ssm_version"):
         assert expected in names
 
@@ -215,6 +215,24 @@ def bwd(lib, **kw):
 ])
 def test_bwd_argument_checks(lib, kw, status):
     assert bwd(lib, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(state=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(ntok=-1), ssm.SSM_ERR_INVALID_ARG),
+    (dict(N=17), ssm.SSM_ERR_UNSUPPORTED),
+    (dict(y=MIS), ssm.SSM_ERR_ALIGNMENT),
+    (dict(ntok=0), ssm.SSM_OK),
+    (dict(batch=0), ssm.SSM_OK),
+])
+def test_step_multi_argument_checks(lib, kw, status):
+    args = dict(state=P, x=P, delta=P, A=P, B=P, C=P, D=P, z=P, y=P, ntok=4, batch=2, dim=3, N=16,
+                din=ssm.SSM_BF16, dout=ssm.SSM_BF16)
+    args.update(kw)
+    assert lib.ssm_state_step_multi(args["state"], args["x"], args["delta"], args["A"], args["B"],
+                                    args["C"], args["D"], args["z"], args["y"], args["ntok"],
+                                    args["batch"], args["dim"], args["N"], args["din"],
+                                    args["dout"], None) == status
 
 
 def test_python_binding_raises_on_error(lib):

@@ -131,3 +131,14 @@ def test_bwd_counts_mamba130m():
 def test_bwd_oracle_rate_single_core():
     r = bench.oracle_rate("bwd130m", threads=4, budget_s=0.2)
     assert r["kind"] == "oracle" and r["cores"] == 1 and r["value"] > 0
+
+
+def test_multi_token_decode_counts():
+    one = bench.step_counts(256, 5120, 16, 2, 2)
+    four = bench.steps_counts(4, 256, 5120, 16, 2, 2)
+    state = 2 * 256 * 5120 * 16 * 4
+    params = 5120 * 16 * 4 + 5120 * 4
+    assert four["tokch"] == 4 * one["tokch"]
+    assert four["bytes"] == state + 4 * (one["bytes"] - state - params) + params
+    r = bench.oracle_rate("decode4", threads=2, budget_s=0.1)
+    assert r["value"] > 0 and r["cores"] == 1

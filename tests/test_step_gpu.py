@@ -99,3 +99,45 @@ def test_chain_from_zero_equals_gpu_scan(cuda_lib, din, dout):
     torch.cuda.synchronize()
     assert_parity(y_step, to64(y_scan), din, dout, what="y chain vs scan")
     assert_parity(state, to64(fs), din, torch.float32, what="state chain vs scan")
+
+
+@pytest.mark.parametrize("ntok,batch,dim,N,din,dout", [
+    (4, 3, 40, 16, torch.bfloat16, torch.bfloat16),
+    (1, 2, 33, 5, torch.float32, torch.float32),
+    (7, 2, 17, 8, torch.float32, torch.bfloat16),
+    (3, 4, 64, 16, torch.bfloat16, torch.float32),
+])
+def test_multi_token_step_matches_chained_steps_and_oracle(cuda_lib, ntok, batch, dim, N, din, dout):
+    inp = inputs.make_decode_inputs(batch, dim, N, ntok, din, device=DEV, seed=ntok + dim)
+    st_multi = inp["state"].clone()
+    y_multi = torch.empty(ntok, batch, dim, device=DEV, dtype=dout)
+    cuda_lib.ssm_state_step_multi(st_multi, inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                                  inp["D"], inp["z"], y_multi)
+    st_chain = inp["state"].clone()
+    ys = []
+    for t in range(ntok):
+        # fresh copies: every pointer the library takes is 16-byte aligned
+        y = torch.empty(batch, dim, device=DEV, dtype=dout)
+        cuda_lib.ssm_state_step(st_chain, inp["x"][t].clone(), inp["delta"][t].clone(), inp["A"],
+                                inp["B"][t].clone(), inp["C"][t].clone(), inp["D"],
+                                inp["z"][t].clone(), y)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert torch.equal(st_multi, st_chain)                 # same arithmetic, same order
+    assert torch.equal(y_multi, torch.stack(ys))
+    h = to64(inp["state"])
+    for t in range(ntok):
+        yr, h = oracle.step(h, inp["x"][t], inp["delta"][t], inp["A"], inp["B"][t], inp["C"][t],
+                            D=inp["D"], z=inp["z"][t])
+        assert_parity(y_multi[t], yr, din, dout, what="y[%d]" % t)
+    assert_parity(st_multi, h, din, torch.float32, what="state")
+
+
+def test_multi_token_step_with_no_tokens_keeps_state(cuda_lib):
+    inp = inputs.make_decode_inputs(2, 8, 16, 1, torch.float32, device=DEV, seed=1)
+    st = inp["state"].clone()
+    cuda_lib.ssm_state_step_multi(st, inp["x"][:0], inp["delta"][:0], inp["A"], inp["B"][:0],
+                                  inp["C"][:0], inp["D"], inp["z"][:0],
+                                  torch.empty(0, 2, 8, device=DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(st, inp["state"])
