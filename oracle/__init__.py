@@ -14,5 +14,7 @@ from .oracle import (  # noqa: F401
     scan,
     scan_bwd,
     scan_parallel_reference,
+    ssd_chunked,
+    ssd_loop,
     step,
 )

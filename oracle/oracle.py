@@ -24,6 +24,10 @@ Functions and the passages they follow:
 ``scan_bwd``        gradients of the scan by reverse-mode differentiation of the same
                     recurrence (Euler gain): the training half; xmarva lesson 10,
                     section 6 (Mamba's kernel recomputes the states in the backward pass).
+``ssd_loop`` / ``ssd_chunked``  Mamba-2's state-space dual (scalar decay per head, a
+                    P x N state per head): the step-by-step loop and the chunked form,
+                    attention inside chunks and the recurrence between them; xmarva
+                    lesson 10, section 8 "Mamba-2: the same model as attention".
 ``causal_conv1d`` / ``conv1d_step``  the causal depthwise convolution with SiLU in front of
                               the scan, and its one-token window form: learnllm "Module 19",
                               "The Causal Convolution"; xmarva lesson 10, sections 4 and 7.
@@ -73,6 +77,8 @@ def _load():
             lib.oracle_scan_bwd.restype = ctypes.c_int
             lib.oracle_scan_bwd.argtypes = [p, p, p, ctypes.c_int, p, p, p, p, p, p, p, p,
                                             p, p, p, p, p, p, p, p, p, i64, i64, i64, i64]
+            lib.oracle_ssd_loop.restype = ctypes.c_int
+            lib.oracle_ssd_loop.argtypes = [p, p, p, p, p, p, p, i64, i64, i64, i64, i64]
             lib.oracle_causal_conv1d.restype = None
             lib.oracle_causal_conv1d.argtypes = [p, p, p, p, ctypes.c_int, p, p, i64, i64, i64, i64]
             lib.oracle_conv1d_step.restype = None
@@ -187,6 +193,75 @@ def scan_bwd(dy, x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softp
     if rc != 0:
         raise ValueError("oracle.scan_bwd: unsupported sizes")
     return out
+
+
+def ssd_loop(x, a, B, C, h0=None):
+    """Mamba-2 SSD as its step-by-step recurrence, in fp64: returns ``(y, final_state)``.
+
+    x [batch, L, heads, P] (already times the step), a [batch, L, heads] (= step * A),
+    B, C [batch, L, heads, N], h0 [batch, heads, P, N].  y [batch, L, heads, P].
+    """
+    x = _f64(x)
+    batch, L, heads, P = x.shape
+    a = _f64(a, (batch, L, heads))
+    B = _f64(B)
+    N = B.shape[-1]
+    B = _f64(B, (batch, L, heads, N))
+    C = _f64(C, (batch, L, heads, N))
+    h0 = _f64(h0, (batch, heads, P, N))
+    y = np.empty((batch, L, heads, P))
+    hN = np.empty((batch, heads, P, N))
+    if _load().oracle_ssd_loop(_ptr(x), _ptr(a), _ptr(B), _ptr(C), _ptr(h0), _ptr(y), _ptr(hN),
+                               batch, L, heads, P, N) != 0:
+        raise ValueError("oracle.ssd_loop: bad sizes")
+    return y, hN
+
+
+def _segment_sums(a):
+    """a [..., T] -> [..., T, T]: entry (t, s) = a[s+1] + ... + a[t] for s <= t, -inf above
+    the diagonal (so that exp() gives the decay mask)."""
+    T = a.shape[-1]
+    cs = np.cumsum(a, axis=-1)
+    out = cs[..., :, None] - cs[..., None, :]
+    return np.where(np.tril(np.ones((T, T), dtype=bool)), out, -np.inf)
+
+
+def ssd_chunked(x, a, B, C, chunk=64, h0=None):
+    """Mamba-2 SSD by chunks, in fp64 numpy: attention with the decay mask inside each chunk,
+    the recurrence between chunks (xmarva lesson 10, section 8: the four steps).  Returns
+    ``(y, final_state)``; the same layouts as ``ssd_loop``."""
+    x, a, B, C = (_f64(v) for v in (x, a, B, C))
+    batch, L, heads, P = x.shape
+    N = B.shape[-1]
+    pad = (-L) % chunk
+    if pad:
+        x = np.concatenate([x, np.zeros((batch, pad, heads, P))], axis=1)
+        a = np.concatenate([a, np.zeros((batch, pad, heads))], axis=1)
+        B = np.concatenate([B, np.zeros((batch, pad, heads, N))], axis=1)
+        C = np.concatenate([C, np.zeros((batch, pad, heads, N))], axis=1)
+    nc = x.shape[1] // chunk
+    xc = x.reshape(batch, nc, chunk, heads, P)
+    Bc = B.reshape(batch, nc, chunk, heads, N)
+    Cc = C.reshape(batch, nc, chunk, heads, N)
+    ac = a.reshape(batch, nc, chunk, heads).transpose(0, 3, 1, 2)       # [b, h, c, l]
+    acum = np.cumsum(ac, axis=-1)
+    # (1) inside a chunk: y_l = sum_{s<=l} (C_l . B_s) exp(a_{s+1} + .. + a_l) x_s
+    mask = np.exp(_segment_sums(ac))                                      # [b, h, c, l, s]
+    y_in = np.einsum("bclhn,bcshn,bhcls,bcshp->bclhp", Cc, Bc, mask, xc)
+    # (2) what each chunk adds to the state: sum_s exp(a_{s+1} + .. + a_end) x_s B_s^T
+    to_end = np.exp(acum[..., -1:] - acum)                                # [b, h, c, l]
+    adds = np.einsum("bclhn,bhcl,bclhp->bchpn", Bc, to_end, xc)           # [b, c, h, p, n]
+    # (3) the state entering each chunk: S_0 = h0, S_{c+1} = exp(sum a of chunk c) S_c + adds_c
+    decay = np.exp(acum[..., -1])                                         # [b, h, c]
+    S = np.zeros((batch, heads, P, N)) if h0 is None else _f64(h0, (batch, heads, P, N)).copy()
+    entering = np.empty((batch, nc, heads, P, N))
+    for ci in range(nc):
+        entering[:, ci] = S
+        S = decay[:, :, ci][..., None, None] * S + adds[:, ci]
+    # (4) what each position reads from the state that entered its chunk
+    y_en = np.einsum("bclhn,bchpn,bhcl->bclhp", Cc, entering, np.exp(acum))
+    y = (y_in + y_en).reshape(batch, nc * chunk, heads, P)[:, :L]
+    return y, S
 
 
 def causal_conv1d(x, weight, bias=None, hist=None, silu=True):

@@ -355,3 +355,51 @@ int oracle_scan_bwd(const double *x, const double *delta, const double *delta_bi
     free(hs);
     return 0;
 }
+
+/*
+ * Mamba-2 state-space dual (SSD) recurrence, written out as the step-by-step loop of the
+ * xmarva lesson 10, section 8 "Mamba-2: the same model as attention": one scalar decay per
+ * head, the state of a head a P x N matrix.  Per sequence b and head h, from S = h0 (zero
+ * if absent):
+ *     for t:  S[p][n] = exp(a[b,t,h]) * S[p][n] + x[b,t,h,p] * B[b,t,h,n]
+ *             y[b,t,h,p] = sum_n S[p][n] * C[b,t,h,n]
+ * x already carries the step (x = Delta * input) and a = Delta * A, as in that section.
+ *   x, y: [batch][L][heads][P];  a: [batch][L][heads];  B, C: [batch][L][heads][N]
+ *   h0, hN: [batch][heads][P][N] (NULL: zero start / not wanted)
+ * Returns 0, or -1 on a failed allocation or bad sizes.
+ */
+int oracle_ssd_loop(const double *x, const double *a, const double *B, const double *C,
+                    const double *h0, double *y, double *hN,
+                    int64_t batch, int64_t L, int64_t heads, int64_t P, int64_t N)
+{
+    if (batch < 0 || L < 0 || heads < 0 || P < 1 || N < 1)
+        return -1;
+    double *S = (double *)malloc(sizeof(double) * (size_t)(P * N));
+    if (!S)
+        return -1;
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t h = 0; h < heads; ++h) {
+            for (int64_t i = 0; i < P * N; ++i)
+                S[i] = h0 ? h0[((b * heads + h) * P) * N + i] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const double e = exp(a[(b * L + t) * heads + h]);
+                const double *x_t = x + ((b * L + t) * heads + h) * P;
+                const double *B_t = B + ((b * L + t) * heads + h) * N;
+                const double *C_t = C + ((b * L + t) * heads + h) * N;
+                double *y_t = y + ((b * L + t) * heads + h) * P;
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) {
+                        S[p * N + n] = e * S[p * N + n] + x_t[p] * B_t[n];
+                        acc += S[p * N + n] * C_t[n];
+                    }
+                    y_t[p] = acc;
+                }
+            }
+            if (hN)
+                for (int64_t i = 0; i < P * N; ++i)
+                    hN[((b * heads + h) * P) * N + i] = S[i];
+        }
+    free(S);
+    return 0;
+}

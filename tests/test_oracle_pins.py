@@ -486,3 +486,98 @@ def test_scan_bwd_gate_and_skip_closed_form():
     # the state never reaches y, so x's gradient is the skip's alone
     np.testing.assert_allclose(g["dx"][0, 0], dy * zs * s, rtol=1e-14, atol=1e-15)
     np.testing.assert_allclose(g["dD"], [np.sum(dy * zs * s * x)], rtol=1e-14)
+
+
+# ----------------------------------------------------------------------------------
+# Mamba-2 SSD (xmarva lesson 10, section 8): the loop, the chunked form, the attention form
+# ----------------------------------------------------------------------------------
+
+def _ssd_case(rng, batch=1, L=150, heads=3, P=8, N=16):
+    return (rng.normal(size=(batch, L, heads, P)), -rng.random((batch, L, heads)) * 0.3,
+            rng.normal(size=(batch, L, heads, N)), rng.normal(size=(batch, L, heads, N)))
+
+
+def test_ssd_loop_equals_the_printed_attention_form():
+    # y_t = sum_{s<=t} (c_t . b_s) exp(a_{s+1} + ... + a_t) x_s, summed term by term
+    rng = np.random.default_rng(41)
+    x, a, b, c = _ssd_case(rng, batch=2, L=9, heads=2, P=3, N=4)
+    y, _ = oracle.ssd_loop(x, a, b, c)
+    brute = np.zeros_like(y)
+    for bi in range(2):
+        for h in range(2):
+            for t in range(9):
+                for s in range(t + 1):
+                    w = np.dot(c[bi, t, h], b[bi, s, h]) * math.exp(a[bi, s + 1:t + 1, h].sum())
+                    brute[bi, t, h] += w * x[bi, s, h]
+    np.testing.assert_allclose(y, brute, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64, 150, 256])
+def test_ssd_chunked_equals_loop(chunk):
+    rng = np.random.default_rng(43)
+    x, a, b, c = _ssd_case(rng)
+    y, hN = oracle.ssd_loop(x, a, b, c)
+    yc, hc = oracle.ssd_chunked(x, a, b, c, chunk=chunk)
+    np.testing.assert_allclose(yc, y, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(hc, hN, rtol=0, atol=1e-11)
+
+
+def test_ssd_chunked_fp32_difference_is_of_the_printed_order():
+    g = load_golden("ssd_chunk_vs_loop.json")
+    rng = np.random.default_rng(47)
+    x, a, b, c = (v.astype(np.float32) for v in _ssd_case(rng))
+    y, _ = oracle.ssd_loop(x, a, b, c)                      # fp64 of the fp32 inputs
+    # the chunked form evaluated in single precision (numpy float32 throughout)
+    cs = [v.astype(np.float32) for v in (x, a, b, c)]
+    L, chunk = 150, g["chunk"]
+    pad = (-L) % chunk
+    xp, ap, bp, cp = (np.concatenate([v, np.zeros((1, pad) + v.shape[2:], np.float32)], axis=1) for v in cs)
+    nc = xp.shape[1] // chunk
+    xr, br, cr = (v.reshape(1, nc, chunk, 3, -1) for v in (xp, bp, cp))
+    ar = ap.reshape(1, nc, chunk, 3).transpose(0, 3, 1, 2)
+    acum = np.cumsum(ar, axis=-1, dtype=np.float32)
+    seg = acum[..., :, None] - acum[..., None, :]
+    mask = np.where(np.tril(np.ones((chunk, chunk), bool)), np.exp(seg), np.float32(0))
+    y_in = np.einsum("bclhn,bcshn,bhcls,bcshp->bclhp", cr, br, mask, xr)
+    adds = np.einsum("bclhn,bhcl,bclhp->bchpn", br, np.exp(acum[..., -1:] - acum), xr)
+    S = np.zeros((1, 3, 8, 16), np.float32)
+    ent = np.empty((1, nc, 3, 8, 16), np.float32)
+    for ci in range(nc):
+        ent[:, ci] = S
+        S = np.exp(acum[..., ci, -1])[..., None, None] * S + adds[:, ci]
+    y_en = np.einsum("bclhn,bchpn,bhcl->bclhp", cr, ent, np.exp(acum))
+    y32 = (y_in + y_en).reshape(1, nc * chunk, 3, 8)[:, :L]
+    diff = float(np.abs(y32 - y).max())
+    assert diff < 10 * g["printed_max_abs_difference_fp32"]
+    assert diff > 0.0                                        # single precision does round
+
+
+def test_ssd_loop_is_the_selective_scan_with_one_decay_per_head():
+    # per head: channels p share B, C and the decay; the S6 oracle with Delta_t, A = A_h
+    # for every (p, n) and input x / Delta gives the same outputs
+    rng = np.random.default_rng(53)
+    batch, L, heads, P, N = 2, 12, 2, 3, 5
+    step = rng.uniform(0.05, 0.6, size=(batch, L, heads))
+    A_h = -rng.uniform(0.2, 2.0, size=heads)
+    u = rng.normal(size=(batch, L, heads, P))
+    b = rng.normal(size=(batch, L, heads, N))
+    c = rng.normal(size=(batch, L, heads, N))
+    y, hN = oracle.ssd_loop(u * step[..., None], step * A_h, b, c)
+    for h in range(heads):
+        ys, hs = oracle.scan(x=u[:, :, h, :].transpose(0, 2, 1),
+                             delta=np.repeat(step[:, None, :, h], P, axis=1),
+                             A=np.full((P, N), A_h[h]), B=b[:, :, h, :], C=c[:, :, h, :])
+        np.testing.assert_allclose(ys.transpose(0, 2, 1), y[:, :, h, :], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(hs, hN[:, h], rtol=1e-12, atol=1e-13)
+
+
+def test_ssd_resumes_from_its_final_state():
+    rng = np.random.default_rng(59)
+    x, a, b, c = _ssd_case(rng, batch=2, L=40, heads=2, P=4, N=6)
+    y, hN = oracle.ssd_loop(x, a, b, c)
+    y1, h1 = oracle.ssd_loop(x[:, :17], a[:, :17], b[:, :17], c[:, :17])
+    y2, h2 = oracle.ssd_loop(x[:, 17:], a[:, 17:], b[:, 17:], c[:, 17:], h0=h1)
+    np.testing.assert_allclose(np.concatenate([y1, y2], axis=1), y, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(h2, hN, rtol=1e-13, atol=1e-14)
+    yc, hc = oracle.ssd_chunked(x[:, 17:], a[:, 17:], b[:, 17:], c[:, 17:], chunk=8, h0=h1)
+    np.testing.assert_allclose(yc, y2, rtol=0, atol=1e-11)
