@@ -41,6 +41,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MHZ = 1965.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -52,7 +53,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba130m",
                     choices=["mamba130m", "mamba2p8b", "long1m", "decode", "tiny",
-                             "conv130m", "conv2p8b", "convstep", "bwd130m", "decode4"])
+                             "conv130m", "conv2p8b", "convstep", "bwd130m", "decode4", "ssd130m"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0,
@@ -109,15 +110,18 @@ def load_peaks():
     try:
         with open(PEAKS_FILE) as f:
             p = json.load(f)
+        bf16 = p.get("bf16_tflops")
         return dict(hbm_gbs=float(p["hbm_gbs"]), sm_max_mhz=float(p.get("sm_max_mhz", FALLBACK_SM_MHZ)),
+                    bf16_tflops=float(bf16) if bf16 is not None else FALLBACK_BF16_TFLOPS,
                     source="measured (MEASURED_PEAKS.json)")
     except (OSError, KeyError, ValueError):
-        return dict(hbm_gbs=FALLBACK_HBM_GBS, sm_max_mhz=FALLBACK_SM_MHZ, source="fallback")
+        return dict(hbm_gbs=FALLBACK_HBM_GBS, sm_max_mhz=FALLBACK_SM_MHZ,
+                    bf16_tflops=FALLBACK_BF16_TFLOPS, source="fallback")
 
 
 # translation unit of libssm.so that holds each kernel and its launch logic
 KERNEL_UNIT = {"scan_fwd_kernel": "scan_api.cu", "state_step_kernel": "step_api.cu",
-               "state_steps_kernel": "step_api.cu",
+               "state_steps_kernel": "step_api.cu", "ssd_fwd_kernel": "ssd_api.cu",
                "scan_bwd_kernel": "bwd_api.cu",
                "causal_conv1d_vec_kernel": "conv_api.cu", "conv1d_step_kernel": "conv_api.cu"}
 
@@ -226,7 +230,20 @@ def bwd_counts(batch, dim, L, N, in_size, g_size):
     return dict(bytes=streams + bc + params, exps=2 * batch * L * dim * N, tokch=batch * L * dim)
 
 
+def ssd_counts(batch, L, heads, P, N, in_size, out_size, Q=64):
+    """SSD by chunks: x, B, C, a read once and y written once; work = the four chunk products
+    (scores C B^T, masked scores times x, C times the entering state, B^T times the weighted
+    inputs), 2 flops per multiply-add, over whole chunks."""
+    toks = batch * L * heads
+    byts = toks * (P * in_size + 2 * N * in_size + 4 + P * out_size)
+    nchunk = batch * heads * (-(-L // Q))
+    flops = nchunk * 2 * (Q * Q * N + Q * Q * P + 2 * Q * N * P)
+    return dict(bytes=byts, flops=flops, exps=0, tokch=toks * P)
+
+
 def workload_kind(name):
+    if name.startswith("ssd"):
+        return "ssd"
     if name.startswith("bwd"):
         return "bwd"
     if name == "decode4":
@@ -272,6 +289,9 @@ class Workload:
         esz = torch.tensor([], dtype=dt).element_size()
         if self.kind == "scan":
             self.counts = scan_counts(c["batch"], c["dim"], c["seqlen"], c["dstate"], esz, esz)
+        elif self.kind == "ssd":
+            self.counts = ssd_counts(c["batch"], c["seqlen"], c["heads"], c["headdim"], c["dstate"],
+                                     esz, esz)
         elif self.kind == "bwd":
             self.counts = bwd_counts(c["batch"], c["dim"], c["seqlen"], c["dstate"], esz, esz)
         elif self.kind == "decode":
@@ -290,6 +310,8 @@ class Workload:
             if self.kind == "scan":
                 inp["y"] = torch.empty(inp["x"].shape, device=device, dtype=dt)
                 inp["fs"] = torch.empty(c["batch"], c["dim"], c["dstate"], device=device)
+            elif self.kind == "ssd":
+                inp["y"] = torch.empty(inp["x"].shape, device=device, dtype=dt)
             elif self.kind == "bwd":
                 for k in ("dx", "ddelta", "dz"):
                     inp[k] = torch.empty(inp["x"].shape, device=device, dtype=dt)
@@ -314,6 +336,8 @@ class Workload:
         if self.kind == "scan":
             ssm.ssm_selective_scan_fwd(s["x"], s["delta"], s["delta_bias"], True, s["A"], s["B"],
                                        s["C"], s["D"], s["z"], s["y"], s["fs"], stream)
+        elif self.kind == "ssd":
+            ssm.ssm_ssd_fwd(s["x"], s["a"], s["B"], s["C"], s["y"], None, None, stream)
         elif self.kind == "decodemulti":
             k = self.cfg["ntok"]
             t = ((i // self.nsets) % (s["x"].shape[0] // k)) * k
@@ -346,6 +370,10 @@ class Workload:
         if self.kind == "convstep":
             return ("decode conv1d step: batch %d, d_inner %d, width %d, fp32 window in place, one %s "
                     "token per sequence" % (c["batch"], c["dim"], c["width"], io))
+        if self.kind == "ssd":
+            return ("%s-shaped Mamba-2 SSD by 64-token chunks: batch %d, L %d, %d heads x %d, state %d, "
+                    "%s x/B/C and y, fp32 a" % (self.name[3:], c["batch"], c["seqlen"], c["heads"],
+                                               c["headdim"], c["dstate"], io))
         if self.kind == "decodemulti":
             return ("decode, %d tokens per call on the carried state: batch %d, d_inner %d, N %d, "
                     "fp32 state in place, %s tokens" % (c["ntok"], c["batch"], c["dim"], c["dstate"], io))
@@ -364,7 +392,7 @@ class Workload:
 def kernel_name(kind):
     return dict(scan="scan_fwd_kernel", decode="state_step_kernel", conv="causal_conv1d_vec_kernel",
                 convstep="conv1d_step_kernel", bwd="scan_bwd_kernel",
-                decodemulti="state_steps_kernel")[kind]
+                decodemulti="state_steps_kernel", ssd="ssd_fwd_kernel")[kind]
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -409,6 +437,13 @@ def _oracle_sample(name, n_target_tokch, seed=0):
                                           seed=seed)
         return kind, inp, per_channel * k, "%d sequences x %d of %d channels, all %d tokens" % (
             c["batch"], k, c["dim"], L)
+    if kind == "ssd":
+        per_head = c["batch"] * c["seqlen"] * c["headdim"]
+        k = int(max(1, min(c["heads"], n_target_tokch // per_head)))
+        inp = inputs.make_ssd_inputs(c["batch"], c["seqlen"], k, c["headdim"], c["dstate"], c["dtype"],
+                                     device="cpu", seed=seed)
+        return kind, inp, per_head * k, "%d sequences x %d of %d heads, all %d tokens" % (
+            c["batch"], k, c["heads"], c["seqlen"])
     if kind == "decodemulti":
         k = int(max(1, min(c["dim"], n_target_tokch // (c["batch"] * c["ntok"]))))
         inp = inputs.make_decode_inputs(c["batch"], k, c["dstate"], c["ntok"], c["dtype"], device="cpu",
@@ -442,6 +477,8 @@ def _oracle_call(kind, inp, threads):
     if kind == "scan":
         oracle.scan(x=inp["x"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], D=inp["D"],
                     z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True, nthreads=threads)
+    elif kind == "ssd":
+        oracle.ssd_loop(inp["x"], inp["a"], inp["B"], inp["C"])
     elif kind == "decodemulti":
         h = inp["state"]
         for t in range(inp["x"].shape[0]):
@@ -545,6 +582,7 @@ def time_e2e(wl, steps, stream):
              ["dx", "ddelta", "dz", "dB", "dC", "dA", "dD", "dbias"]),
         decode=(["state", "x", "delta", "z", "B", "C", "A", "D"], ["y", "state"]),
         decodemulti=(["state", "x", "delta", "z", "B", "C", "A", "D"], ["y", "state"]),
+        ssd=(["x", "a", "B", "C"], ["y"]),
         conv=(["x", "weight", "bias"], ["u", "fw"]),
         convstep=(["window", "x", "weight", "bias"], ["u", "window"]))[wl.kind]
 
@@ -568,6 +606,8 @@ def time_e2e(wl, steps, stream):
         if wl.kind == "scan":
             ssm.ssm_selective_scan_fwd(dev["x"], dev["delta"], dev["delta_bias"], True, dev["A"],
                                        dev["B"], dev["C"], dev["D"], dev["z"], dev["y"], dev["fs"])
+        elif wl.kind == "ssd":
+            ssm.ssm_ssd_fwd(dev["x"], dev["a"], dev["B"], dev["C"], dev["y"])
         elif wl.kind == "decodemulti":
             ssm.ssm_state_step_multi(dev["state"], dev_view("x"), dev_view("delta"), dev["A"],
                                      dev_view("B"), dev_view("C"), dev["D"], dev_view("z"), dev["y"])
@@ -668,6 +708,16 @@ def run_ours(args):
                     peak_basis="148 SMs x 16 ex2/clk/SM x %.0f MHz max SM clock" % peaks["sm_max_mhz"],
                     hbm=dict(achieved_gbs=gbs, peak_gbs=peaks["hbm_gbs"], frac=gbs / peaks["hbm_gbs"],
                              peak_source=peaks["source"]))
+    elif wl.kind == "ssd":
+        tfl = wl.counts["flops"] / kern_s / 1e12
+        roof = dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                    frac=gbs / peaks["hbm_gbs"],
+                    traffic=recorded_traffic(kernel_name(wl.kind), wl.name),
+                    kernel=kernel_name(wl.kind), kernel_ms=kern_ms,
+                    peak_basis="measured copy bandwidth, burst (%s)" % peaks["source"],
+                    tensor=dict(achieved_tflops=tfl, peak_tflops=peaks.get("bf16_tflops"),
+                                frac=(tfl / peaks["bf16_tflops"]) if peaks.get("bf16_tflops") else None,
+                                note="bf16 tensor-core work of the chunk products"))
     else:
         roof = dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
                     frac=gbs / peaks["hbm_gbs"],
@@ -681,7 +731,8 @@ def run_ours(args):
 
     if rank == 0:
         c = wl.cfg
-        config = dict(workload=wl.description(), batch=c["batch"], d_inner=c["dim"],
+        config = dict(workload=wl.description(), batch=c["batch"],
+                      d_inner=c.get("dim", c.get("heads", 0) * c.get("headdim", 0)),
                       parallelism="replicas x%d" % world,
                       l2=("%d rotating input sets of %.0f MB (%.0f MB touched per cycle) > 126 MB L2"
                           % (wl.nsets, wl.counts["bytes"] / 1e6, wl.nsets * wl.counts["bytes"] / 1e6)))
@@ -689,6 +740,8 @@ def run_ours(args):
             config.update(dstate=c["dstate"])
         if "width" in c:
             config.update(width=c["width"])
+        if "heads" in c:
+            config.update(heads=c["heads"], headdim=c["headdim"], chunk=64)
         if "seqlen" in c:
             config.update(seqlen=c["seqlen"], global_batch=c["batch"] * world)
         line = dict(metric=METRIC, value=total_units / sec, unit=UNIT, n_gpus=world, steps=args.steps,

@@ -7,7 +7,8 @@
  *   ssm_state_step_multi    several decode tokens on a carried state in one call;
  *   ssm_causal_conv1d_fwd   the causal depthwise convolution + SiLU that feeds the scan;
  *   ssm_causal_conv1d_step  its one-token form on a carried window, updated in place;
- *   ssm_selective_scan_bwd  the gradients of the scan (training), states recomputed.
+ *   ssm_selective_scan_bwd  the gradients of the scan (training), states recomputed;
+ *   ssm_ssd_fwd             Mamba-2's state-space dual by chunks, on tensor cores.
  *
  * The scan and the state step compute, per sequence b and channel d, with an N-wide fp32 state h:
  *     Delta_t = softplus(delta[b,d,t] + delta_bias[d])   (bias and softplus optional)
@@ -254,6 +255,29 @@ int ssm_state_step_multi(float *state, const void *x, const void *delta, const f
                          const void *B, const void *C, const float *D, const void *z, void *y,
                          int ntok, int batch, int dim, int dstate, int in_dtype, int out_dtype,
                          void *cuda_stream);
+
+/*
+ * Mamba-2's state-space dual (SSD) by chunks ("Beyond attention with Mamba, state space
+ * models and hybrids", xmarva lesson 10, section 8 "Mamba-2: the same model as
+ * attention"): one decay per head and a headdim x dstate state per head,
+ *     S <- exp(a_t) S + x_t B_t^T,    y_t = S C_t    (per sequence and head)
+ * computed as attention with the decay mask inside chunks of 64 tokens and the recurrence
+ * between chunks.  x already carries the step (x = Delta * input), a = Delta * A.
+ *
+ *   x, y          : [batch][seqlen][heads][headdim]; x bf16, y out_dtype (written).
+ *   a             : [batch][seqlen][heads] fp32.
+ *   B, C          : [batch][seqlen][heads][dstate] bf16.
+ *   initial_state : [batch][heads][headdim][dstate] fp32 or NULL (zero).
+ *   final_state   : [batch][heads][headdim][dstate] fp32 or NULL (not written).
+ * in_dtype must be SSM_BF16 (the tensor-core operands); headdim 32 or 64 and dstate 64 or
+ * 128 (SSM_ERR_UNSUPPORTED otherwise).  Products run on bf16 operands with fp32
+ * accumulation; the masked scores, the decay-weighted inputs and the state are rounded to
+ * bf16 where they enter a product.  seqlen = 0 copies the start state through.
+ */
+int ssm_ssd_fwd(const void *x, const float *a, const void *B, const void *C, void *y,
+                const float *initial_state, float *final_state,
+                int batch, int seqlen, int heads, int headdim, int dstate,
+                int in_dtype, int out_dtype, void *cuda_stream);
 
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char *ssm_status_string(int status);

@@ -1,5 +1,5 @@
 """B200 (sm_100a) selective state-space scan (S6): forward scan, its backward and the decode
-step, and the causal depthwise convolution in front of it.
+step, the causal depthwise convolution in front of it, and Mamba-2's chunked SSD.
 
 The computation lives in ``libssm.so`` (C ABI in ``include/ssm.h``); this package only
 loads it and marshals torch tensors into it.
@@ -19,12 +19,14 @@ from ._lib import (  # noqa: F401
     load_library,
     selective_scan,
     selective_scan_bwd,
+    ssd,
     ssm_causal_conv1d_fwd,
     ssm_causal_conv1d_step,
     ssm_selective_scan_bwd,
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_ex,
     ssm_selective_scan_fwd_noalloc,
+    ssm_ssd_fwd,
     ssm_state_step,
     ssm_state_step_multi,
     ssm_status_string,

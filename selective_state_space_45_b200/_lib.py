@@ -57,6 +57,8 @@ def load_library(path: str | None = None):
         lib.ssm_causal_conv1d_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
         lib.ssm_causal_conv1d_step.restype = i
         lib.ssm_causal_conv1d_step.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+        lib.ssm_ssd_fwd.restype = i
+        lib.ssm_ssd_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
         lib.ssm_state_step_multi.restype = i
         lib.ssm_state_step_multi.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
         lib.ssm_selective_scan_bwd.restype = i
@@ -148,6 +150,26 @@ def ssm_state_step(state, x, delta, A, B, C, D, z, y, stream=None):
     _check(load_library().ssm_state_step(
         _ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(y),
         batch, dim, N, _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, state, y)))
+
+
+def ssm_ssd_fwd(x, a, B, C, y, initial_state=None, final_state=None, stream=None):
+    """Mamba-2 SSD by chunks (see include/ssm.h): x, y [batch, L, heads, P]; a [batch, L,
+    heads] fp32; B, C [batch, L, heads, N] bf16; states [batch, heads, P, N] fp32."""
+    batch, L, heads, P = x.shape
+    N = B.shape[-1]
+    _check(load_library().ssm_ssd_fwd(
+        _ptr(x), _ptr(a), _ptr(B), _ptr(C), _ptr(y), _ptr(initial_state), _ptr(final_state),
+        batch, L, heads, P, N, _DTYPE_CODE[x.dtype], _DTYPE_CODE[y.dtype], _stream(stream, x, y)))
+
+
+def ssd(x, a, B, C, initial_state=None, out_dtype=None, return_final_state=True, stream=None):
+    """Allocate y (and the final state) with torch and run ``ssm_ssd_fwd``."""
+    batch, L, heads, P = x.shape
+    y = torch.empty(x.shape, device=x.device, dtype=out_dtype or torch.float32)
+    fs = (torch.empty((batch, heads, P, B.shape[-1]), device=x.device, dtype=torch.float32)
+          if return_final_state else None)
+    ssm_ssd_fwd(x, a, B, C, y, initial_state, fs, stream)
+    return (y, fs) if return_final_state else y
 
 
 def ssm_state_step_multi(state, x, delta, A, B, C, D, z, y, stream=None):

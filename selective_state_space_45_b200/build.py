@@ -20,7 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJDIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libssm.so")
-UNITS = ["ssm_api.cu", "scan_api.cu", "step_api.cu", "conv_api.cu", "bwd_api.cu"]
+UNITS = ["ssm_api.cu", "scan_api.cu", "step_api.cu", "conv_api.cu", "bwd_api.cu", "ssd_api.cu"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

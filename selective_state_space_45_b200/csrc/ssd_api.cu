@@ -1,0 +1,74 @@
+// ssd_api.cu -- C ABI of Mamba-2's state-space dual by chunks (ssm_ssd_fwd).
+//
+// Arguments are checked on the host before anything is launched; the kernel runs on the
+// caller's stream, asynchronously.
+#include <climits>
+
+#include "api_host.cuh"
+#include "ssd_fwd.cuh"
+
+using namespace ssm_host;
+
+namespace {
+
+template <int P, int N, typename Tout>
+int launch_ssd(const ssm::SsdArgs &a, cudaStream_t s) {
+    using Cfg = ssm::SsdCfg<P, N, Tout>;
+    const long long grid = (long long)a.batch * a.heads;
+    if (grid > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    if (grid == 0) return SSM_OK;
+    if (cudaFuncSetAttribute(ssm::ssd_fwd_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(Cfg::SMEM_BYTES)) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    ssm::ssd_fwd_kernel<Cfg><<<unsigned(grid), Cfg::NT, Cfg::SMEM_BYTES, s>>>(a);
+    return status_of(cudaGetLastError());
+}
+
+template <typename Tout>
+int dispatch_ssd(const ssm::SsdArgs &a, int P, int N, cudaStream_t s) {
+    if (P == 64 && N == 128) return launch_ssd<64, 128, Tout>(a, s);
+    if (P == 64 && N == 64) return launch_ssd<64, 64, Tout>(a, s);
+    if (P == 32 && N == 128) return launch_ssd<32, 128, Tout>(a, s);
+    if (P == 32 && N == 64) return launch_ssd<32, 64, Tout>(a, s);
+    return SSM_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssm_ssd_fwd(const void *x, const float *a, const void *B, const void *C, void *y,
+                const float *initial_state, float *final_state,
+                int batch, int seqlen, int heads, int headdim, int dstate,
+                int in_dtype, int out_dtype, void *cuda_stream) {
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return SSM_ERR_INVALID_ARG;
+    if (batch < 0 || seqlen < 0 || heads < 0 || headdim < 1 || dstate < 1) return SSM_ERR_INVALID_ARG;
+    if (in_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+    if (!((headdim == 32 || headdim == 64) && (dstate == 64 || dstate == 128))) return SSM_ERR_UNSUPPORTED;
+    const long long heads_total = (long long)batch * heads;
+    const bool work = heads_total > 0 && seqlen > 0;
+    if (work && (!x || !a || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, a, B, C, y, initial_state, final_state};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return SSM_ERR_ALIGNMENT;
+    if (heads_total == 0) return SSM_OK;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if (!work) {   // no tokens: the final state is the start state
+        if (!final_state) return SSM_OK;
+        const size_t bytes = size_t(heads_total) * headdim * dstate * sizeof(float);
+        if (initial_state)
+            return status_of(cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, stream));
+        return status_of(cudaMemsetAsync(final_state, 0, bytes, stream));
+    }
+    ssm::SsdArgs s{};
+    s.x = static_cast<const __nv_bfloat16 *>(x);
+    s.a = a;
+    s.B = static_cast<const __nv_bfloat16 *>(B);
+    s.C = static_cast<const __nv_bfloat16 *>(C);
+    s.y = y; s.h0 = initial_state; s.hN = final_state;
+    s.batch = batch; s.seqlen = seqlen; s.heads = heads;
+    if (out_dtype == SSM_F32) return dispatch_ssd<float>(s, headdim, dstate, stream);
+    return dispatch_ssd<__nv_bfloat16>(s, headdim, dstate, stream);
+}
+
+}  // extern "C"

@@ -20,6 +20,7 @@ long1m         1       1048576    1536     16   bf16
 decode         256     1 x 64     5120     16   bf16 tokens, fp32 state
 decode4        256     4 x 16     5120     16   as decode, 4 tokens per call
 bwd130m        8       2048       1536     16   bf16 inputs, dy and gradients (backward)
+ssd130m        8       2048       24 x 64  128  Mamba-2 SSD: bf16 x, B, C; fp32 a
 conv130m       8       2048       1536     --   bf16 x and u; width 4, fp32 taps/bias
 conv2p8b       4       4096       5120     --   bf16 x and u; width 4
 convstep       256     1 x 64     5120     --   bf16 tokens, fp32 window (width 4)
@@ -56,6 +57,8 @@ CONFIGS = {
     # the backward of the mamba130m-shaped scan (training), bf16 inputs and gradients
     "bwd130m": dict(batch=8, seqlen=2048, dim=1536, dstate=16, dtype=torch.bfloat16,
                     dt_dist="uniform"),
+    # Mamba-2's SSD in the 130m shape: 24 heads of 64 channels, state 128
+    "ssd130m": dict(batch=8, seqlen=2048, heads=24, headdim=64, dstate=128, dtype=torch.bfloat16),
     # the causal convolution in front of the scan, in the same block shapes (width 4)
     "conv130m": dict(batch=8, seqlen=2048, dim=1536, width=4, dtype=torch.bfloat16),
     "conv2p8b": dict(batch=4, seqlen=4096, dim=5120, width=4, dtype=torch.bfloat16),
@@ -122,8 +125,25 @@ def make_scan_bwd_inputs(batch, dim, seqlen, dstate, dtype=torch.bfloat16, devic
     return inp
 
 
+def make_ssd_inputs(batch, seqlen, heads, headdim, dstate, dtype=torch.bfloat16, device="cpu",
+                    seed=0):
+    """Inputs of one SSD call, following the worked example of the Mamba-2 section: x, B, C
+    ~ N(0, 1) in ``dtype`` (x [batch, L, heads, P], B, C [batch, L, heads, N]) and the
+    per-head log-decay a = -U[0, 0.3) fp32 [batch, L, heads].  Draw order: x, a, B, C."""
+    g = _generator(device, seed)
+    f32 = torch.float32
+    x = torch.randn(batch, seqlen, heads, headdim, generator=g, device=device, dtype=f32).to(dtype)
+    a = -0.3 * torch.rand(batch, seqlen, heads, generator=g, device=device, dtype=f32)
+    B = torch.randn(batch, seqlen, heads, dstate, generator=g, device=device, dtype=f32).to(dtype)
+    C = torch.randn(batch, seqlen, heads, dstate, generator=g, device=device, dtype=f32).to(dtype)
+    return dict(x=x, a=a, B=B, C=C)
+
+
 def make_config_inputs(name, device="cpu", seed=0):
     c = CONFIGS[name]
+    if name.startswith("ssd"):
+        return make_ssd_inputs(c["batch"], c["seqlen"], c["heads"], c["headdim"], c["dstate"],
+                               c["dtype"], device=device, seed=seed)
     if name == "convstep":
         return make_conv_step_inputs(c["batch"], c["dim"], c["steps"], c["width"], c["dtype"],
                                      device=device, seed=seed)

@@ -142,3 +142,22 @@ def test_multi_token_decode_counts():
     assert four["bytes"] == state + 4 * (one["bytes"] - state - params) + params
     r = bench.oracle_rate("decode4", threads=2, budget_s=0.1)
     assert r["value"] > 0 and r["cores"] == 1
+
+
+def test_ssd_counts():
+    c = bench.ssd_counts(8, 2048, 24, 64, 128, 2, 2)
+    toks = 8 * 2048 * 24
+    assert c["bytes"] == toks * (64 * 2 + 2 * 128 * 2 + 4 + 64 * 2)
+    assert c["flops"] == 8 * 24 * 32 * 2 * (64 * 64 * 128 + 64 * 64 * 64 + 2 * 64 * 128 * 64)
+    assert c["tokch"] == toks * 64
+    r = bench.oracle_rate("ssd130m", threads=2, budget_s=0.1)
+    assert r["value"] > 0
+
+
+@pytest.mark.parametrize("name", ["mamba130m", "decode", "ssd130m", "bwd130m", "decode4", "conv130m",
+                                  "convstep"])
+def test_oracle_sample_and_call_for_every_workload_kind(name):
+    kind, inp, units, what = bench._oracle_sample(name, 4096)
+    assert kind == bench.workload_kind(name) or (kind == "scan" and name == "mamba130m")
+    assert units > 0 and what
+    bench._oracle_call(kind, inp, 2)
