@@ -47,9 +47,13 @@ def dependency_files(unit: str) -> list[str]:
 
 
 def source_hash(unit: str) -> str:
-    """Short hash of a unit's sources: names the exact device code and launch logic."""
+    """Short hash of a unit's sources under csrc/ (kernels, helpers, launch logic): names the
+    exact device code and launch configuration.  The public header holds declarations only
+    and is left out, so documenting a new entry point does not change the hash."""
     h = hashlib.sha256()
     for path in dependency_files(unit):
+        if not path.startswith(CSRC):
+            continue
         with open(path, "rb") as f:
             h.update(os.path.basename(path).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
