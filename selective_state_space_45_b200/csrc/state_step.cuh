@@ -133,12 +133,24 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
 
 // Several decode tokens per call (speculative or chunked decoding): the state of a
 // channel-quad is loaded once, carried through the ntok tokens in registers and stored
-// once, so the state traffic is that of one step whatever ntok is.  Per token the
-// arithmetic is the one-step kernel's, in the same order: ntok chained one-token calls
-// give bit-identical results.
+// once, so the state traffic is that of one step whatever ntok is.  The token inputs of a
+// round of up to kStepsRound tokens are first staged in shared memory by the whole block,
+// every load independent of the others, so no thread waits on one token's loads before
+// issuing the next token's.  Per token the arithmetic is the one-step kernel's, in the
+// same order: ntok chained one-token calls give bit-identical results.
+constexpr int kStepsRound = 8;
+
+// Shared memory of one block of state_steps_kernel: per round token, x, delta, z of the
+// block's channels and B, C of the sequences they belong to (nb of them).
+__host__ __device__ constexpr size_t steps_smem_bytes(int ch_per_block, int nb, int N) {
+    return size_t(kStepsRound) * (3 * size_t(ch_per_block) + 2 * size_t(nb) * N) * sizeof(float);
+}
+
 template <int NP, typename Tin, typename Tout, bool VEC4>
-__global__ void __launch_bounds__(256) state_steps_kernel(const StepArgs p) {
+__global__ void __launch_bounds__(256) state_steps_kernel(const StepArgs p, int nb_max) {
     constexpr int G = NP / 4;
+    constexpr int CPB = 256 / G;                     // channels per block
+    extern __shared__ __align__(16) float sm[];
     const long long nquad = (long long)p.batch * p.dim * G;
     const long long chans = (long long)p.batch * p.dim;
     const int N = p.dstate;
@@ -150,6 +162,19 @@ __global__ void __launch_bounds__(256) state_steps_kernel(const StepArgs p) {
     const int b = int(ch / p.dim);
     const int d = int(ch - (long long)b * p.dim);
     const int n0 = 4 * r;
+    // the block's channels ch0 .. ch0+CPB-1 and the sequences b_lo .. they belong to
+    const long long ch0 = (long long)blockIdx.x * CPB;
+    const int b_lo = int(ch0 / p.dim);
+    // this thread's channel within the block and its sequence among the staged ones
+    // (0 for the idle threads past the last channel, which read but never use them)
+    const int cl = act ? int(ch - ch0) : 0;
+    const int bsel = act ? b - b_lo : 0;
+    float *sx = sm;                           // [round][CPB]
+    float *sd = sx + kStepsRound * CPB;
+    float *sz = sd + kStepsRound * CPB;
+    float *sb = sz + kStepsRound * CPB;       // [round][nb_max][N]
+    float *sc = sb + (size_t)kStepsRound * nb_max * N;
+
     float *hp = p.state + (size_t)ch * N + n0;
     const float *Ap = p.A + (size_t)d * N + n0;
     float h[4], a4[4];
@@ -172,44 +197,59 @@ __global__ void __launch_bounds__(256) state_steps_kernel(const StepArgs p) {
         }
     }
     const float Dv = p.D != nullptr ? p.D[d] : 0.f;
-    for (int t = 0; t < p.ntok; ++t) {
-        const size_t tc = (size_t)t * chans + ch;                  // [t][b][d]
-        const size_t tb = ((size_t)t * p.batch + b) * N + n0;      // [t][b][n]
-        const Tin *Bb = static_cast<const Tin *>(p.B) + tb;
-        const Tin *Cb = static_cast<const Tin *>(p.C) + tb;
-        float bb[4], cc[4];
-        if constexpr (VEC4) {
-            if (act && n0 < N) {
-                load4_nc<Tin>(Bb, bb);
-                load4_nc<Tin>(Cb, cc);
-            } else {
-#pragma unroll
-                for (int s = 0; s < 4; ++s) bb[s] = cc[s] = 0.f;
-            }
-        } else {
+    const Tin *gx = static_cast<const Tin *>(p.x);
+    const Tin *gd = static_cast<const Tin *>(p.delta);
+    const Tin *gz = static_cast<const Tin *>(p.z);
+    const Tin *gB = static_cast<const Tin *>(p.B);
+    const Tin *gC = static_cast<const Tin *>(p.C);
+    for (int t0 = 0; t0 < p.ntok; t0 += kStepsRound) {
+        const int nt = min(kStepsRound, p.ntok - t0);
+        __syncthreads();                      // the previous round's reads are done
+        for (int i = threadIdx.x; i < nt * CPB; i += blockDim.x) {
+            const int tt = i / CPB, c = i % CPB;
+            const long long cg = ch0 + c;
+            const bool ok = cg < chans;
+            const size_t idx = (size_t)(t0 + tt) * chans + (ok ? cg : 0);
+            sx[tt * CPB + c] = ok ? to_f32(gx[idx]) : 0.f;
+            sd[tt * CPB + c] = ok ? to_f32(gd[idx]) : 0.f;
+            sz[tt * CPB + c] = (ok && gz != nullptr) ? to_f32(gz[idx]) : 0.f;
+        }
+        for (int i = threadIdx.x; i < nt * nb_max * N; i += blockDim.x) {
+            const int tt = i / (nb_max * N), rem = i % (nb_max * N);
+            const int bb = b_lo + rem / N, n = rem % N;
+            const bool ok = bb < p.batch;
+            const size_t idx = ((size_t)(t0 + tt) * p.batch + (ok ? bb : 0)) * N + n;
+            sb[(size_t)tt * nb_max * N + rem] = ok ? to_f32(gB[idx]) : 0.f;
+            sc[(size_t)tt * nb_max * N + rem] = ok ? to_f32(gC[idx]) : 0.f;
+        }
+        __syncthreads();
+        for (int tt = 0; tt < nt; ++tt) {
+            const float dl = sd[tt * CPB + cl];
+            const float xv = sx[tt * CPB + cl];
+            const float zv = sz[tt * CPB + cl];
+            const float *bq = sb + ((size_t)tt * nb_max + bsel) * N + n0;
+            const float *cq = sc + ((size_t)tt * nb_max + bsel) * N + n0;
+            float bb[4], cc[4];
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 const bool ok = act && n0 + s < N;
-                bb[s] = ok ? to_f32(Bb[s]) : 0.f;
-                cc[s] = ok ? to_f32(Cb[s]) : 0.f;
+                bb[s] = ok ? bq[s] : 0.f;
+                cc[s] = ok ? cq[s] : 0.f;
             }
-        }
-        const float dl = to_f32(static_cast<const Tin *>(p.delta)[tc]);
-        const float xv = to_f32(static_cast<const Tin *>(p.x)[tc]);
-        const float zv = p.z != nullptr ? to_f32(static_cast<const Tin *>(p.z)[tc]) : 0.f;
-        const float dx = dl * xv;
-        float acc = 0.f;
+            const float dx = dl * xv;
+            float acc = 0.f;
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            h[s] = fmaf(ex2_approx(dl * a4[s] * kLog2e), h[s], dx * bb[s]);
-            acc = fmaf(cc[s], h[s], acc);
-        }
+            for (int s = 0; s < 4; ++s) {
+                h[s] = fmaf(ex2_approx(dl * a4[s] * kLog2e), h[s], dx * bb[s]);
+                acc = fmaf(cc[s], h[s], acc);
+            }
 #pragma unroll
-        for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (act && r == 0) {
-            float yv = fmaf(Dv, xv, acc);
-            if (p.z != nullptr) yv *= silu_f(zv);
-            static_cast<Tout *>(p.y)[tc] = from_f32<Tout>(yv);
+            for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (act && r == 0) {
+                float yv = fmaf(Dv, xv, acc);
+                if (p.z != nullptr) yv *= silu_f(zv);
+                static_cast<Tout *>(p.y)[(size_t)(t0 + tt) * chans + ch] = from_f32<Tout>(yv);
+            }
         }
     }
     if constexpr (VEC4) {

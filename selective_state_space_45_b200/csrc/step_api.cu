@@ -1,5 +1,6 @@
 // step_api.cu -- C ABI of the decode steps: one token (ssm_state_step) and several tokens
 // on the carried state (ssm_state_step_multi).
+#include <algorithm>
 #include <climits>
 
 #include "api_host.cuh"
@@ -42,10 +43,22 @@ int launch_steps_np(const ssm::StepArgs &a, cudaStream_t s) {
     const long long quads = (long long)a.batch * a.dim * G;
     const long long blocks = (quads + 255) / 256;
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    // sequences a block's 256 / G consecutive channels can span
+    constexpr int CPB = 256 / G;
+    const int nb_max = int(std::min<long long>(a.batch, (CPB - 1) / a.dim + 2));
+    const size_t smem = ssm::steps_smem_bytes(CPB, nb_max, a.dstate);   // at most ~91 KB
+    if (smem > 48 * 1024) {
+        const int bytes = int(smem);
+        if (cudaFuncSetAttribute(ssm::state_steps_kernel<NP, Tin, Tout, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+            cudaFuncSetAttribute(ssm::state_steps_kernel<NP, Tin, Tout, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return SSM_ERR_CUDA;
+    }
     if (a.dstate % 4 == 0)
-        ssm::state_steps_kernel<NP, Tin, Tout, true><<<unsigned(blocks), 256, 0, s>>>(a);
+        ssm::state_steps_kernel<NP, Tin, Tout, true><<<unsigned(blocks), 256, smem, s>>>(a, nb_max);
     else
-        ssm::state_steps_kernel<NP, Tin, Tout, false><<<unsigned(blocks), 256, 0, s>>>(a);
+        ssm::state_steps_kernel<NP, Tin, Tout, false><<<unsigned(blocks), 256, smem, s>>>(a, nb_max);
     return status_of(cudaGetLastError());
 }
 

@@ -141,3 +141,21 @@ def test_multi_token_step_with_no_tokens_keeps_state(cuda_lib):
                                   torch.empty(0, 2, 8, device=DEV))
     torch.cuda.synchronize()
     assert torch.equal(st, inp["state"])
+
+
+@pytest.mark.parametrize("batch,dim,N", [(40, 1, 16), (9, 3, 4), (5, 70, 8)])
+def test_multi_token_step_small_dims_span_many_sequences(cuda_lib, batch, dim, N):
+    # a block's channels then cover several sequences, whose B, C are all staged
+    ntok = 11
+    inp = inputs.make_decode_inputs(batch, dim, N, ntok, torch.float32, device=DEV, seed=batch + dim)
+    st = inp["state"].clone()
+    y = torch.empty(ntok, batch, dim, device=DEV)
+    cuda_lib.ssm_state_step_multi(st, inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                  inp["z"], y)
+    torch.cuda.synchronize()
+    h = to64(inp["state"])
+    for t in range(ntok):
+        yr, h = oracle.step(h, inp["x"][t], inp["delta"][t], inp["A"], inp["B"][t], inp["C"][t],
+                            D=inp["D"], z=inp["z"][t])
+        assert_parity(y[t], yr, torch.float32, torch.float32, what="y[%d]" % t)
+    assert_parity(st, h, torch.float32, torch.float32, what="state")
