@@ -121,7 +121,7 @@ def load_peaks():
 
 # translation unit of libssm.so that holds each kernel and its launch logic
 KERNEL_UNIT = {"scan_fwd_kernel": "scan_api.cu", "state_step_kernel": "step_api.cu",
-               "state_steps_kernel": "step_api.cu", "ssd_fwd_kernel": "ssd_api.cu",
+               "state_steps_kernel": "step_api.cu", "ssd_chunk_scan_kernel": "ssd_api.cu",
                "scan_bwd_kernel": "bwd_api.cu",
                "causal_conv1d_vec_kernel": "conv_api.cu", "conv1d_step_kernel": "conv_api.cu"}
 
@@ -392,7 +392,7 @@ class Workload:
 def kernel_name(kind):
     return dict(scan="scan_fwd_kernel", decode="state_step_kernel", conv="causal_conv1d_vec_kernel",
                 convstep="conv1d_step_kernel", bwd="scan_bwd_kernel",
-                decodemulti="state_steps_kernel", ssd="ssd_fwd_kernel")[kind]
+                decodemulti="state_steps_kernel", ssd="ssd_chunk_scan_kernel")[kind]
 
 
 # ------------------------------------------------------------------ CPU oracle timing

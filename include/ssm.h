@@ -272,7 +272,10 @@ int ssm_state_step_multi(float *state, const void *x, const void *delta, const f
  * in_dtype must be SSM_BF16 (the tensor-core operands); headdim 32 or 64 and dstate 64 or
  * 128 (SSM_ERR_UNSUPPORTED otherwise).  Products run on bf16 operands with fp32
  * accumulation; the masked scores, the decay-weighted inputs and the state are rounded to
- * bf16 where they enter a product.  seqlen = 0 copies the start state through.
+ * bf16 where they enter a product.  seqlen = 0 copies the start state through.  Takes a
+ * stream-ordered scratch buffer (cudaMallocAsync / cudaFreeAsync on cuda_stream) of
+ * 6 * headdim * dstate bytes per (sequence, head, 64-token chunk): every chunk's state
+ * contribution (fp32) and entering state (bf16).
  */
 int ssm_ssd_fwd(const void *x, const float *a, const void *B, const void *C, void *y,
                 const float *initial_state, float *final_state,

@@ -12,16 +12,40 @@ using namespace ssm_host;
 namespace {
 
 template <int P, int N, typename Tout>
-int launch_ssd(const ssm::SsdArgs &a, cudaStream_t s) {
+int launch_ssd(ssm::SsdArgs a, cudaStream_t s) {
     using Cfg = ssm::SsdCfg<P, N, Tout>;
-    const long long grid = (long long)a.batch * a.heads;
-    if (grid > INT_MAX) return SSM_ERR_UNSUPPORTED;
-    if (grid == 0) return SSM_OK;
-    if (cudaFuncSetAttribute(ssm::ssd_fwd_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(Cfg::SMEM_BYTES)) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    ssm::ssd_fwd_kernel<Cfg><<<unsigned(grid), Cfg::NT, Cfg::SMEM_BYTES, s>>>(a);
-    return status_of(cudaGetLastError());
+    const long long bh = (long long)a.batch * a.heads;
+    const long long nchunk = (a.seqlen + Cfg::Q - 1) / Cfg::Q;
+    const long long ctas = bh * nchunk;
+    const long long pass_blocks = (bh * N * P + 255) / 256;
+    if (ctas > INT_MAX || pass_blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    if (ctas == 0) return SSM_OK;
+    a.nchunk = int(nchunk);
+    // scratch: the chunks' state contributions (fp32), their total decays, the entering
+    // states (bf16)
+    const size_t ds_bytes = size_t(ctas) * N * P * sizeof(float);
+    const size_t tot_bytes = (size_t(ctas) * sizeof(float) + 255) & ~size_t(255);
+    const size_t e_bytes = size_t(ctas) * N * P * sizeof(__nv_bfloat16);
+    void *ws = nullptr;
+    if (cudaMallocAsync(&ws, ds_bytes + tot_bytes + e_bytes, s) != cudaSuccess) return SSM_ERR_CUDA;
+    a.dS = static_cast<float *>(ws);
+    a.tot = reinterpret_cast<float *>(static_cast<char *>(ws) + ds_bytes);
+    a.E = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + ds_bytes + tot_bytes);
+    int st = SSM_OK;
+    if (cudaFuncSetAttribute(ssm::ssd_chunk_scan_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(Cfg::SC_SMEM)) != cudaSuccess ||
+        cudaFuncSetAttribute(ssm::ssd_chunk_state_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(Cfg::ST_SMEM)) != cudaSuccess)
+        st = SSM_ERR_CUDA;
+    if (st == SSM_OK) {
+        ssm::ssd_chunk_state_kernel<Cfg><<<unsigned(ctas), Cfg::NT, Cfg::ST_SMEM, s>>>(a);
+        ssm::ssd_state_pass_kernel<Cfg><<<unsigned(pass_blocks), 256, 0, s>>>(a);
+        ssm::ssd_chunk_scan_kernel<Cfg><<<unsigned(ctas), Cfg::NT, Cfg::SC_SMEM, s>>>(a);
+        st = status_of(cudaGetLastError());
+    }
+    const cudaError_t fe = cudaFreeAsync(ws, s);
+    if (st == SSM_OK && fe != cudaSuccess) st = SSM_ERR_CUDA;
+    return st;
 }
 
 template <typename Tout>
