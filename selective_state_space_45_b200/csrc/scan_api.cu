@@ -52,8 +52,26 @@ int launch_scan_kernel(const ssm::ScanArgs &a, long long blocks, cudaStream_t st
     return status_of(cudaGetLastError());
 }
 
-// One scan: a single pass when the sequence fits one CTA per channel group, else the two
-// segment passes with a stream-ordered scratch buffer of batch*dim*nseg*(NP+1) floats.
+// The passes before the segment scans: each earlier segment's tail sum and step sum, then
+// the fold of those into the carry of every segment.
+template <class Cfg, bool ZOH>
+int launch_tail_fold(const ssm::ScanArgs &a, cudaStream_t stream) {
+    constexpr int NP = Cfg::NP;
+    const long long rows = (long long)a.batch * a.dim;
+    const long long tail_blocks = rows * (a.nseg - 1);
+    const long long fold_blocks = (rows * NP + 255) / 256;
+    if (tail_blocks > INT_MAX || fold_blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    ssm::scan_tail_kernel<NP, typename Cfg::Tin, ZOH>
+        <<<unsigned(tail_blocks), 32 * ssm::kTailWarps, 0, stream>>>(a);
+    int st = status_of(cudaGetLastError());
+    if (st != SSM_OK) return st;
+    ssm::scan_fold_kernel<NP><<<unsigned(fold_blocks), 256, 0, stream>>>(a);
+    return status_of(cudaGetLastError());
+}
+
+// One scan: a single pass when the sequence fits one CTA per channel group, else the tail
+// and fold passes and one scan per segment from its carry, with a stream-ordered scratch
+// buffer of batch*dim*nseg*(NP+1) floats.
 template <class Cfg, bool ZOH>
 int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     ssm::ScanArgs a = a0;
@@ -75,7 +93,6 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
     nseg = int((a.seqlen + seg_len - 1) / seg_len);
     if (nseg <= 1) {
-        a.pass = 0;
         a.nseg = 1;
         a.seg_len = a.seqlen;
         return launch_scan_kernel<Cfg, false, ZOH>(a, cgroups, stream);
@@ -88,12 +105,8 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     a.seg_len = int(seg_len);
     a.seg_h = static_cast<float *>(ws);
     a.seg_s = a.seg_h + rows * Cfg::NP;
-    a.pass = 1;
-    int st = launch_scan_kernel<Cfg, true, ZOH>(a, cgroups * nseg, stream);
-    if (st == SSM_OK) {
-        a.pass = 2;
-        st = launch_scan_kernel<Cfg, true, ZOH>(a, cgroups * (nseg - 1), stream);
-    }
+    int st = launch_tail_fold<Cfg, ZOH>(a, stream);
+    if (st == SSM_OK) st = launch_scan_kernel<Cfg, true, ZOH>(a, cgroups * nseg, stream);
     const cudaError_t fe = cudaFreeAsync(ws, stream);
     if (st == SSM_OK && fe != cudaSuccess) st = SSM_ERR_CUDA;
     return st;
@@ -155,8 +168,9 @@ int noalloc_scratch(float **out) {
 }
 
 // Same scan as run_scan, with the segment aggregates in the static array: nothing is
-// allocated.  Pass 1 writes every (channel, segment) row that pass 2 reads within the
-// same call, so the array needs no clearing between calls.
+// allocated.  The tail pass writes every (channel, segment) row that the fold reads, and
+// the fold every row that the segment scans read, within the same call, so the array
+// needs no clearing between calls.
 template <class Cfg>
 int run_scan_noalloc(const ssm::ScanArgs &a0, cudaStream_t stream) {
     ssm::ScanArgs a = a0;
@@ -178,7 +192,6 @@ int run_scan_noalloc(const ssm::ScanArgs &a0, cudaStream_t stream) {
     seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
     nseg = int((a.seqlen + seg_len - 1) / seg_len);
     if (nseg <= 1) {
-        a.pass = 0;
         a.nseg = 1;
         a.seg_len = a.seqlen;
         return launch_scan_kernel<Cfg, false>(a, cgroups, stream);
@@ -192,13 +205,8 @@ int run_scan_noalloc(const ssm::ScanArgs &a0, cudaStream_t stream) {
     a.seg_len = int(seg_len);
     a.seg_h = ws;
     a.seg_s = ws + rows * Cfg::NP;
-    a.pass = 1;
-    int st = launch_scan_kernel<Cfg, true>(a, cgroups * nseg, stream);
-    if (st == SSM_OK) {
-        a.pass = 2;
-        st = launch_scan_kernel<Cfg, true>(a, cgroups * (nseg - 1), stream);
-    }
-    return st;
+    const int st = launch_tail_fold<Cfg, false>(a, stream);
+    return st == SSM_OK ? launch_scan_kernel<Cfg, true>(a, cgroups * nseg, stream) : st;
 }
 
 template <int NP, typename Tin, typename Tout, bool VEC>

@@ -27,15 +27,18 @@
 //     when every row is 16-byte aligned, else by guarded scalar loads; y is staged in
 //     shared memory and stored as 16-byte rows.
 //
-// Long sequences with few channels are split into segments scanned by different CTAs
-// (the scan is linear in its carry):
-//   pass 1  every segment scans from a zero state, writes its y and leaves its end state
-//           h_end and its step sum S = sum Delta in a scratch buffer;
-//   pass 2  every later segment folds the earlier segments' (S, h_end) into its true
-//           carry h_in (h <- exp(A*S) h + h_end), re-scans from h_in and overwrites y,
-//           stopping at the first tile boundary where exp(A * S_t) * |h_in| is exactly 0
-//           in fp32 for every state of every channel of the CTA -- from there on the
-//           carry no longer changes any value and the pass-1 output stands.
+// Long sequences with few channels are split into segments scanned by different CTAs.
+// The scan is linear in its carry, so a segment's end state from a zero start is
+//     h_end[n] = sum_t exp(A_n R_t) * Delta_t B_t[n] x_t,   R_t = sum of the steps after t
+// and only the tokens whose decay exp(A_n R_t) is not yet 0 in fp32 enter it:
+//   tail    every segment but the last sums h_end over its last tokens, walking back from
+//           its end until every state's decay has flushed to 0, and records its step sum S
+//           (or +inf once the decay over the whole segment is certain to be 0)
+//           (scan_tail_kernel);
+//   fold    the end states are folded in order into each segment's true carry
+//           h <- exp(A*S) h + h_end, from the start state (scan_fold_kernel);
+//   scan    every segment is scanned once from its true carry, writing y, the last one
+//           also the final state (scan_fwd_kernel with SEG).
 #pragma once
 
 #include "common.cuh"
@@ -57,13 +60,11 @@ struct ScanArgs {
     int softplus;
     int zoh;              // host side: exact zero-order-hold gain requested
     int groups_per_seq;   // ceil(dim / CH)
-    // segmented scan (long sequences): pass 0 = whole sequence in one CTA,
-    // 1 = segments from a zero state, 2 = carry correction of segments 1..nseg-1
-    int pass;
+    // segmented scan (long sequences): nseg segments of seg_len tokens
     int nseg;
     int seg_len;          // tokens per segment, a multiple of the tile
-    float *seg_h;         // [batch*dim][nseg][NP] end states of pass 1
-    float *seg_s;         // [batch*dim][nseg] step sums of pass 1
+    float *seg_h;         // [batch*dim][nseg][NP] tail sums h_end, carries after the fold
+    float *seg_s;         // [batch*dim][nseg] step sums of the segments (+inf: decay is 0)
     const float *h0;      // [batch][dim][dstate] start state, or null for zero
 };
 
@@ -192,7 +193,8 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
 }
 
 
-// SEG: segment passes 1/2 (else pass 0, the whole sequence).  ZOH: exact zero-order-hold
+// SEG: one segment of the segmented scan, from the folded carry into it (else the whole
+// sequence from the start state).  ZOH: exact zero-order-hold
 // input gain (exp(Delta a) - 1) / a * B instead of the Euler gain Delta * B.
 template <class Cfg, bool SEG, bool ZOH>
 __global__ void __launch_bounds__(Cfg::NTHREADS, Cfg::MINB)
@@ -210,9 +212,8 @@ scan_fwd_kernel(const ScanArgs p) {
     // CTA -> (sequence, channel group[, segment])
     int bg = blockIdx.x, seg = 0;
     if constexpr (SEG) {
-        const int per = (p.pass == 1) ? p.nseg : p.nseg - 1;
-        seg = bg % per + (p.pass == 2 ? 1 : 0);
-        bg /= per;
+        seg = bg % p.nseg;
+        bg /= p.nseg;
     }
     const int b = bg / p.groups_per_seq;
     const int d0 = (bg - b * p.groups_per_seq) * CH;
@@ -265,37 +266,15 @@ scan_fwd_kernel(const ScanArgs p) {
     }
 
     float h[4] = {0.f, 0.f, 0.f, 0.f};
-    if (p.h0 != nullptr && dvalid && (!SEG || (p.pass == 1 && seg == 0))) {
-        // a given start state enters the first token range (pass 2 folds it in through
-        // segment 0's end state)
+    if (SEG) {                              // the folded carry into the segment
+        if (dvalid) {
+            const float4 hv = *reinterpret_cast<const float4 *>(p.seg_h + (chrow * p.nseg + seg) * NP + 4 * q);
+            h[0] = hv.x; h[1] = hv.y; h[2] = hv.z; h[3] = hv.w;
+        }
+    } else if (p.h0 != nullptr && dvalid) {
 #pragma unroll
         for (int s = 0; s < 4; ++s)
             if (4 * q + s < N) h[s] = p.h0[chrow * N + 4 * q + s];
-    }
-    float hin[4] = {0.f, 0.f, 0.f, 0.f};   // carry into the segment (pass 2)
-    float sdl = 0.f;                        // running sum of this lane's steps in the range
-    if constexpr (SEG) {
-        if (p.pass == 2 && dvalid) {
-            // fold the earlier segments: h <- exp(A * S_j) h + h_end_j
-            for (int j = 0; j < seg; ++j) {
-                const float sj = p.seg_s[chrow * p.nseg + j];
-                const float4 hv = *reinterpret_cast<const float4 *>(p.seg_h + (chrow * p.nseg + j) * NP + 4 * q);
-                const float hj[4] = {hv.x, hv.y, hv.z, hv.w};
-#pragma unroll
-                for (int s = 0; s < 4; ++s) hin[s] = fmaf(ex2_approx(A2[s] * sj), hin[s], hj[s]);
-            }
-            if (seg == p.nseg - 1 && p.final_state != nullptr) {   // state after the last token
-                const float sj = p.seg_s[chrow * p.nseg + seg];
-                const float4 hv = *reinterpret_cast<const float4 *>(p.seg_h + (chrow * p.nseg + seg) * NP + 4 * q);
-                const float hj[4] = {hv.x, hv.y, hv.z, hv.w};
-                float *fs = p.final_state + chrow * N;
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    if (4 * q + s < N) fs[4 * q + s] = fmaf(ex2_approx(A2[s] * sj), hin[s], hj[s]);
-            }
-#pragma unroll
-            for (int s = 0; s < 4; ++s) h[s] = hin[s];
-        }
     }
 
     // the state in the recurrence: pairs (0,1), (2,3) for the packed FP32 instructions
@@ -305,15 +284,7 @@ scan_fwd_kernel(const ScanArgs p) {
         const int st = tile % Cfg::NSTAGE;
         const int t0 = tbeg + tile * T;
         cp_async_wait<Cfg::NSTAGE - 2>();
-        if (SEG && p.pass == 2) {
-            // stop once the carry's influence exp(A * S_t) * h_in is 0 in fp32 everywhere
-            bool alive = false;
-#pragma unroll
-            for (int s = 0; s < 4; ++s) alive |= ex2_approx(A2[s] * sdl) * fabsf(hin[s]) != 0.f;
-            if (!__syncthreads_or(alive)) break;
-        } else {
-            __syncthreads();
-        }
+        __syncthreads();
         {
             const int nt = tile + Cfg::NSTAGE - 1;
             if (nt < ntiles) load_tile<Cfg>(p, smem, nt % Cfg::NSTAGE, tbeg + nt * T, row0, bc0, nch);
@@ -394,7 +365,6 @@ scan_fwd_kernel(const ScanArgs p) {
                 const float4 d23 = pp[(2 * g + 1) * CH];
                 const float dl[4] = {d01.x, d01.z, d23.x, d23.z};
                 const float dx[4] = {d01.y, d01.w, d23.y, d23.w};
-                if constexpr (SEG) sdl += (dl[0] + dl[1]) + (dl[2] + dl[3]);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const float4 bq = *reinterpret_cast<const float4 *>(Bf + (4 * g + u) * NP + 4 * q);
@@ -515,17 +485,221 @@ scan_fwd_kernel(const ScanArgs p) {
     cp_async_wait<0>();
     h[0] = hp[0].x; h[1] = hp[0].y; h[2] = hp[1].x; h[3] = hp[1].y;
 
-    if (SEG && p.pass == 1) {           // segment aggregates for pass 2
-        if (dvalid) {
-            *reinterpret_cast<float4 *>(p.seg_h + (chrow * p.nseg + seg) * NP + 4 * q) =
-                make_float4(h[0], h[1], h[2], h[3]);
-            if (q == 0) p.seg_s[chrow * p.nseg + seg] = sdl;
-        }
-    } else if (!SEG && p.final_state != nullptr && dvalid) {
+    if ((!SEG || seg == p.nseg - 1) && p.final_state != nullptr && dvalid) {
         float *fs = p.final_state + chrow * N;
 #pragma unroll
         for (int s = 0; s < 4; ++s)
             if (4 * q + s < N) fs[4 * q + s] = h[s];
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Tail and fold passes of the segmented scan.
+
+// scan_tail_kernel: one CTA per (sequence, channel, segment but the last), tokens in lanes.
+// The CTA walks back from the segment's end in windows of kTailWarps x kTailBlocks 32-token
+// blocks, warp w taking the w-th run of kTailBlocks blocks of the window; R_t (the steps
+// after t) comes from a shuffle suffix scan inside each block and a shared scan over the
+// warps.  exp(A_n R_t) is ex2 with subnormal results flushed to 0, so a state whose log2
+// decay A_n log2(e) R_t stays below -127 over a whole block adds exactly 0 there and is
+// skipped, and a block with no state left is not read.  With the softplus step every step
+// is positive and R only grows going back: the walk stops at the first window that starts
+// with every state spent, and the segment's step sum S is then recorded as +inf (its decay
+// is 0 for every state).  Without the softplus a step can be negative, so every block is
+// visited and tested on its own range of R.  Lane sums are reduced in a fixed order.
+constexpr int kTailWarps = 8;
+constexpr int kTailBlocks = 8;       // 32-token blocks per warp and window
+constexpr int kTailBatch = 4;        // blocks whose loads are issued together
+constexpr float kSpentLog2 = -127.f; // log2 decay below which ex2 flushes to 0
+
+template <int NP, typename Tin, bool ZOH>
+__global__ void __launch_bounds__(32 * kTailWarps)
+scan_tail_kernel(const ScanArgs p) {
+    __shared__ float wsum[2][kTailWarps];
+    __shared__ float hred[kTailWarps][NP];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per = p.nseg - 1;
+    const int seg = int(blockIdx.x % unsigned(per));
+    const long long row = blockIdx.x / unsigned(per);     // b * dim + d
+    const int d = int(row % p.dim);
+    const int b = int(row / p.dim);
+    const int L = p.seqlen, N = p.dstate;
+    const int tbeg = seg * p.seg_len;
+    const int tend = min(L, tbeg + p.seg_len);
+
+    float A2[NP], invA[NP];
+#pragma unroll
+    for (int n = 0; n < NP; ++n) {
+        A2[n] = n < N ? p.A[size_t(d) * N + n] * kLog2e : 0.f;
+        const float a = A2[n] * (1.f / kLog2e);
+        invA[n] = (ZOH && a != 0.f) ? 1.f / a : 0.f;
+    }
+    const float bias = p.delta_bias != nullptr ? p.delta_bias[d] : 0.f;
+    const size_t row0 = size_t(row) * L;
+    const Tin *gd = static_cast<const Tin *>(p.delta) + row0;
+    const Tin *gx = static_cast<const Tin *>(p.x) + row0;
+    const Tin *gb = static_cast<const Tin *>(p.B) + size_t(b) * L * N;
+
+    // states whose decay is not 0 for some step sum in [lo, hi] (padded states: none)
+    auto live = [&](float lo, float hi) {
+        unsigned m = 0;
+#pragma unroll
+        for (int n = 0; n < NP; ++n) {
+            const float e = A2[n] * (A2[n] < 0.f ? lo : hi);   // the largest log2 decay
+            if (n < N && !(e < kSpentLog2)) m |= 1u << n;
+        }
+        return m;
+    };
+
+    const bool grows = p.softplus != 0;
+    constexpr int WT = 32 * kTailBlocks;               // tokens per warp and window
+    constexpr int WIN = kTailWarps * WT;
+    float acc[NP];
+#pragma unroll
+    for (int n = 0; n < NP; ++n) acc[n] = 0.f;
+    float R = 0.f;                                     // steps after the window
+    bool spent = false;
+    int par = 0;
+    for (int w1 = tend; w1 > tbeg; w1 -= WIN, par ^= 1) {
+        if (grows && live(R, R) == 0u) { spent = true; break; }   // the same R in every thread
+        const int ts = w1 - WIN + warp * WT;           // this warp's first token (may be < tbeg)
+        float dl[kTailBlocks], suf[kTailBlocks];
+#pragma unroll
+        for (int j = 0; j < kTailBlocks; ++j) {
+            const int t = ts + 32 * j + lane;
+            float v = 0.f;
+            if (t >= tbeg && t < w1) {
+                v = to_f32(gd[t]) + bias;
+                if (p.softplus) v = softplus_f(v);
+            }
+            dl[j] = v;
+        }
+        // suf[j]: steps after this lane's token up to the end of the warp's run
+        float tot = 0.f;
+#pragma unroll
+        for (int j = kTailBlocks - 1; j >= 0; --j) {
+            float v = dl[j];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_down_sync(0xffffffffu, v, o);
+                if (lane + o < 32) v += u;
+            }
+            float ex = __shfl_down_sync(0xffffffffu, v, 1);
+            if (lane == 31) ex = 0.f;
+            suf[j] = tot + ex;
+            tot += __shfl_sync(0xffffffffu, v, 0);
+        }
+        if (lane == 0) wsum[par][warp] = tot;
+        __syncthreads();
+        float Rw = R;                                  // steps after this warp's run
+#pragma unroll
+        for (int k = kTailWarps - 1; k >= 0; --k) {
+            const float v = wsum[par][k];
+            if (k > warp) Rw += v;
+            R += v;
+        }
+
+#pragma unroll
+        for (int j0 = 0; j0 < kTailBlocks; j0 += kTailBatch) {
+            unsigned lm[kTailBatch];
+            float xv[kTailBatch], bv[kTailBatch][NP];
+#pragma unroll
+            for (int jj = 0; jj < kTailBatch; ++jj) {
+                const int j = j0 + jj;
+                const int t = ts + 32 * j + lane;
+                const float Rt = Rw + suf[j];
+                float lo = Rt, hi = Rt;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+                }
+                const bool any_tok = ts + 32 * j + 31 >= tbeg && ts + 32 * j < w1;
+                lm[jj] = any_tok ? live(lo, hi) : 0u;
+                const bool tok = lm[jj] != 0u && t >= tbeg && t < w1;
+                xv[jj] = tok ? to_f32(gx[t]) : 0.f;
+                if (tok && N == NP) {
+                    const Tin *br = gb + size_t(t) * NP;
+                    if constexpr (NP == 16) {
+                        float v0[8], v1[8];
+                        loadn<8, Tin>(br, v0);
+                        loadn<8, Tin>(br + 8, v1);
+#pragma unroll
+                        for (int n = 0; n < 8; ++n) { bv[jj][n] = v0[n]; bv[jj][8 + n] = v1[n]; }
+                    } else {
+                        float v0[NP];
+                        loadn<NP, Tin>(br, v0);
+#pragma unroll
+                        for (int n = 0; n < NP; ++n) bv[jj][n] = v0[n];
+                    }
+                } else {
+#pragma unroll
+                    for (int n = 0; n < NP; ++n)
+                        bv[jj][n] = (tok && n < N) ? to_f32(gb[size_t(t) * N + n]) : 0.f;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < kTailBatch; ++jj) {
+                if (lm[jj] == 0u) continue;            // uniform over the warp
+                const int j = j0 + jj;
+                const float Rt = Rw + suf[j];
+                const float dlt = dl[j];
+                const float dx = ZOH ? xv[jj] : dlt * xv[jj];
+#pragma unroll
+                for (int n = 0; n < NP; ++n) {
+                    if (!((lm[jj] >> n) & 1u)) continue;
+                    float w = dx * bv[jj][n];
+                    if constexpr (ZOH) {   // gain expm1(Delta a) / a, Delta where a = 0
+                        const float v = dlt * A2[n] * (1.f / kLog2e);
+                        const float em1 = fabsf(v) < 0.1f ? expm1_small(v) : ex2_approx(dlt * A2[n]) - 1.f;
+                        w *= invA[n] != 0.f ? em1 * invA[n] : dlt;
+                    }
+                    acc[n] = fmaf(ex2_approx(A2[n] * Rt), w, acc[n]);
+                }
+            }
+        }
+    }
+    // h_end: lanes (butterfly), then warps in order
+#pragma unroll
+    for (int n = 0; n < NP; ++n) {
+        float v = acc[n];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) hred[warp][n] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < NP) {
+        float h = 0.f;
+#pragma unroll
+        for (int k = 0; k < kTailWarps; ++k) h += hred[k][threadIdx.x];
+        p.seg_h[(size_t(row) * p.nseg + seg) * NP + threadIdx.x] = h;
+    }
+    if (threadIdx.x == 0) p.seg_s[size_t(row) * p.nseg + seg] = spent ? __int_as_float(0x7f800000) : R;
+}
+
+// scan_fold_kernel: one thread per (sequence, channel, padded state).  Walks the segments
+// in order from the start state, replacing each tail sum h_end_j by the carry into segment
+// j and stepping h <- exp(A S_j) h + h_end_j (S_j = +inf: decay 0).  The last segment's
+// slot only receives its carry.
+template <int NP>
+__global__ void scan_fold_kernel(const ScanArgs p) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long rows = (long long)p.batch * p.dim;
+    if (i >= rows * NP) return;
+    const long long row = i / NP;
+    const int n = int(i - row * NP);
+    const int d = int(row % p.dim);
+    const int N = p.dstate;
+    const float A2 = n < N ? p.A[size_t(d) * N + n] * kLog2e : 0.f;
+    float h = (p.h0 != nullptr && n < N) ? p.h0[size_t(row) * N + n] : 0.f;
+    for (int j = 0; j < p.nseg; ++j) {
+        float *hj = p.seg_h + (size_t(row) * p.nseg + j) * NP + n;
+        if (j == p.nseg - 1) { *hj = h; break; }
+        const float hend = *hj;
+        const float sj = p.seg_s[size_t(row) * p.nseg + j];
+        *hj = h;
+        const float decay = isinf(sj) ? 0.f : ex2_approx(A2 * sj);
+        h = fmaf(decay, h, hend);
     }
 }
 

@@ -17,8 +17,8 @@ DEV = "cuda"
 @pytest.fixture(params=[None, "3"], ids=["oneCTA", "segments3"])
 def split(request):
     """Both scan paths: one CTA per channel group over the whole sequence, and the
-    sequence cut into (up to) 3 segments -- pass 1 from a zero state, pass 2 carrying
-    the true state into every later segment."""
+    sequence cut into (up to) 3 segments -- pass 1 from a zero state, then the fold of the
+    end states and the carry's share of the output of every later segment."""
     old = os.environ.get("SSM_SCAN_SEGMENTS")
     if request.param is None:
         os.environ.pop("SSM_SCAN_SEGMENTS", None)
@@ -183,7 +183,7 @@ def test_misaligned_pointer_rejected_on_device(cuda_lib):
 @pytest.mark.parametrize("nseg", ["2", "5"])
 def test_segment_carry_never_dies(cuda_lib, nseg, monkeypatch):
     """A = 0 keeps exp(A * S) = 1: the carry reaches every token of every later segment,
-    so pass 2 must re-scan whole segments."""
+    so the carry pass must cover whole segments."""
     monkeypatch.setenv("SSM_SCAN_SEGMENTS", nseg)
     inp = inputs.make_scan_inputs(1, 40, 700, 16, torch.float32, device=DEV, seed=21)
     inp["A"][:, :3] = 0.0
@@ -195,8 +195,8 @@ def test_segment_carry_never_dies(cuda_lib, nseg, monkeypatch):
 
 
 def test_segment_carry_dies_at_once(cuda_lib, monkeypatch):
-    """Huge steps wipe the carry within one token: pass 2 stops after its first tile and
-    the pass-1 output stands."""
+    """Huge steps wipe the carry within one token: the carry pass stops in its first
+    window and the pass-1 output stands."""
     monkeypatch.setenv("SSM_SCAN_SEGMENTS", "4")
     inp = inputs.make_scan_inputs(2, 33, 512, 16, torch.bfloat16, device=DEV, seed=22)
     inp["delta_bias"].fill_(60.0)
@@ -204,6 +204,23 @@ def test_segment_carry_dies_at_once(cuda_lib, monkeypatch):
     yr, fr = run_oracle(inp)
     assert_parity(y, yr, torch.bfloat16, torch.bfloat16, what="y")
     assert_parity(fs, fr, torch.bfloat16, torch.float32, what="final_state")
+
+
+@pytest.mark.parametrize("nseg", ["3", "7"])
+def test_segment_carry_with_negative_steps(cuda_lib, nseg, monkeypatch):
+    """Without the softplus a raw step can be negative, so the step sum S_t of a segment
+    can fall again after rising: the carry's share exp(A S_t) h_in is checked against the
+    oracle on every block, not cut off at the first small value."""
+    monkeypatch.setenv("SSM_SCAN_SEGMENTS", nseg)
+    inp = inputs.make_scan_inputs(2, 24, 900, 16, torch.float32, device=DEV, seed=24)
+    g = torch.Generator(DEV).manual_seed(25)
+    inp["delta"] = (0.05 * torch.randn(inp["delta"].shape, device=DEV, generator=g) + 0.01).contiguous()
+    inp["A"].mul_(0.25)
+    y, fs = run_gpu(cuda_lib, inp, torch.float32, use_bias=False, softplus=False)
+    yr, fr = run_oracle(inp, use_bias=False, softplus=False)
+    assert (inp["delta"] < 0).float().mean().item() > 0.3
+    assert_parity(y, yr, torch.float32, what="y")
+    assert_parity(fs, fr, torch.float32, what="final_state")
 
 
 def test_long_sequence_default_segmentation(cuda_lib):
