@@ -78,9 +78,11 @@ typedef enum {
  * and seqlen below 2^31.
  * The N-wide state never leaves the chip: only y and final_state are written.
  * When batch * ceil(dim / 32) CTAs cannot fill the GPU, each sequence is cut into segments
- * scanned in parallel and stitched by their carries; their end states (batch * dim *
- * segments * (padded dstate + 1) floats, a few MiB at most) go to a stream-ordered
- * temporary buffer that is freed on the same stream before the call returns.
+ * scanned in parallel, each from its true carry.  Before the scans, each earlier segment's
+ * end state is summed from its last tokens, those whose decay is not yet 0 in fp32.  Those
+ * end states and step sums (batch * dim * segments * (padded dstate + 1) floats, a few MiB
+ * at most) go to a stream-ordered temporary buffer freed on the same stream before the
+ * call returns.
  */
 int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_bias,
                            int delta_softplus, const float *A, const void *B, const void *C,
@@ -118,8 +120,8 @@ int ssm_selective_scan_fwd_ex(const void *x, const void *delta, const float *del
  * critical loop that must not touch the allocator after start-up.
  *
  * Where ssm_selective_scan_fwd takes a stream-ordered temporary buffer (long sequences
- * with few channels are scanned in segments whose end states must be kept between two
- * passes), this call uses a fixed 4 MiB array in device memory instead.  That array
+ * with few channels are scanned in segments whose end states must be kept between
+ * launches), this call uses a fixed 4 MiB array in device memory instead.  That array
  * exists on every GPU that loads the library and stays there until the process exits.
  *  - The first call on a device looks up the array's device address (a one-time set-up
  *    per device, done with that device current); make that first call before any CUDA

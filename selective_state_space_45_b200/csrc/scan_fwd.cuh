@@ -496,25 +496,49 @@ scan_fwd_kernel(const ScanArgs p) {
 // ---------------------------------------------------------------------------------------
 // Tail and fold passes of the segmented scan.
 
-// scan_tail_kernel: one CTA per (sequence, channel, segment but the last), tokens in lanes.
-// The CTA walks back from the segment's end in windows of kTailWarps x kTailBlocks 32-token
-// blocks, warp w taking the w-th run of kTailBlocks blocks of the window; R_t (the steps
-// after t) comes from a shuffle suffix scan inside each block and a shared scan over the
-// warps.  exp(A_n R_t) is ex2 with subnormal results flushed to 0, so a state whose log2
-// decay A_n log2(e) R_t stays below -127 over a whole block adds exactly 0 there and is
-// skipped, and a block with no state left is not read.  With the softplus step every step
-// is positive and R only grows going back: the walk stops at the first window that starts
-// with every state spent, and the segment's step sum S is then recorded as +inf (its decay
-// is 0 for every state).  Without the softplus a step can be negative, so every block is
-// visited and tested on its own range of R.  Lane sums are reduced in a fixed order.
-constexpr int kTailWarps = 8;
-constexpr int kTailBlocks = 8;       // 32-token blocks per warp and window
-constexpr int kTailBatch = 4;        // blocks whose loads are issued together
-constexpr float kSpentLog2 = -127.f; // log2 decay below which ex2 flushes to 0
+// scan_tail_kernel: one CTA per (sequence, channel, segment but the last).  The CTA walks
+// back from the segment's end in windows of kTailWarps x 32 lanes x kTailTok tokens; lane l
+// of warp w takes kTailTok consecutive tokens of the w-th run of the window, so its steps
+// and inputs arrive in single vector loads.  R_t (the steps after t) comes from a serial
+// suffix sum over the lane's tokens, a shuffle suffix scan over the lanes and a shared scan
+// over the warps.  exp(A_n R_t) is ex2 with subnormal results flushed to 0, so a state whose
+// log2 decay A_n log2(e) R_t stays below -127 over a warp's run adds exactly 0 there and is
+// skipped (states go in pairs; a spent state computed beside a live one adds exactly 0).
+// With the softplus step every step is positive and R only grows going back: a state n
+// with A_n < 0 is spent for R > -127 / (A_n log2 e), tested once per run against the R
+// after the run, and the walk stops at the first window that starts with every state
+// spent; the segment's step sum S is then recorded as +inf (its decay is 0 for every
+// state).  Without the softplus a step can be negative, so each run is tested on its own
+// range of R and the walk covers the whole segment.  Lane sums are reduced in a fixed order.
+#ifndef SSM_TAIL_WARPS
+#define SSM_TAIL_WARPS 8      // warps per CTA
+#endif
+#ifndef SSM_TAIL_MINB
+#define SSM_TAIL_MINB 3       // resident CTAs per SM the registers target
+#endif
+constexpr int kTailWarps = SSM_TAIL_WARPS;
+constexpr int kTailTok = 4;           // consecutive tokens per lane and window
+constexpr float kSpentLog2 = -127.f;  // log2 decay below which ex2 flushes to 0
+
+// kTailTok consecutive values from src (vector load when `vec`: 4 values, 8- or 16-byte
+// aligned) as fp32; zeros when !ok.
+template <typename Tin>
+__device__ __forceinline__ void load_run4(const Tin *src, bool vec, bool ok, float (&v)[4]) {
+    if (!ok) {
+        v[0] = v[1] = v[2] = v[3] = 0.f;
+    } else if (vec) {
+        loadn<4, Tin>(src, v);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = to_f32(src[i]);
+    }
+}
 
 template <int NP, typename Tin, bool ZOH>
-__global__ void __launch_bounds__(32 * kTailWarps)
+__global__ void __launch_bounds__(32 * kTailWarps, SSM_TAIL_MINB)
 scan_tail_kernel(const ScanArgs p) {
+    constexpr int NQ = NP / 2;                          // state pairs
+    constexpr int EC = int(16 / sizeof(Tin));           // values per 16-byte chunk
     __shared__ float wsum[2][kTailWarps];
     __shared__ float hred[kTailWarps][NP];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -524,71 +548,95 @@ scan_tail_kernel(const ScanArgs p) {
     const int d = int(row % p.dim);
     const int b = int(row / p.dim);
     const int L = p.seqlen, N = p.dstate;
-    const int tbeg = seg * p.seg_len;
-    const int tend = min(L, tbeg + p.seg_len);
+    const int tbeg = seg * p.seg_len;                   // a multiple of 32, as is tend:
+    const int tend = tbeg + p.seg_len;                  // segments before the last are whole
+    const bool vec = (L % 4) == 0;                      // 4-token runs aligned in every row
 
-    float A2[NP], invA[NP];
+    float2 A2p[NQ];
+    float Rdead[NQ];      // (softplus) the pair is spent once R exceeds this
 #pragma unroll
-    for (int n = 0; n < NP; ++n) {
-        A2[n] = n < N ? p.A[size_t(d) * N + n] * kLog2e : 0.f;
-        const float a = A2[n] * (1.f / kLog2e);
-        invA[n] = (ZOH && a != 0.f) ? 1.f / a : 0.f;
+    for (int k = 0; k < NQ; ++k) {
+        float a[2], r = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int n = 2 * k + e;
+            a[e] = n < N ? p.A[size_t(d) * N + n] * kLog2e : 0.f;
+            if (n < N) r = fmaxf(r, a[e] < 0.f ? kSpentLog2 / a[e] : INFINITY);
+        }
+        A2p[k] = f2(a[0], a[1]);
+        Rdead[k] = r;
     }
+    // pairs not yet spent over a run whose R lies in [lo, hi] (any sign of the steps)
+    auto live_range = [&](float lo, float hi) {
+        unsigned m = 0;
+#pragma unroll
+        for (int k = 0; k < NQ; ++k) {
+            const float ex = A2p[k].x * (A2p[k].x < 0.f ? lo : hi);   // the largest log2 decay
+            const float ey = A2p[k].y * (A2p[k].y < 0.f ? lo : hi);
+            if ((2 * k < N && !(ex < kSpentLog2)) || (2 * k + 1 < N && !(ey < kSpentLog2)))
+                m |= 1u << k;
+        }
+        return m;
+    };
+    // (softplus) pairs not yet spent at step sum lo, R >= lo
+    auto live_from = [&](float lo) {
+        unsigned m = 0;
+#pragma unroll
+        for (int k = 0; k < NQ; ++k)
+            if (!(lo > Rdead[k])) m |= 1u << k;
+        return m;
+    };
+
     const float bias = p.delta_bias != nullptr ? p.delta_bias[d] : 0.f;
     const size_t row0 = size_t(row) * L;
     const Tin *gd = static_cast<const Tin *>(p.delta) + row0;
     const Tin *gx = static_cast<const Tin *>(p.x) + row0;
     const Tin *gb = static_cast<const Tin *>(p.B) + size_t(b) * L * N;
 
-    // states whose decay is not 0 for some step sum in [lo, hi] (padded states: none)
-    auto live = [&](float lo, float hi) {
-        unsigned m = 0;
-#pragma unroll
-        for (int n = 0; n < NP; ++n) {
-            const float e = A2[n] * (A2[n] < 0.f ? lo : hi);   // the largest log2 decay
-            if (n < N && !(e < kSpentLog2)) m |= 1u << n;
-        }
-        return m;
-    };
-
     const bool grows = p.softplus != 0;
-    constexpr int WT = 32 * kTailBlocks;               // tokens per warp and window
+    constexpr int WT = 32 * kTailTok;                  // tokens per warp and window
     constexpr int WIN = kTailWarps * WT;
-    float acc[NP];
+    float2 acc[NQ];
 #pragma unroll
-    for (int n = 0; n < NP; ++n) acc[n] = 0.f;
+    for (int k = 0; k < NQ; ++k) acc[k] = f2(0.f, 0.f);
     float R = 0.f;                                     // steps after the window
     bool spent = false;
     int par = 0;
+    // this lane's raw steps in the window ending at w1, loaded one window ahead
+    float draw[kTailTok];
+    auto load_steps = [&](int w1) {
+        const int t0 = w1 - WIN + warp * WT + kTailTok * lane;
+        load_run4<Tin>(gd + (t0 >= tbeg ? t0 : tbeg), vec, t0 >= tbeg, draw);
+    };
+    load_steps(tend);
     for (int w1 = tend; w1 > tbeg; w1 -= WIN, par ^= 1) {
-        if (grows && live(R, R) == 0u) { spent = true; break; }   // the same R in every thread
-        const int ts = w1 - WIN + warp * WT;           // this warp's first token (may be < tbeg)
-        float dl[kTailBlocks], suf[kTailBlocks];
+        if (grows && live_from(R) == 0u) { spent = true; break; }   // the same R in every thread
+        const int t0 = w1 - WIN + warp * WT + kTailTok * lane;   // this lane's first token
+        const bool ok = t0 >= tbeg;                    // all kTailTok tokens or none
+        float dl[kTailTok];
 #pragma unroll
-        for (int j = 0; j < kTailBlocks; ++j) {
-            const int t = ts + 32 * j + lane;
-            float v = 0.f;
-            if (t >= tbeg && t < w1) {
-                v = to_f32(gd[t]) + bias;
-                if (p.softplus) v = softplus_f(v);
-            }
-            dl[j] = v;
+        for (int i = 0; i < kTailTok; ++i) {
+            float v = draw[i] + bias;
+            if (p.softplus) v = softplus_f(v);
+            dl[i] = ok ? v : 0.f;
         }
-        // suf[j]: steps after this lane's token up to the end of the warp's run
-        float tot = 0.f;
+        if (w1 - WIN > tbeg) load_steps(w1 - WIN);
+        float xv[kTailTok];
+        load_run4<Tin>(gx + (ok ? t0 : tbeg), vec, ok, xv);
+        // steps after each of this lane's tokens, within the lane, then across the lanes
+        float sl[kTailTok];
+        sl[kTailTok - 1] = 0.f;
 #pragma unroll
-        for (int j = kTailBlocks - 1; j >= 0; --j) {
-            float v = dl[j];
+        for (int i = kTailTok - 2; i >= 0; --i) sl[i] = sl[i + 1] + dl[i + 1];
+        float incl = sl[0] + dl[0];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_down_sync(0xffffffffu, v, o);
-                if (lane + o < 32) v += u;
-            }
-            float ex = __shfl_down_sync(0xffffffffu, v, 1);
-            if (lane == 31) ex = 0.f;
-            suf[j] = tot + ex;
-            tot += __shfl_sync(0xffffffffu, v, 0);
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_down_sync(0xffffffffu, incl, o);
+            if (lane + o < 32) incl += u;
         }
+        float excl = __shfl_down_sync(0xffffffffu, incl, 1);
+        if (lane == 31) excl = 0.f;
+        const float tot = __shfl_sync(0xffffffffu, incl, 0);
         if (lane == 0) wsum[par][warp] = tot;
         __syncthreads();
         float Rw = R;                                  // steps after this warp's run
@@ -598,74 +646,79 @@ scan_tail_kernel(const ScanArgs p) {
             if (k > warp) Rw += v;
             R += v;
         }
+        const float Rl = Rw + excl;                    // steps after this lane's last token
+        unsigned m;
+        if (grows) {
+            m = live_from(Rw);
+        } else {
+            float lo = Rl, hi = Rl;
+#pragma unroll
+            for (int i = 0; i < kTailTok; ++i) { lo = fminf(lo, Rl + sl[i]); hi = fmaxf(hi, Rl + sl[i]); }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+            }
+            m = live_range(lo, hi);
+        }
+        if (m == 0u || w1 - WIN + warp * WT + WT <= tbeg) continue;   // uniform over the warp
 
+        // B rows of this lane's tokens, raw, then the live pairs
 #pragma unroll
-        for (int j0 = 0; j0 < kTailBlocks; j0 += kTailBatch) {
-            unsigned lm[kTailBatch];
-            float xv[kTailBatch], bv[kTailBatch][NP];
+        for (int i = 0; i < kTailTok; ++i) {
+            const int t = t0 + i;
+            float bf[NP];
+            if (ok && N == NP) {                       // dense rows: 16-byte (or 8-byte) loads
+                const Tin *br = gb + size_t(t) * NP;
+                if constexpr (NP >= EC) {
 #pragma unroll
-            for (int jj = 0; jj < kTailBatch; ++jj) {
-                const int j = j0 + jj;
-                const int t = ts + 32 * j + lane;
-                const float Rt = Rw + suf[j];
-                float lo = Rt, hi = Rt;
+                    for (int c = 0; c < NP; c += EC) {
+                        float v[EC];
+                        loadn<EC, Tin>(br + c, v);
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-                    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-                }
-                const bool any_tok = ts + 32 * j + 31 >= tbeg && ts + 32 * j < w1;
-                lm[jj] = any_tok ? live(lo, hi) : 0u;
-                const bool tok = lm[jj] != 0u && t >= tbeg && t < w1;
-                xv[jj] = tok ? to_f32(gx[t]) : 0.f;
-                if (tok && N == NP) {
-                    const Tin *br = gb + size_t(t) * NP;
-                    if constexpr (NP == 16) {
-                        float v0[8], v1[8];
-                        loadn<8, Tin>(br, v0);
-                        loadn<8, Tin>(br + 8, v1);
-#pragma unroll
-                        for (int n = 0; n < 8; ++n) { bv[jj][n] = v0[n]; bv[jj][8 + n] = v1[n]; }
-                    } else {
-                        float v0[NP];
-                        loadn<NP, Tin>(br, v0);
-#pragma unroll
-                        for (int n = 0; n < NP; ++n) bv[jj][n] = v0[n];
+                        for (int e = 0; e < EC; ++e) bf[c + e] = v[e];
                     }
                 } else {
-#pragma unroll
-                    for (int n = 0; n < NP; ++n)
-                        bv[jj][n] = (tok && n < N) ? to_f32(gb[size_t(t) * N + n]) : 0.f;
+                    loadn<NP, Tin>(br, bf);
                 }
+            } else {
+#pragma unroll
+                for (int n = 0; n < NP; ++n) bf[n] = (ok && n < N) ? to_f32(gb[size_t(t) * N + n]) : 0.f;
             }
+            const float Rt = Rl + sl[i];
+            const float2 Rt2 = f2(Rt, Rt);
+            const float dx = ZOH ? xv[i] : dl[i] * xv[i];
+            const float2 dx2 = f2(dx, dx);
 #pragma unroll
-            for (int jj = 0; jj < kTailBatch; ++jj) {
-                if (lm[jj] == 0u) continue;            // uniform over the warp
-                const int j = j0 + jj;
-                const float Rt = Rw + suf[j];
-                const float dlt = dl[j];
-                const float dx = ZOH ? xv[jj] : dlt * xv[jj];
+            for (int k = 0; k < NQ; ++k) {
+                if (!((m >> k) & 1u)) continue;
+                float2 w = fmul2(dx2, f2(bf[2 * k], bf[2 * k + 1]));
+                if constexpr (ZOH) {   // gain expm1(Delta a) / a, Delta where a = 0
+                    float g[2];
 #pragma unroll
-                for (int n = 0; n < NP; ++n) {
-                    if (!((lm[jj] >> n) & 1u)) continue;
-                    float w = dx * bv[jj][n];
-                    if constexpr (ZOH) {   // gain expm1(Delta a) / a, Delta where a = 0
-                        const float v = dlt * A2[n] * (1.f / kLog2e);
-                        const float em1 = fabsf(v) < 0.1f ? expm1_small(v) : ex2_approx(dlt * A2[n]) - 1.f;
-                        w *= invA[n] != 0.f ? em1 * invA[n] : dlt;
+                    for (int e = 0; e < 2; ++e) {
+                        const float a2 = e ? A2p[k].y : A2p[k].x;
+                        const float a = a2 * (1.f / kLog2e);
+                        const float v = dl[i] * a;
+                        const float em1 = fabsf(v) < 0.1f ? expm1_small(v) : ex2_approx(dl[i] * a2) - 1.f;
+                        g[e] = a != 0.f ? em1 / a : dl[i];
                     }
-                    acc[n] = fmaf(ex2_approx(A2[n] * Rt), w, acc[n]);
+                    w = fmul2(w, f2(g[0], g[1]));
                 }
+                acc[k] = ffma2(ex2_pair(fmul2(A2p[k], Rt2)), w, acc[k]);
             }
         }
     }
     // h_end: lanes (butterfly), then warps in order
 #pragma unroll
-    for (int n = 0; n < NP; ++n) {
-        float v = acc[n];
+    for (int k = 0; k < NQ; ++k) {
+        float vx = acc[k].x, vy = acc[k].y;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) hred[warp][n] = v;
+        for (int o = 16; o > 0; o >>= 1) {
+            vx += __shfl_xor_sync(0xffffffffu, vx, o);
+            vy += __shfl_xor_sync(0xffffffffu, vy, o);
+        }
+        if (lane == 0) { hred[warp][2 * k] = vx; hred[warp][2 * k + 1] = vy; }
     }
     __syncthreads();
     if (threadIdx.x < NP) {
