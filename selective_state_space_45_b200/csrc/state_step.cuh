@@ -131,133 +131,128 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
     }
 }
 
-// Several decode tokens per call (speculative or chunked decoding): the state of a
-// channel-quad is loaded once, carried through the ntok tokens in registers and stored
-// once, so the state traffic is that of one step whatever ntok is.  The token inputs of a
-// round of up to kStepsRound tokens are first staged in shared memory by the whole block,
-// every load independent of the others, so no thread waits on one token's loads before
-// issuing the next token's.  Per token the arithmetic is the one-step kernel's, in the
-// same order: ntok chained one-token calls give bit-identical results.
-constexpr int kStepsRound = 8;
+// Several decode tokens per call (ssm_state_step_multi: speculative or chunked decoding),
+// one channel per thread with all of its states in registers: the state (and A) is read
+// once, carried through the ntok tokens in registers and written once, so the state
+// traffic is that of one step whatever ntok is.  A block holds kStepThreads consecutive
+// channels of one sequence (blockIdx.x = b * dblocks + channel block).  Per round of up to
+// kStepsRound tokens every thread issues the loads of its (x, Delta, z) for all the
+// round's tokens at once, and the block stages the sequence's B and C rows of the round in
+// shared memory (padded to NP with zeros), read back as 16-byte broadcasts.
+//
+// Per token the arithmetic is the one-token kernel's, in the same order: each quad of 4
+// states is updated and read out as one thread of state_step_kernel does, and the quad
+// shares are summed in the order the xor-butterfly over the G lanes of a channel gives
+// lane 0.  ntok chained one-token calls therefore give bit-identical states and outputs.
+constexpr int kStepThreads = 256;
+constexpr int kStepsRound = 4;
 
-// Shared memory of one block of state_steps_kernel: per round token, x, delta, z of the
-// block's channels and B, C of the sequences they belong to (nb of them).
-__host__ __device__ constexpr size_t steps_smem_bytes(int ch_per_block, int nb, int N) {
-    return size_t(kStepsRound) * (3 * size_t(ch_per_block) + 2 * size_t(nb) * N) * sizeof(float);
+// The readout of a channel from its G = NP / 4 quad shares, in the xor-butterfly order
+// (offsets G/2, ..., 1) as seen by lane 0.
+template <int G> __device__ __forceinline__ float quad_sum(const float (&s)[G]) {
+    if constexpr (G == 1) return s[0];
+    else if constexpr (G == 2) return s[0] + s[1];
+    else return (s[0] + s[2]) + (s[1] + s[3]);
 }
 
 template <int NP, typename Tin, typename Tout, bool VEC4>
-__global__ void __launch_bounds__(256) state_steps_kernel(const StepArgs p, int nb_max) {
+__global__ void __launch_bounds__(kStepThreads, 3) state_steps_kernel(const StepArgs p, int dblocks) {
     constexpr int G = NP / 4;
-    constexpr int CPB = 256 / G;                     // channels per block
-    extern __shared__ __align__(16) float sm[];
-    const long long nquad = (long long)p.batch * p.dim * G;
-    const long long chans = (long long)p.batch * p.dim;
+    static_assert(2 * kStepsRound * NP <= kStepThreads, "one thread per staged B/C value");
+    __shared__ __align__(16) float sbc[2][kStepsRound][NP];
+    const int b = int(blockIdx.x / unsigned(dblocks));
+    const int d = (int(blockIdx.x) - b * dblocks) * kStepThreads + int(threadIdx.x);
+    const bool act = d < p.dim;
     const int N = p.dstate;
-    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const bool act = g < nquad;
-    const long long q = act ? g : 0;          // inactive lanes still join the shuffles
-    const long long ch = q / G;
-    const int r = int(q - ch * G);
-    const int b = int(ch / p.dim);
-    const int d = int(ch - (long long)b * p.dim);
-    const int n0 = 4 * r;
-    // the block's channels ch0 .. ch0+CPB-1 and the sequences b_lo .. they belong to
-    const long long ch0 = (long long)blockIdx.x * CPB;
-    const int b_lo = int(ch0 / p.dim);
-    // this thread's channel within the block and its sequence among the staged ones
-    // (0 for the idle threads past the last channel, which read but never use them)
-    const int cl = act ? int(ch - ch0) : 0;
-    const int bsel = act ? b - b_lo : 0;
-    float *sx = sm;                           // [round][CPB]
-    float *sd = sx + kStepsRound * CPB;
-    float *sz = sd + kStepsRound * CPB;
-    float *sb = sz + kStepsRound * CPB;       // [round][nb_max][N]
-    float *sc = sb + (size_t)kStepsRound * nb_max * N;
+    const size_t chans = size_t(p.batch) * p.dim;
+    const size_t ch = size_t(b) * p.dim + (act ? d : 0);
 
-    float *hp = p.state + (size_t)ch * N + n0;
-    const float *Ap = p.A + (size_t)d * N + n0;
-    float h[4], a4[4];
-    if constexpr (VEC4) {
-        if (act && n0 < N) {
-            const float4 hv = *reinterpret_cast<const float4 *>(hp);
-            const float4 av = __ldg(reinterpret_cast<const float4 *>(Ap));
-            h[0] = hv.x; h[1] = hv.y; h[2] = hv.z; h[3] = hv.w;
-            a4[0] = av.x; a4[1] = av.y; a4[2] = av.z; a4[3] = av.w;
-        } else {
+    float *hs = p.state + ch * N;
+    const float *As = p.A + size_t(act ? d : 0) * N;
+    float h[NP], a[NP];
+    if constexpr (VEC4) {                            // rows of whole 16-byte quads
 #pragma unroll
-            for (int s = 0; s < 4; ++s) h[s] = a4[s] = 0.f;
+        for (int q = 0; q < G; ++q) {
+            float4 hv = make_float4(0.f, 0.f, 0.f, 0.f), av = hv;
+            if (act && 4 * q < N) {
+                hv = *reinterpret_cast<const float4 *>(hs + 4 * q);
+                av = __ldg(reinterpret_cast<const float4 *>(As + 4 * q));
+            }
+            h[4 * q] = hv.x; h[4 * q + 1] = hv.y; h[4 * q + 2] = hv.z; h[4 * q + 3] = hv.w;
+            a[4 * q] = av.x; a[4 * q + 1] = av.y; a[4 * q + 2] = av.z; a[4 * q + 3] = av.w;
         }
     } else {
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const bool ok = act && n0 + s < N;
-            h[s] = ok ? hp[s] : 0.f;
-            a4[s] = ok ? Ap[s] : 0.f;
+        for (int n = 0; n < NP; ++n) {
+            const bool ok = act && n < N;
+            h[n] = ok ? hs[n] : 0.f;
+            a[n] = ok ? As[n] : 0.f;
         }
     }
-    const float Dv = p.D != nullptr ? p.D[d] : 0.f;
+    const float Dv = (p.D != nullptr && act) ? p.D[d] : 0.f;
     const Tin *gx = static_cast<const Tin *>(p.x);
     const Tin *gd = static_cast<const Tin *>(p.delta);
     const Tin *gz = static_cast<const Tin *>(p.z);
     const Tin *gB = static_cast<const Tin *>(p.B);
     const Tin *gC = static_cast<const Tin *>(p.C);
+    Tout *gy = static_cast<Tout *>(p.y);
     for (int t0 = 0; t0 < p.ntok; t0 += kStepsRound) {
         const int nt = min(kStepsRound, p.ntok - t0);
-        __syncthreads();                      // the previous round's reads are done
-        for (int i = threadIdx.x; i < nt * CPB; i += blockDim.x) {
-            const int tt = i / CPB, c = i % CPB;
-            const long long cg = ch0 + c;
-            const bool ok = cg < chans;
-            const size_t idx = (size_t)(t0 + tt) * chans + (ok ? cg : 0);
-            sx[tt * CPB + c] = ok ? to_f32(gx[idx]) : 0.f;
-            sd[tt * CPB + c] = ok ? to_f32(gd[idx]) : 0.f;
-            sz[tt * CPB + c] = (ok && gz != nullptr) ? to_f32(gz[idx]) : 0.f;
+        float xr[kStepsRound], dr[kStepsRound], zr[kStepsRound];
+#pragma unroll
+        for (int tt = 0; tt < kStepsRound; ++tt) {
+            const bool ok = act && tt < nt;
+            const size_t idx = size_t(t0 + tt) * chans + ch;
+            xr[tt] = ok ? to_f32(gx[idx]) : 0.f;
+            dr[tt] = ok ? to_f32(gd[idx]) : 0.f;
+            zr[tt] = (ok && gz != nullptr) ? to_f32(gz[idx]) : 0.f;
         }
-        for (int i = threadIdx.x; i < nt * nb_max * N; i += blockDim.x) {
-            const int tt = i / (nb_max * N), rem = i % (nb_max * N);
-            const int bb = b_lo + rem / N, n = rem % N;
-            const bool ok = bb < p.batch;
-            const size_t idx = ((size_t)(t0 + tt) * p.batch + (ok ? bb : 0)) * N + n;
-            sb[(size_t)tt * nb_max * N + rem] = ok ? to_f32(gB[idx]) : 0.f;
-            sc[(size_t)tt * nb_max * N + rem] = ok ? to_f32(gC[idx]) : 0.f;
+        __syncthreads();                      // the previous round's reads are done
+        {
+            const int i = threadIdx.x;
+            const int which = i / (kStepsRound * NP);
+            const int tt = (i / NP) % kStepsRound, n = i % NP;
+            if (i < 2 * kStepsRound * NP && tt < nt) {
+                const size_t idx = (size_t(t0 + tt) * p.batch + b) * N + n;
+                sbc[which][tt][n] = n < N ? to_f32((which ? gC : gB)[idx]) : 0.f;
+            }
         }
         __syncthreads();
-        for (int tt = 0; tt < nt; ++tt) {
-            const float dl = sd[tt * CPB + cl];
-            const float xv = sx[tt * CPB + cl];
-            const float zv = sz[tt * CPB + cl];
-            const float *bq = sb + ((size_t)tt * nb_max + bsel) * N + n0;
-            const float *cq = sc + ((size_t)tt * nb_max + bsel) * N + n0;
-            float bb[4], cc[4];
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const bool ok = act && n0 + s < N;
-                bb[s] = ok ? bq[s] : 0.f;
-                cc[s] = ok ? cq[s] : 0.f;
-            }
+        for (int tt = 0; tt < kStepsRound; ++tt) {
+            if (tt >= nt) break;
+            const float dl = dr[tt], xv = xr[tt];
             const float dx = dl * xv;
-            float acc = 0.f;
+            float sq[G];
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                h[s] = fmaf(ex2_approx(dl * a4[s] * kLog2e), h[s], dx * bb[s]);
-                acc = fmaf(cc[s], h[s], acc);
-            }
+            for (int q = 0; q < G; ++q) {
+                const float4 bq = *reinterpret_cast<const float4 *>(&sbc[0][tt][4 * q]);
+                const float4 cq = *reinterpret_cast<const float4 *>(&sbc[1][tt][4 * q]);
+                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+                const float cc[4] = {cq.x, cq.y, cq.z, cq.w};
+                float acc = 0.f;
 #pragma unroll
-            for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (act && r == 0) {
-                float yv = fmaf(Dv, xv, acc);
-                if (p.z != nullptr) yv *= silu_f(zv);
-                static_cast<Tout *>(p.y)[(size_t)(t0 + tt) * chans + ch] = from_f32<Tout>(yv);
+                for (int s = 0; s < 4; ++s) {
+                    const int n = 4 * q + s;
+                    h[n] = fmaf(ex2_approx(dl * a[n] * kLog2e), h[n], dx * bb[s]);
+                    acc = fmaf(cc[s], h[n], acc);
+                }
+                sq[q] = acc;
             }
+            float yv = fmaf(Dv, xv, quad_sum<G>(sq));
+            if (gz != nullptr) yv *= silu_f(zr[tt]);
+            if (act) gy[size_t(t0 + tt) * chans + ch] = from_f32<Tout>(yv);
         }
     }
     if constexpr (VEC4) {
-        if (act && n0 < N) *reinterpret_cast<float4 *>(hp) = make_float4(h[0], h[1], h[2], h[3]);
+#pragma unroll
+        for (int q = 0; q < G; ++q)
+            if (act && 4 * q < N)
+                *reinterpret_cast<float4 *>(hs + 4 * q) = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
     } else {
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            if (act && n0 + s < N) hp[s] = h[s];
+        for (int n = 0; n < NP; ++n)
+            if (act && n < N) hs[n] = h[n];
     }
 }
 

@@ -37,28 +37,18 @@ int launch_step(const ssm::StepArgs &a, cudaStream_t s) {
     return launch_step_np<16, Tin, Tout>(a, s);
 }
 
+// Several tokens: one channel per thread, kStepThreads consecutive channels of one
+// sequence per block.
 template <int NP, typename Tin, typename Tout>
 int launch_steps_np(const ssm::StepArgs &a, cudaStream_t s) {
-    constexpr int G = NP / 4;
-    const long long quads = (long long)a.batch * a.dim * G;
-    const long long blocks = (quads + 255) / 256;
+    const long long dblocks = (a.dim + ssm::kStepThreads - 1) / ssm::kStepThreads;
+    const long long blocks = dblocks * a.batch;
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
-    // sequences a block's 256 / G consecutive channels can span
-    constexpr int CPB = 256 / G;
-    const int nb_max = int(std::min<long long>(a.batch, (CPB - 1) / a.dim + 2));
-    const size_t smem = ssm::steps_smem_bytes(CPB, nb_max, a.dstate);   // at most ~91 KB
-    if (smem > 48 * 1024) {
-        const int bytes = int(smem);
-        if (cudaFuncSetAttribute(ssm::state_steps_kernel<NP, Tin, Tout, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
-            cudaFuncSetAttribute(ssm::state_steps_kernel<NP, Tin, Tout, false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
-            return SSM_ERR_CUDA;
-    }
+    if (blocks == 0) return SSM_OK;
     if (a.dstate % 4 == 0)
-        ssm::state_steps_kernel<NP, Tin, Tout, true><<<unsigned(blocks), 256, smem, s>>>(a, nb_max);
+        ssm::state_steps_kernel<NP, Tin, Tout, true><<<unsigned(blocks), ssm::kStepThreads, 0, s>>>(a, int(dblocks));
     else
-        ssm::state_steps_kernel<NP, Tin, Tout, false><<<unsigned(blocks), 256, smem, s>>>(a, nb_max);
+        ssm::state_steps_kernel<NP, Tin, Tout, false><<<unsigned(blocks), ssm::kStepThreads, 0, s>>>(a, int(dblocks));
     return status_of(cudaGetLastError());
 }
 
