@@ -280,6 +280,52 @@ def test_decode_step_hand_example():
     assert abs(y[0, 0] - (0.5 * h + 8.0)) < 1e-14
 
 
+def _steps(case):
+    return np.log1p(np.exp(case["delta"] + case["delta_bias"][None, :, None]))
+
+
+def test_end_state_from_zero_is_the_decayed_sum_of_writes():
+    # Unrolling h_t = exp(Delta_t A) h_{t-1} + Delta_t B_t x_t ("Module 19", "The Math: The
+    # State-Space Recurrence") from h_0 = 0 gives h_L = sum_t exp(A R_t) Delta_t B_t x_t,
+    # R_t the sum of the steps after t: evaluated here directly, token by token.
+    rng = np.random.default_rng(21)
+    batch, dim, L, N = 2, 3, 40, 5
+    case = _random_case(rng, batch, dim, L, N)
+    steps = _steps(case)
+    _, hN = oracle.scan(x=case["x"], delta=steps, A=case["A"], B=case["B"], C=case["C"])
+    R = np.cumsum(steps[..., ::-1], axis=-1)[..., ::-1] - steps           # steps after t
+    w = steps[..., None] * case["x"][..., None] * case["B"][:, None, :, :]  # [b, d, t, n]
+    h = (np.exp(case["A"][None, :, None, :] * R[..., None]) * w).sum(axis=2)
+    np.testing.assert_allclose(hN, h, rtol=1e-12, atol=1e-14)
+
+
+def test_segments_scanned_from_folded_carries_give_the_whole_scan():
+    # The affine steps compose ("Module 19", "The Parallel Scan"): a segment maps its carry
+    # h to exp(A S) h + h_end, with S its step sum and h_end its end state from zero.
+    # Folding the segments in order from the start state gives the carry into each one,
+    # and scanning every segment from its carry gives the whole sequence's outputs.
+    rng = np.random.default_rng(22)
+    batch, dim, L, N = 2, 3, 50, 4
+    case = _random_case(rng, batch, dim, L, N)
+    steps = _steps(case)
+    h0 = rng.normal(size=(batch, dim, N))
+    kw = dict(A=case["A"], D=case["D"])
+    y_all, h_all = oracle.scan(x=case["x"], delta=steps, B=case["B"], C=case["C"],
+                               z=case["z"], h0=h0, **kw)
+    h, ys = h0, []
+    for a, b in [(0, 13), (13, 29), (29, 50)]:
+        seg = dict(x=case["x"][..., a:b], delta=steps[..., a:b], B=case["B"][:, a:b],
+                   C=case["C"][:, a:b])
+        _, h_end = oracle.scan(**seg, A=case["A"])                        # from zero
+        y_seg, h_seg = oracle.scan(**seg, z=case["z"][..., a:b], h0=h, **kw)
+        S = steps[..., a:b].sum(axis=-1)
+        h = np.exp(case["A"][None] * S[..., None]) * h + h_end
+        np.testing.assert_allclose(h, h_seg, rtol=1e-12, atol=1e-13)
+        ys.append(y_seg)
+    np.testing.assert_allclose(np.concatenate(ys, axis=-1), y_all, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(h, h_all, rtol=1e-12, atol=1e-13)
+
+
 def test_empty_sequence_keeps_initial_state():
     y, hN = oracle.scan(x=np.zeros((2, 3, 0)), delta=np.zeros((2, 3, 0)), A=-np.ones((3, 4)),
                         B=np.zeros((2, 0, 4)), C=np.zeros((2, 0, 4)))
