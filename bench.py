@@ -8,11 +8,11 @@ for bwd130m one ``ssm_selective_scan_bwd`` call (all gradients of the scan);
 the conv workloads time the causal convolution in front of the scan
 (``ssm_causal_conv1d_fwd`` with its final window, or one ``ssm_causal_conv1d_step``).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mamba130m]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mamba2p8b]
   python bench.py --impl reference ...        # the fp64 CPU oracle, timed on host cores
 
-Workloads (selective_state_space_45_b200.inputs.CONFIGS): mamba130m (default: batch 8,
-L 2048, d_inner 1536, N 16, bf16 in/out, fp32 state), mamba2p8b, long1m, decode, the
+Workloads (selective_state_space_45_b200.inputs.CONFIGS): mamba2p8b (default: batch 4,
+L 4096, d_inner 5120, N 16, bf16 in/out, fp32 state), mamba130m, long1m, decode, the
 backward's bwd130m, and the convolution's conv130m, conv2p8b, convstep.
 Multi-GPU: every rank runs its own replica (channels are independent; the path has no
 exchange step), timing is the max over ranks, value counts all ranks' work.
@@ -51,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mamba130m",
+    ap.add_argument("--workload", default="mamba2p8b",
                     choices=["mamba130m", "mamba2p8b", "long1m", "decode", "tiny",
                              "conv130m", "conv2p8b", "convstep", "bwd130m", "decode4", "ssd130m"])
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -361,32 +361,39 @@ class Workload:
                                        stream)
 
     def description(self):
-        c = self.cfg
-        io = str(c["dtype"]).split(".")[-1]
-        if self.kind == "conv":
-            return ("%s-shaped causal depthwise conv1d + SiLU: batch %d, L %d, d_inner %d, width %d, "
-                    "%s x and u, fp32 taps/bias/final window" % (self.name[4:], c["batch"], c["seqlen"],
-                                                                 c["dim"], c["width"], io))
-        if self.kind == "convstep":
-            return ("decode conv1d step: batch %d, d_inner %d, width %d, fp32 window in place, one %s "
-                    "token per sequence" % (c["batch"], c["dim"], c["width"], io))
-        if self.kind == "ssd":
-            return ("%s-shaped Mamba-2 SSD by 64-token chunks: batch %d, L %d, %d heads x %d, state %d, "
-                    "%s x/B/C and y, fp32 a" % (self.name[3:], c["batch"], c["seqlen"], c["heads"],
-                                               c["headdim"], c["dstate"], io))
-        if self.kind == "decodemulti":
-            return ("decode, %d tokens per call on the carried state: batch %d, d_inner %d, N %d, "
-                    "fp32 state in place, %s tokens" % (c["ntok"], c["batch"], c["dim"], c["dstate"], io))
-        if self.kind == "bwd":
-            return ("%s-shaped selective scan backward (states recomputed): batch %d, L %d, d_inner %d, "
-                    "N %d, %s inputs, dy and gradients, fp32 A/D/bias gradients"
-                    % (self.name[3:], c["batch"], c["seqlen"], c["dim"], c["dstate"], io))
-        if self.kind == "scan":
-            return ("%s-shaped selective scan: batch %d, L %d, d_inner %d, N %d, %s x/delta/z/B/C "
-                    "and y, fp32 A/D/bias/state" % (self.name, c["batch"], c["seqlen"], c["dim"],
-                                                     c["dstate"], str(c["dtype"]).split(".")[-1]))
-        return ("decode state step: batch %d, d_inner %d, N %d, fp32 state in place, one %s token "
-                "per sequence" % (c["batch"], c["dim"], c["dstate"], str(c["dtype"]).split(".")[-1]))
+        return describe_workload(self.name)
+
+
+def describe_workload(name):
+    """The workload's name and shape, as both arms print it in ``config.workload``."""
+    from selective_state_space_45_b200 import inputs
+    c = inputs.CONFIGS[name]
+    kind = workload_kind(name)
+    io = str(c["dtype"]).split(".")[-1]
+    if kind == "conv":
+        return ("%s-shaped causal depthwise conv1d + SiLU: batch %d, L %d, d_inner %d, width %d, "
+                "%s x and u, fp32 taps/bias/final window" % (name[4:], c["batch"], c["seqlen"],
+                                                             c["dim"], c["width"], io))
+    if kind == "convstep":
+        return ("decode conv1d step: batch %d, d_inner %d, width %d, fp32 window in place, one %s "
+                "token per sequence" % (c["batch"], c["dim"], c["width"], io))
+    if kind == "ssd":
+        return ("%s-shaped Mamba-2 SSD by 64-token chunks: batch %d, L %d, %d heads x %d, state %d, "
+                "%s x/B/C and y, fp32 a" % (name[3:], c["batch"], c["seqlen"], c["heads"],
+                                           c["headdim"], c["dstate"], io))
+    if kind == "decodemulti":
+        return ("decode, %d tokens per call on the carried state: batch %d, d_inner %d, N %d, "
+                "fp32 state in place, %s tokens" % (c["ntok"], c["batch"], c["dim"], c["dstate"], io))
+    if kind == "bwd":
+        return ("%s-shaped selective scan backward (states recomputed): batch %d, L %d, d_inner %d, "
+                "N %d, %s inputs, dy and gradients, fp32 A/D/bias gradients"
+                % (name[3:], c["batch"], c["seqlen"], c["dim"], c["dstate"], io))
+    if kind == "scan":
+        return ("%s-shaped selective scan: batch %d, L %d, d_inner %d, N %d, %s x/delta/z/B/C "
+                "and y, fp32 A/D/bias/state" % (name, c["batch"], c["seqlen"], c["dim"],
+                                                 c["dstate"], str(c["dtype"]).split(".")[-1]))
+    return ("decode state step: batch %d, d_inner %d, N %d, fp32 state in place, one %s token "
+            "per sequence" % (c["batch"], c["dim"], c["dstate"], str(c["dtype"]).split(".")[-1]))
 
 
 def kernel_name(kind):
@@ -535,7 +542,7 @@ def run_reference(args):
     line = dict(metric=METRIC, value=value, unit=UNIT, impl="reference", n_gpus=args.gpus,
                 steps=args.steps, warmup=args.warmup, ms_per_step=1e3 * wall / args.steps,
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
-                data="synthetic", config=dict(workload=args.workload, sample=what),
+                data="synthetic", config=dict(workload=describe_workload(args.workload), sample=what),
                 cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle", sample=what),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)

@@ -24,10 +24,11 @@
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library keeps
- *    no state between calls.  ssm_selective_scan_fwd may take a temporary scratch
- *    buffer with cudaMallocAsync / cudaFreeAsync on cuda_stream (long sequences with
- *    few channels, see below), and so does ssm_selective_scan_bwd; every other call
- *    allocates nothing.
+ *    no state between calls.  Three calls may take a temporary scratch buffer with
+ *    cudaMallocAsync / cudaFreeAsync on cuda_stream: ssm_selective_scan_fwd (and _ex)
+ *    for long sequences with few channels (see below), ssm_selective_scan_bwd and
+ *    ssm_ssd_fwd.  ssm_selective_scan_fwd_noalloc is the scan's form that never
+ *    allocates; every other call allocates nothing.
  *  - Every pointer must be 16-byte aligned (SSM_ERR_ALIGNMENT otherwise).
  *  - The call is asynchronous on `cuda_stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and never synchronises.  Argument errors are returned before
@@ -35,7 +36,8 @@
  *    kernel surface, as usual for CUDA, at the caller's next synchronisation.
  *  - dtype codes: SSM_F32 (fp32) or SSM_BF16 (bf16).  A, D, delta_bias and the state
  *    are always fp32; the state arithmetic is fp32 whatever the input dtype.
- *  - dstate (N) must be in 1..16 (SSM_ERR_UNSUPPORTED above 16).
+ *  - For the S6 calls (scan, backward, state steps) dstate (N) must be in 1..16
+ *    (SSM_ERR_UNSUPPORTED above 16); ssm_ssd_fwd takes its own sizes (below).
  *  - Output buffers must not overlap input buffers (the convolution checks and returns
  *    SSM_ERR_INVALID_ARG; for the scan the result of an overlap is undefined).
  */
@@ -123,9 +125,10 @@ int ssm_selective_scan_fwd_ex(const void *x, const void *delta, const float *del
  * with few channels are scanned in segments whose end states must be kept between
  * launches), this call uses a fixed 4 MiB array in device memory instead.  That array
  * exists on every GPU that loads the library and stays there until the process exits.
- *  - The first call on a device looks up the array's device address (a one-time set-up
- *    per device, done with that device current); make that first call before any CUDA
- *    stream capture on the device.
+ *  - Every call asks the runtime for the array's address in the current device's
+ *    context (a lookup, no allocation), so the address stays right after a
+ *    cudaDeviceReset.  The first call on a device may load the library's device code;
+ *    make that first call before any CUDA stream capture on the device.
  *  - A call whose segmented scan would need more than 4 MiB of scratch (batch * dim *
  *    segments * (padded dstate + 1) floats, padded dstate = 4, 8 or 16) returns
  *    SSM_ERR_SCRATCH and launches nothing.  Calls that need no segments work at any size.

@@ -217,51 +217,43 @@ def ssd_loop(x, a, B, C, h0=None):
     return y, hN
 
 
-def _segment_sums(a):
-    """a [..., T] -> [..., T, T]: entry (t, s) = a[s+1] + ... + a[t] for s <= t, -inf above
-    the diagonal (so that exp() gives the decay mask)."""
-    T = a.shape[-1]
-    cs = np.cumsum(a, axis=-1)
-    out = cs[..., :, None] - cs[..., None, :]
-    return np.where(np.tril(np.ones((T, T), dtype=bool)), out, -np.inf)
+def ssd_chunked(x, a, B, C, chunk=64, h0=None, dtype=np.float64):
+    """Mamba-2 SSD by chunks (xmarva lesson 10, section 8): inside a chunk the outputs are
+    masked attention, between chunks a recurrence on the P x N state.  Returns
+    ``(y, final_state)`` with the layouts of ``ssd_loop``.
 
-
-def ssd_chunked(x, a, B, C, chunk=64, h0=None):
-    """Mamba-2 SSD by chunks, in fp64 numpy: attention with the decay mask inside each chunk,
-    the recurrence between chunks (xmarva lesson 10, section 8: the four steps).  Returns
-    ``(y, final_state)``; the same layouts as ``ssd_loop``."""
-    x, a, B, C = (_f64(v) for v in (x, a, B, C))
+    Written per (sequence, head, chunk) with the chunk's own cumulative log-decay
+    g_i = a_{c0} + ... + a_{c0+i}:
+      within   y_i  = sum_{j<=i} (C_i . B_j) e^{g_i - g_j} x_j      (the decay-masked scores)
+      entering y_i += e^{g_i} S C_i                                 (the state that entered)
+      state    S    = e^{g_last} S + sum_j e^{g_last - g_j} x_j B_j^T
+    ``dtype`` is the arithmetic type (fp64 by default; fp32 shows the rounding of the
+    chunked order in single precision).
+    """
+    cast = lambda v: np.asarray(v, dtype=np.float64).astype(dtype)
+    x, a, B, C = cast(x), cast(a), cast(B), cast(C)
     batch, L, heads, P = x.shape
     N = B.shape[-1]
-    pad = (-L) % chunk
-    if pad:
-        x = np.concatenate([x, np.zeros((batch, pad, heads, P))], axis=1)
-        a = np.concatenate([a, np.zeros((batch, pad, heads))], axis=1)
-        B = np.concatenate([B, np.zeros((batch, pad, heads, N))], axis=1)
-        C = np.concatenate([C, np.zeros((batch, pad, heads, N))], axis=1)
-    nc = x.shape[1] // chunk
-    xc = x.reshape(batch, nc, chunk, heads, P)
-    Bc = B.reshape(batch, nc, chunk, heads, N)
-    Cc = C.reshape(batch, nc, chunk, heads, N)
-    ac = a.reshape(batch, nc, chunk, heads).transpose(0, 3, 1, 2)       # [b, h, c, l]
-    acum = np.cumsum(ac, axis=-1)
-    # (1) inside a chunk: y_l = sum_{s<=l} (C_l . B_s) exp(a_{s+1} + .. + a_l) x_s
-    mask = np.exp(_segment_sums(ac))                                      # [b, h, c, l, s]
-    y_in = np.einsum("bclhn,bcshn,bhcls,bcshp->bclhp", Cc, Bc, mask, xc)
-    # (2) what each chunk adds to the state: sum_s exp(a_{s+1} + .. + a_end) x_s B_s^T
-    to_end = np.exp(acum[..., -1:] - acum)                                # [b, h, c, l]
-    adds = np.einsum("bclhn,bhcl,bclhp->bchpn", Bc, to_end, xc)           # [b, c, h, p, n]
-    # (3) the state entering each chunk: S_0 = h0, S_{c+1} = exp(sum a of chunk c) S_c + adds_c
-    decay = np.exp(acum[..., -1])                                         # [b, h, c]
-    S = np.zeros((batch, heads, P, N)) if h0 is None else _f64(h0, (batch, heads, P, N)).copy()
-    entering = np.empty((batch, nc, heads, P, N))
-    for ci in range(nc):
-        entering[:, ci] = S
-        S = decay[:, :, ci][..., None, None] * S + adds[:, ci]
-    # (4) what each position reads from the state that entered its chunk
-    y_en = np.einsum("bclhn,bchpn,bhcl->bclhp", Cc, entering, np.exp(acum))
-    y = (y_in + y_en).reshape(batch, nc * chunk, heads, P)[:, :L]
-    return y, S
+    a = a.reshape(batch, L, heads)
+    y = np.zeros((batch, L, heads, P), dtype=dtype)
+    final = np.zeros((batch, heads, P, N), dtype=dtype)
+    for bi in range(batch):
+        for h in range(heads):
+            S = np.zeros((P, N), dtype=dtype) if h0 is None else cast(h0)[bi, h].copy()
+            for c0 in range(0, L, chunk):
+                c1 = min(L, c0 + chunk)
+                g = np.cumsum(a[bi, c0:c1, h], dtype=dtype)          # [l]
+                xs, bs, cs = x[bi, c0:c1, h], B[bi, c0:c1, h], C[bi, c0:c1, h]
+                n = c1 - c0
+                scores = cs @ bs.T                                  # [i, j] = C_i . B_j
+                mask = np.zeros((n, n), dtype=dtype)
+                for i in range(n):
+                    mask[i, :i + 1] = np.exp(g[i] - g[:i + 1])
+                y[bi, c0:c1, h] = (scores * mask) @ xs + np.exp(g)[:, None] * (cs @ S.T)
+                w = np.exp(g[-1] - g)                               # decay to the chunk end
+                S = np.exp(g[-1]) * S + (xs * w[:, None]).T @ bs
+            final[bi, h] = S
+    return y, final
 
 
 def causal_conv1d(x, weight, bias=None, hist=None, silu=True):

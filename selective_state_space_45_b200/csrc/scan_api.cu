@@ -6,7 +6,6 @@
 #include <algorithm>
 #include <climits>
 #include <cstdlib>
-#include <mutex>
 #include <type_traits>
 
 #include "api_host.cuh"
@@ -145,25 +144,18 @@ int dispatch_np(const ssm::ScanArgs &a, bool vec, cudaStream_t s) {
 constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;      // 4 MiB per GPU
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-float *g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device.  In host code the array's
-// name stands for a host-side shadow, not for device memory, so the address is looked up
-// once per device (with that device current) and cached.
+// Device address of g_noalloc_scratch in the current device's context.  In host code the
+// array's name stands for a host-side shadow, not for device memory, so the address is
+// asked of the runtime with the device current.  It is asked on every call rather than
+// cached: once the module is loaded this is a table lookup, and a context that was torn
+// down and recreated (cudaDeviceReset) may place the array elsewhere, so a cached address
+// could outlive the memory it named.  The first call on a device may load the module,
+// which is why that first call should come before any stream capture.
 int noalloc_scratch(float **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return SSM_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
-            return SSM_ERR_CUDA;
-        g_noalloc_ptr[dev] = static_cast<float *>(ptr);
-    }
-    *out = g_noalloc_ptr[dev];
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+        return SSM_ERR_CUDA;
+    *out = static_cast<float *>(ptr);
     return SSM_OK;
 }
 

@@ -573,26 +573,8 @@ def test_ssd_chunked_fp32_difference_is_of_the_printed_order():
     rng = np.random.default_rng(47)
     x, a, b, c = (v.astype(np.float32) for v in _ssd_case(rng))
     y, _ = oracle.ssd_loop(x, a, b, c)                      # fp64 of the fp32 inputs
-    # the chunked form evaluated in single precision (numpy float32 throughout)
-    cs = [v.astype(np.float32) for v in (x, a, b, c)]
-    L, chunk = 150, g["chunk"]
-    pad = (-L) % chunk
-    xp, ap, bp, cp = (np.concatenate([v, np.zeros((1, pad) + v.shape[2:], np.float32)], axis=1) for v in cs)
-    nc = xp.shape[1] // chunk
-    xr, br, cr = (v.reshape(1, nc, chunk, 3, -1) for v in (xp, bp, cp))
-    ar = ap.reshape(1, nc, chunk, 3).transpose(0, 3, 1, 2)
-    acum = np.cumsum(ar, axis=-1, dtype=np.float32)
-    seg = acum[..., :, None] - acum[..., None, :]
-    mask = np.where(np.tril(np.ones((chunk, chunk), bool)), np.exp(seg), np.float32(0))
-    y_in = np.einsum("bclhn,bcshn,bhcls,bcshp->bclhp", cr, br, mask, xr)
-    adds = np.einsum("bclhn,bhcl,bclhp->bchpn", br, np.exp(acum[..., -1:] - acum), xr)
-    S = np.zeros((1, 3, 8, 16), np.float32)
-    ent = np.empty((1, nc, 3, 8, 16), np.float32)
-    for ci in range(nc):
-        ent[:, ci] = S
-        S = np.exp(acum[..., ci, -1])[..., None, None] * S + adds[:, ci]
-    y_en = np.einsum("bclhn,bchpn,bhcl->bclhp", cr, ent, np.exp(acum))
-    y32 = (y_in + y_en).reshape(1, nc * chunk, 3, 8)[:, :L]
+    # the chunked form evaluated in single precision throughout
+    y32, _ = oracle.ssd_chunked(x, a, b, c, chunk=g["chunk"], dtype=np.float32)
     diff = float(np.abs(y32 - y).max())
     assert diff < 10 * g["printed_max_abs_difference_fp32"]
     assert diff > 0.0                                        # single precision does round
