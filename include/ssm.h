@@ -145,6 +145,17 @@ int ssm_selective_scan_fwd_noalloc(const void *x, const void *delta, const float
                                    int in_dtype, int out_dtype, void *cuda_stream);
 
 /*
+ * Testing and tuning only: force the number of time segments every following scan call
+ * (ssm_selective_scan_fwd, _ex, _noalloc) cuts each sequence into, whatever its shape, so
+ * that the long-sequence plan (tail sums, fold, segment scans) can be exercised on small
+ * inputs.  segments = 0 restores the automatic choice; a value above the sequence's tile
+ * count gives fewer, whole-tile segments.  Returns the previous setting, or -1 (nothing
+ * changed) for a negative argument.  Process-wide: calls that race with a scan on another
+ * host thread may see either setting.  The pages have no counterpart to this call.
+ */
+int ssm_scan_force_segments(int segments);
+
+/*
  * One decode step: every (b, d) channel takes one token and its state is updated in place.
  *
  *   state       : [batch][dim][dstate] fp32, read and overwritten.

@@ -69,6 +69,8 @@ def load_library(path: str | None = None):
         lib.ssm_status_string.argtypes = [i]
         lib.ssm_version.restype = i
         lib.ssm_version.argtypes = []
+        lib.ssm_scan_force_segments.restype = i
+        lib.ssm_scan_force_segments.argtypes = [i]
         _lib = lib
         return lib
 
@@ -79,6 +81,15 @@ def ssm_status_string(status: int) -> str:
 
 def ssm_version() -> int:
     return int(load_library().ssm_version())
+
+
+def ssm_scan_force_segments(segments: int) -> int:
+    """Testing and tuning: force the time-segment count of the following scans (0 restores
+    the automatic plan).  Returns the previous setting (see include/ssm.h)."""
+    prev = int(load_library().ssm_scan_force_segments(int(segments)))
+    if prev < 0:
+        raise ValueError("segments must be >= 0")
+    return prev
 
 
 def _ptr(t):

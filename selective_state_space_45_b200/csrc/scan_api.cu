@@ -4,8 +4,8 @@
 // Arguments are checked on the host before anything is launched; kernels run on the
 // caller's stream, asynchronously.
 #include <algorithm>
+#include <atomic>
 #include <climits>
-#include <cstdlib>
 #include <type_traits>
 
 #include "api_host.cuh"
@@ -17,15 +17,14 @@ namespace {
 
 constexpr int kMinSegTokens = 4096;     // shortest segment worth a carry correction
 
+// Segment count forced by ssm_scan_force_segments (0: automatic).
+std::atomic<int> g_forced_segments{0};
+
 // Segments per sequence: 1 while the channel groups alone fill every resident CTA slot
 // (`slots` = SMs x resident CTAs per SM); otherwise as many as fit in one wave of slots,
-// each at least kMinSegTokens long.  SSM_SCAN_SEGMENTS=k forces k (used by the tests to
-// reach the two-pass path).
+// each at least kMinSegTokens long.  A count forced through ssm_scan_force_segments wins.
 int choose_segments(long long channel_groups, int seqlen, long long slots) {
-    if (const char *e = std::getenv("SSM_SCAN_SEGMENTS")) {
-        const int v = std::atoi(e);
-        if (v >= 1) return v;
-    }
+    if (const int v = g_forced_segments.load(std::memory_order_relaxed); v >= 1) return v;
     if (2 * channel_groups >= slots) return 1;
     const long long want = slots / channel_groups;
     const long long room = seqlen / kMinSegTokens;
@@ -220,6 +219,11 @@ int dispatch_np_noalloc(const ssm::ScanArgs &a, bool vec, cudaStream_t s) {
 }  // namespace
 
 extern "C" {
+
+int ssm_scan_force_segments(int segments) {
+    if (segments < 0) return -1;
+    return g_forced_segments.exchange(segments);
+}
 
 int ssm_selective_scan_fwd(const void *x, const void *delta, const float *delta_bias,
                            int delta_softplus, const float *A, const void *B, const void *C,

@@ -31,3 +31,13 @@ def cuda_lib():
 
     ssm.load_library()
     return ssm
+
+
+@pytest.fixture
+def force_segments(cuda_lib):
+    """Set the library's forced time-segment count for one test (None or 0: automatic);
+    the automatic plan is restored afterwards."""
+    def setter(k):
+        cuda_lib.ssm_scan_force_segments(int(k or 0))
+    yield setter
+    cuda_lib.ssm_scan_force_segments(0)

@@ -1,5 +1,4 @@
 """GPU parity of ssm_selective_scan_fwd against the fp64 oracle (called through the C ABI)."""
-import os
 
 import numpy as np
 import pytest
@@ -14,21 +13,13 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.fixture(params=[None, "3"], ids=["oneCTA", "segments3"])
-def split(request):
+@pytest.fixture(params=[None, 3], ids=["oneCTA", "segments3"])
+def split(request, force_segments):
     """Both scan paths: one CTA per channel group over the whole sequence, and the
-    sequence cut into (up to) 3 segments -- pass 1 from a zero state, then the fold of the
-    end states and the carry's share of the output of every later segment."""
-    old = os.environ.get("SSM_SCAN_SEGMENTS")
-    if request.param is None:
-        os.environ.pop("SSM_SCAN_SEGMENTS", None)
-    else:
-        os.environ["SSM_SCAN_SEGMENTS"] = request.param
+    sequence cut into (up to) 3 segments -- the tail sums of the earlier segments, their
+    fold into every segment's carry, and one scan per segment from its carry."""
+    force_segments(request.param)
     yield request.param
-    if old is None:
-        os.environ.pop("SSM_SCAN_SEGMENTS", None)
-    else:
-        os.environ["SSM_SCAN_SEGMENTS"] = old
 
 
 def run_gpu(ssm, inp, out_dtype, use_z=True, use_D=True, use_bias=True, softplus=True):
@@ -181,10 +172,10 @@ def test_misaligned_pointer_rejected_on_device(cuda_lib):
 
 
 @pytest.mark.parametrize("nseg", ["2", "5"])
-def test_segment_carry_never_dies(cuda_lib, nseg, monkeypatch):
+def test_segment_carry_never_dies(cuda_lib, nseg, force_segments):
     """A = 0 keeps exp(A * S) = 1: the carry reaches every token of every later segment,
     so the carry pass must cover whole segments."""
-    monkeypatch.setenv("SSM_SCAN_SEGMENTS", nseg)
+    force_segments(int(nseg))
     inp = inputs.make_scan_inputs(1, 40, 700, 16, torch.float32, device=DEV, seed=21)
     inp["A"][:, :3] = 0.0
     inp["A"][:, 3:8] = 0.05          # a slowly growing state as well
@@ -194,10 +185,10 @@ def test_segment_carry_never_dies(cuda_lib, nseg, monkeypatch):
     assert_parity(fs, fr, torch.float32, what="final_state")
 
 
-def test_segment_carry_dies_at_once(cuda_lib, monkeypatch):
+def test_segment_carry_dies_at_once(cuda_lib, force_segments):
     """Huge steps wipe the carry within one token: the carry pass stops in its first
     window and the pass-1 output stands."""
-    monkeypatch.setenv("SSM_SCAN_SEGMENTS", "4")
+    force_segments(4)
     inp = inputs.make_scan_inputs(2, 33, 512, 16, torch.bfloat16, device=DEV, seed=22)
     inp["delta_bias"].fill_(60.0)
     y, fs = run_gpu(cuda_lib, inp, torch.bfloat16)
@@ -207,11 +198,11 @@ def test_segment_carry_dies_at_once(cuda_lib, monkeypatch):
 
 
 @pytest.mark.parametrize("nseg", ["3", "7"])
-def test_segment_carry_with_negative_steps(cuda_lib, nseg, monkeypatch):
+def test_segment_carry_with_negative_steps(cuda_lib, nseg, force_segments):
     """Without the softplus a raw step can be negative, so the step sum S_t of a segment
     can fall again after rising: the carry's share exp(A S_t) h_in is checked against the
     oracle on every block, not cut off at the first small value."""
-    monkeypatch.setenv("SSM_SCAN_SEGMENTS", nseg)
+    force_segments(int(nseg))
     inp = inputs.make_scan_inputs(2, 24, 900, 16, torch.float32, device=DEV, seed=24)
     g = torch.Generator(DEV).manual_seed(25)
     inp["delta"] = (0.05 * torch.randn(inp["delta"].shape, device=DEV, generator=g) + 0.01).contiguous()
