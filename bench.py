@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2p8b",
-                    choices=["mamba130m", "mamba2p8b", "long1m", "decode", "tiny",
+                    choices=["mamba130m", "mamba2p8b", "long1m", "long1m_slow", "decode", "tiny",
                              "conv130m", "conv2p8b", "convstep", "bwd130m", "decode4", "ssd130m"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -121,7 +121,7 @@ def load_peaks():
 
 # translation unit of libssm.so that holds each kernel and its launch logic
 KERNEL_UNIT = {"scan_fwd_kernel": "scan_api.cu", "state_step_kernel": "step_api.cu",
-               "state_steps_kernel": "step_api.cu", "ssd_chunk_scan_kernel": "ssd_api.cu",
+               "state_steps_kernel": "step_api.cu", "ssd_tc_kernel": "ssd_api.cu",
                "scan_bwd_kernel": "bwd_api.cu",
                "causal_conv1d_vec_kernel": "conv_api.cu", "conv1d_step_kernel": "conv_api.cu"}
 
@@ -230,7 +230,7 @@ def bwd_counts(batch, dim, L, N, in_size, g_size):
     return dict(bytes=streams + bc + params, exps=2 * batch * L * dim * N, tokch=batch * L * dim)
 
 
-def ssd_counts(batch, L, heads, P, N, in_size, out_size, Q=64):
+def ssd_counts(batch, L, heads, P, N, in_size, out_size, Q=128):
     """SSD by chunks: x, B, C, a read once and y written once; work = the four chunk products
     (scores C B^T, masked scores times x, C times the entering state, B^T times the weighted
     inputs), 2 flops per multiply-add, over whole chunks."""
@@ -378,7 +378,7 @@ def describe_workload(name):
         return ("decode conv1d step: batch %d, d_inner %d, width %d, fp32 window in place, one %s "
                 "token per sequence" % (c["batch"], c["dim"], c["width"], io))
     if kind == "ssd":
-        return ("%s-shaped Mamba-2 SSD by 64-token chunks: batch %d, L %d, %d heads x %d, state %d, "
+        return ("%s-shaped Mamba-2 SSD by 128-token chunks: batch %d, L %d, %d heads x %d, state %d, "
                 "%s x/B/C and y, fp32 a" % (name[3:], c["batch"], c["seqlen"], c["heads"],
                                            c["headdim"], c["dstate"], io))
     if kind == "decodemulti":
@@ -399,7 +399,7 @@ def describe_workload(name):
 def kernel_name(kind):
     return dict(scan="scan_fwd_kernel", decode="state_step_kernel", conv="causal_conv1d_vec_kernel",
                 convstep="conv1d_step_kernel", bwd="scan_bwd_kernel",
-                decodemulti="state_steps_kernel", ssd="ssd_chunk_scan_kernel")[kind]
+                decodemulti="state_steps_kernel", ssd="ssd_tc_kernel")[kind]
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -471,10 +471,10 @@ def _oracle_sample(name, n_target_tokch, seed=0):
     if k == 1 and n_target_tokch < per_channel:  # one channel of one sequence, shortened
         L = int(max(64, min(L, n_target_tokch)))
         inp = inputs.make_scan_inputs(1, 1, L, c["dstate"], c["dtype"], device="cpu", seed=seed,
-                                      dt_dist=c["dt_dist"])
+                                      dt_dist=c["dt_dist"], a_dist=c.get("a_dist", "index"))
         return "scan", inp, L, "1 channel of 1 sequence, first %d of %d tokens" % (L, c["seqlen"])
     inp = inputs.make_scan_inputs(c["batch"], k, L, c["dstate"], c["dtype"], device="cpu", seed=seed,
-                                  dt_dist=c["dt_dist"])
+                                  dt_dist=c["dt_dist"], a_dist=c.get("a_dist", "index"))
     return "scan", inp, per_channel * k, "%d sequences x %d of %d channels, all %d tokens" % (
         c["batch"], k, c["dim"], L)
 
@@ -712,7 +712,10 @@ def run_ours(args):
                     frac=achieved / peak_gexp,
                     traffic=recorded_traffic(kernel_name(wl.kind), wl.name),
                     kernel=kernel_name(wl.kind), kernel_ms=kern_ms,
-                    peak_basis="148 SMs x 16 ex2/clk/SM x %.0f MHz max SM clock" % peaks["sm_max_mhz"],
+                    peak_basis=("148 SMs x 16 ex2/clk/SM x %.0f MHz max SM clock; the 16 ex2/clk/SM "
+                                "is the SFU rate of the CUDA programming guide's throughput table "
+                                "for compute capability 10.x, not measured by this script"
+                                % peaks["sm_max_mhz"]),
                     hbm=dict(achieved_gbs=gbs, peak_gbs=peaks["hbm_gbs"], frac=gbs / peaks["hbm_gbs"],
                              peak_source=peaks["source"]))
     elif wl.kind == "ssd":
@@ -748,7 +751,7 @@ def run_ours(args):
         if "width" in c:
             config.update(width=c["width"])
         if "heads" in c:
-            config.update(heads=c["heads"], headdim=c["headdim"], chunk=64)
+            config.update(heads=c["heads"], headdim=c["headdim"], chunk=128)
         if "seqlen" in c:
             config.update(seqlen=c["seqlen"], global_batch=c["batch"] * world)
         line = dict(metric=METRIC, value=total_units / sec, unit=UNIT, n_gpus=world, steps=args.steps,

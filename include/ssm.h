@@ -24,11 +24,11 @@
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library keeps
- *    no state between calls.  Three calls may take a temporary scratch buffer with
+ *    no state between calls.  Two calls may take a temporary scratch buffer with
  *    cudaMallocAsync / cudaFreeAsync on cuda_stream: ssm_selective_scan_fwd (and _ex)
- *    for long sequences with few channels (see below), ssm_selective_scan_bwd and
- *    ssm_ssd_fwd.  ssm_selective_scan_fwd_noalloc is the scan's form that never
- *    allocates; every other call allocates nothing.
+ *    for long sequences with few channels (see below), and ssm_selective_scan_bwd.
+ *    ssm_selective_scan_fwd_noalloc is the scan's form that never allocates; every
+ *    other call allocates nothing.
  *  - Every pointer must be 16-byte aligned (SSM_ERR_ALIGNMENT otherwise).
  *  - The call is asynchronous on `cuda_stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and never synchronises.  Argument errors are returned before
@@ -277,8 +277,8 @@ int ssm_state_step_multi(float *state, const void *x, const void *delta, const f
  * models and hybrids", xmarva lesson 10, section 8 "Mamba-2: the same model as
  * attention"): one decay per head and a headdim x dstate state per head,
  *     S <- exp(a_t) S + x_t B_t^T,    y_t = S C_t    (per sequence and head)
- * computed as attention with the decay mask inside chunks of 64 tokens and the recurrence
- * between chunks.  x already carries the step (x = Delta * input), a = Delta * A.
+ * computed as attention with the decay mask inside chunks of 128 tokens and the
+ * recurrence between chunks.  x already carries the step (x = Delta * input), a = Delta * A.
  *
  *   x, y          : [batch][seqlen][heads][headdim]; x bf16, y out_dtype (written).
  *   a             : [batch][seqlen][heads] fp32.
@@ -286,17 +286,26 @@ int ssm_state_step_multi(float *state, const void *x, const void *delta, const f
  *   initial_state : [batch][heads][headdim][dstate] fp32 or NULL (zero).
  *   final_state   : [batch][heads][headdim][dstate] fp32 or NULL (not written).
  * in_dtype must be SSM_BF16 (the tensor-core operands); headdim 32 or 64 and dstate 64 or
- * 128 (SSM_ERR_UNSUPPORTED otherwise).  Products run on bf16 operands with fp32
- * accumulation; the masked scores, the decay-weighted inputs and the state are rounded to
- * bf16 where they enter a product.  seqlen = 0 copies the start state through.  Takes a
- * stream-ordered scratch buffer (cudaMallocAsync / cudaFreeAsync on cuda_stream) of
- * 6 * headdim * dstate bytes per (sequence, head, 64-token chunk): every chunk's state
- * contribution (fp32) and entering state (bf16).
+ * 128 (SSM_ERR_UNSUPPORTED otherwise).  Products run on the tensor cores (tcgen05) on bf16
+ * operands with fp32 accumulation; the masked scores, the decay-weighted inputs and the
+ * state are rounded to bf16 where they enter a product.  The state stays on the chip
+ * between chunks (fp32): the call allocates nothing and writes only y and final_state.
+ * seqlen = 0 copies the start state through.  Uses up to 227 KB of shared memory and 512
+ * tensor-memory columns per CTA (one CTA per SM).
  */
 int ssm_ssd_fwd(const void *x, const float *a, const void *B, const void *C, void *y,
                 const float *initial_state, float *final_state,
                 int batch, int seqlen, int heads, int headdim, int dstate,
                 int in_dtype, int out_dtype, void *cuda_stream);
+
+/*
+ * Number of times, since the library was loaded on the current device, that a kernel gave
+ * up waiting on its own asynchronous copies or tensor-core operations (each such wait is
+ * bounded, about a second).  0 in normal operation; a nonzero count means the results of
+ * the call that timed out are not valid.  Synchronises with the device; ~0u if the count
+ * cannot be read.  The pages have no counterpart to this call.
+ */
+unsigned ssm_device_timeouts(void);
 
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char *ssm_status_string(int status);

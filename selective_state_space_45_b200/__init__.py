@@ -22,6 +22,7 @@ from ._lib import (  # noqa: F401
     ssd,
     ssm_causal_conv1d_fwd,
     ssm_causal_conv1d_step,
+    ssm_device_timeouts,
     ssm_selective_scan_bwd,
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_ex,

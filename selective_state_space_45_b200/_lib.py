@@ -69,6 +69,8 @@ def load_library(path: str | None = None):
         lib.ssm_status_string.argtypes = [i]
         lib.ssm_version.restype = i
         lib.ssm_version.argtypes = []
+        lib.ssm_device_timeouts.restype = ctypes.c_uint
+        lib.ssm_device_timeouts.argtypes = []
         lib.ssm_scan_force_segments.restype = i
         lib.ssm_scan_force_segments.argtypes = [i]
         _lib = lib
@@ -81,6 +83,12 @@ def ssm_status_string(status: int) -> str:
 
 def ssm_version() -> int:
     return int(load_library().ssm_version())
+
+
+def ssm_device_timeouts() -> int:
+    """How many bounded waits inside the library's kernels gave up on this device (0 in
+    normal operation; see include/ssm.h).  Synchronises with the device."""
+    return int(load_library().ssm_device_timeouts())
 
 
 def ssm_scan_force_segments(segments: int) -> int:

@@ -99,6 +99,12 @@ __device__ __forceinline__ float2 exp2_poly_pair(float2 v) {
     return f2(__uint_as_float(ex), __uint_as_float(ey));
 }
 
+// A pair of bf16 values packed in 32 bits (first in the low half) as an fp32 pair: bf16 ->
+// fp32 is a 16-bit shift (exact).
+__device__ __forceinline__ float2 bf16x2_to_f2(unsigned w) {
+    return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {

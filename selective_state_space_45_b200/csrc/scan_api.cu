@@ -42,11 +42,16 @@ long long resident_slots(Kernel kernel, int threads, size_t smem) {
     return (long long)sms * per_sm;
 }
 
-template <class Cfg, bool SEG, bool ZOH = false>
+template <class Cfg, bool SEG, bool ZOH>
+constexpr auto scan_kernel() {
+    return &ssm::scan_fwd_kernel<Cfg, SEG, ZOH>;
+}
+
+template <class Cfg, bool SEG, bool ZOH>
 int launch_scan_kernel(const ssm::ScanArgs &a, long long blocks, cudaStream_t stream) {
     if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
     if (blocks == 0) return SSM_OK;
-    ssm::scan_fwd_kernel<Cfg, SEG, ZOH><<<unsigned(blocks), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(a);
+    scan_kernel<Cfg, SEG, ZOH>()<<<unsigned(blocks), Cfg::NTHREADS, Cfg::SMEM_BYTES, stream>>>(a);
     return status_of(cudaGetLastError());
 }
 
@@ -67,63 +72,67 @@ int launch_tail_fold(const ssm::ScanArgs &a, cudaStream_t stream) {
     return status_of(cudaGetLastError());
 }
 
+// The launch plan shared by the regular and the allocation-free scans: channel groups,
+// the shared-memory opt-in of both kernel variants, and the segment count and length.
+template <class Cfg, bool ZOH>
+int plan_scan(ssm::ScanArgs &a, long long &cgroups) {
+    const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
+    if (groups > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    a.groups_per_seq = int(groups);
+    cgroups = groups * a.batch;
+    const size_t smem = Cfg::SMEM_BYTES;
+    if (smem > 48 * 1024) {   // opt in to large shared memory for both kernel variants
+        if (cudaFuncSetAttribute(scan_kernel<Cfg, false, ZOH>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess ||
+            cudaFuncSetAttribute(scan_kernel<Cfg, true, ZOH>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess)
+            return SSM_ERR_CUDA;
+    }
+    const long long slots = resident_slots(scan_kernel<Cfg, true, ZOH>(), Cfg::NTHREADS, smem);
+    int nseg = choose_segments(cgroups, a.seqlen, slots > 0 ? slots : 2 * cgroups);
+    long long seg_len = (a.seqlen + nseg - 1) / nseg;
+    seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
+    a.nseg = int((a.seqlen + seg_len - 1) / seg_len);
+    a.seg_len = a.nseg <= 1 ? a.seqlen : int(seg_len);
+    if (a.nseg < 1) a.nseg = 1;
+    return SSM_OK;
+}
+
 // One scan: a single pass when the sequence fits one CTA per channel group, else the tail
 // and fold passes and one scan per segment from its carry, with a stream-ordered scratch
 // buffer of batch*dim*nseg*(NP+1) floats.
 template <class Cfg, bool ZOH>
 int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
     ssm::ScanArgs a = a0;
-    const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
-    if (groups > INT_MAX) return SSM_ERR_UNSUPPORTED;
-    a.groups_per_seq = int(groups);
-    const long long cgroups = groups * a.batch;
-    const size_t smem = Cfg::SMEM_BYTES;
-    if (smem > 48 * 1024) {   // opt in to large shared memory for both kernel variants
-        if (cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, false, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, true, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(smem)) != cudaSuccess)
-            return SSM_ERR_CUDA;
-    }
-    const long long slots = resident_slots(ssm::scan_fwd_kernel<Cfg, true, ZOH>, Cfg::NTHREADS, smem);
-    int nseg = choose_segments(cgroups, a.seqlen, slots > 0 ? slots : 2 * cgroups);
-    long long seg_len = (a.seqlen + nseg - 1) / nseg;
-    seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
-    nseg = int((a.seqlen + seg_len - 1) / seg_len);
-    if (nseg <= 1) {
-        a.nseg = 1;
-        a.seg_len = a.seqlen;
-        return launch_scan_kernel<Cfg, false, ZOH>(a, cgroups, stream);
-    }
-    const size_t rows = size_t(a.batch) * a.dim * nseg;
+    long long cgroups = 0;
+    int st = plan_scan<Cfg, ZOH>(a, cgroups);
+    if (st != SSM_OK) return st;
+    if (a.nseg == 1) return launch_scan_kernel<Cfg, false, ZOH>(a, cgroups, stream);
+    const size_t rows = size_t(a.batch) * a.dim * a.nseg;
     const size_t bytes = rows * Cfg::NP * sizeof(float) + rows * sizeof(float);
     void *ws = nullptr;
     if (cudaMallocAsync(&ws, bytes, stream) != cudaSuccess) return SSM_ERR_CUDA;
-    a.nseg = nseg;
-    a.seg_len = int(seg_len);
     a.seg_h = static_cast<float *>(ws);
     a.seg_s = a.seg_h + rows * Cfg::NP;
-    int st = launch_tail_fold<Cfg, ZOH>(a, stream);
-    if (st == SSM_OK) st = launch_scan_kernel<Cfg, true, ZOH>(a, cgroups * nseg, stream);
+    st = launch_tail_fold<Cfg, ZOH>(a, stream);
+    if (st == SSM_OK) st = launch_scan_kernel<Cfg, true, ZOH>(a, cgroups * a.nseg, stream);
     const cudaError_t fe = cudaFreeAsync(ws, stream);
     if (st == SSM_OK && fe != cudaSuccess) st = SSM_ERR_CUDA;
     return st;
 }
 
 // Tile shape per padded state width: 32-token tiles; 32 channels per CTA (64 at N <= 4).
-#ifndef SSM_SCAN16_MINB
-#define SSM_SCAN16_MINB 4     // resident CTAs per SM the 16-state kernel's registers target
-#endif
-#ifndef SSM_SCAN16_NSTAGE
-#define SSM_SCAN16_NSTAGE 3   // cp.async ring depth of the 16-state kernel
-#endif
+template <int NP, typename Tin, typename Tout, bool VEC>
+struct ScanConfig {
+    using C16 = ssm::ScanCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>;
+    using C8 = ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>;
+    using C4 = ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>;
+    using type = std::conditional_t<NP == 16, C16, std::conditional_t<NP == 8, C8, C4>>;
+};
 
 template <int NP, typename Tin, typename Tout, bool VEC>
 int dispatch_cfg(const ssm::ScanArgs &a, cudaStream_t s) {
-    using C16 = ssm::ScanCfg<16, 1, 32, SSM_SCAN16_NSTAGE, Tin, Tout, VEC, SSM_SCAN16_MINB>;
-    using C8 = ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>;
-    using C4 = ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>;
-    using Cfg = std::conditional_t<NP == 16, C16, std::conditional_t<NP == 8, C8, C4>>;
+    using Cfg = typename ScanConfig<NP, Tin, Tout, VEC>::type;
     return a.zoh ? run_scan<Cfg, true>(a, s) : run_scan<Cfg, false>(a, s);
 }
 
@@ -165,47 +174,24 @@ int noalloc_scratch(float **out) {
 template <class Cfg>
 int run_scan_noalloc(const ssm::ScanArgs &a0, cudaStream_t stream) {
     ssm::ScanArgs a = a0;
-    const long long groups = (a.dim + Cfg::CH - 1) / Cfg::CH;
-    if (groups > INT_MAX) return SSM_ERR_UNSUPPORTED;
-    a.groups_per_seq = int(groups);
-    const long long cgroups = groups * a.batch;
-    const size_t smem = Cfg::SMEM_BYTES;
-    if (smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(ssm::scan_fwd_kernel<Cfg, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(smem)) != cudaSuccess)
-            return SSM_ERR_CUDA;
-    }
-    const long long slots = resident_slots(ssm::scan_fwd_kernel<Cfg, true, false>, Cfg::NTHREADS, smem);
-    int nseg = choose_segments(cgroups, a.seqlen, slots > 0 ? slots : 2 * cgroups);
-    long long seg_len = (a.seqlen + nseg - 1) / nseg;
-    seg_len = (seg_len + Cfg::T - 1) / Cfg::T * Cfg::T;
-    nseg = int((a.seqlen + seg_len - 1) / seg_len);
-    if (nseg <= 1) {
-        a.nseg = 1;
-        a.seg_len = a.seqlen;
-        return launch_scan_kernel<Cfg, false>(a, cgroups, stream);
-    }
-    const size_t rows = size_t(a.batch) * a.dim * nseg;
+    long long cgroups = 0;
+    int st = plan_scan<Cfg, false>(a, cgroups);
+    if (st != SSM_OK) return st;
+    if (a.nseg == 1) return launch_scan_kernel<Cfg, false, false>(a, cgroups, stream);
+    const size_t rows = size_t(a.batch) * a.dim * a.nseg;
     if (rows * (Cfg::NP + 1) > kNoAllocScratchFloats) return SSM_ERR_SCRATCH;
     float *ws = nullptr;
-    const int st0 = noalloc_scratch(&ws);
-    if (st0 != SSM_OK) return st0;
-    a.nseg = nseg;
-    a.seg_len = int(seg_len);
+    st = noalloc_scratch(&ws);
+    if (st != SSM_OK) return st;
     a.seg_h = ws;
     a.seg_s = ws + rows * Cfg::NP;
-    const int st = launch_tail_fold<Cfg, false>(a, stream);
-    return st == SSM_OK ? launch_scan_kernel<Cfg, true>(a, cgroups * nseg, stream) : st;
+    st = launch_tail_fold<Cfg, false>(a, stream);
+    return st == SSM_OK ? launch_scan_kernel<Cfg, true, false>(a, cgroups * a.nseg, stream) : st;
 }
 
 template <int NP, typename Tin, typename Tout, bool VEC>
 int dispatch_cfg_noalloc(const ssm::ScanArgs &a, cudaStream_t s) {
-    if constexpr (NP == 16)
-        return run_scan_noalloc<ssm::ScanCfg<16, 1, 32, SSM_SCAN16_NSTAGE, Tin, Tout, VEC, SSM_SCAN16_MINB>>(a, s);
-    else if constexpr (NP == 8) return run_scan_noalloc<ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>>(a, s);
-    else return run_scan_noalloc<ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>>(a, s);
+    return run_scan_noalloc<typename ScanConfig<NP, Tin, Tout, VEC>::type>(a, s);
 }
 
 template <typename Tin, typename Tout>

@@ -93,6 +93,12 @@ struct ScanCfg {
     static_assert(T % 8 == 0, "tile must hold whole 8-token chunks");
     static_assert(NTASK % NTHREADS == 0, "tasks must divide evenly");
 
+    // bf16 inputs: the recurrence reads B and C of a state quad as one 16-byte word of
+    // bf16 pairs (B quad, then C quad) and widens them in registers.  A shared-memory load
+    // that all lanes of a warp share still costs one wavefront per 4 bytes, so this halves
+    // the shared-memory traffic of the recurrence against fp32 B and C rows.
+    static constexpr bool BCPACK = sizeof(Tin) == 2;
+
     static constexpr size_t al(size_t v) { return (v + 15) & ~size_t(15); }
     static constexpr size_t RAW_ARR = al(size_t(CH) * RAW_ROW * sizeof(Tin));
     static constexpr size_t RAW_BC = al(size_t(T) * NP * sizeof(Tin));
@@ -100,9 +106,12 @@ struct ScanCfg {
     static constexpr size_t OFF_RAW = 0;
     // prep: float4 [T/2][CH] = (Delta_t, Delta_t x_t, Delta_t+1, Delta_t+1 x_t+1)
     static constexpr size_t OFF_PREP = OFF_RAW + NSTAGE * STAGE_BYTES;
+    // B, C of the tile: packed uint4 [T][Q] (bf16 inputs), else fp32 rows [T][NP] each
+    static constexpr size_t BF_BYTES = BCPACK ? al(size_t(T) * Q * 16) : al(size_t(T) * NP * sizeof(float));
+    static constexpr size_t CF_BYTES = BCPACK ? 0 : al(size_t(T) * NP * sizeof(float));
     static constexpr size_t OFF_BF = OFF_PREP + al(size_t(T / 2) * CH * sizeof(float4));
-    static constexpr size_t OFF_CF = OFF_BF + al(size_t(T) * NP * sizeof(float));
-    static constexpr size_t OFF_YP = OFF_CF + al(size_t(T) * NP * sizeof(float));
+    static constexpr size_t OFF_CF = OFF_BF + BF_BYTES;
+    static constexpr size_t OFF_YP = OFF_CF + CF_BYTES;
     static constexpr size_t OFF_Y = OFF_YP + al(size_t(Q) * CH * YP_ROW * sizeof(float));
     static constexpr size_t SMEM_BYTES = OFF_Y + al(size_t(CH) * Y_ROW * sizeof(Tout));
 };
@@ -121,13 +130,14 @@ template <class Cfg> struct Stage {
 };
 
 // Stage tile [t0, t0 + T) of x, delta, z (rows of nch channels) and of B, C into ring stage
-// st, with every index split by compile-time divisors.  VEC: 16-byte cp.async chunks, each
-// wholly inside or wholly outside [0, L) because L is a multiple of the chunk width.
-template <class Cfg>
+// st, with every index split by compile-time divisors; thread `me` of the NT staging
+// threads.  VEC: 16-byte cp.async chunks, each wholly inside or wholly outside [0, L)
+// because L is a multiple of the chunk width.
+template <class Cfg, int NT = Cfg::NTHREADS>
 __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem, int st, int t0,
-                                                size_t row0, size_t bc0, int nch) {
+                                          size_t row0, size_t bc0, int nch, int me = tid_x()) {
     using Tin = typename Cfg::Tin;
-    constexpr int CH = Cfg::CH, T = Cfg::T, NT = Cfg::NTHREADS, EIN = Cfg::EIN, NP = Cfg::NP;
+    constexpr int CH = Cfg::CH, T = Cfg::T, EIN = Cfg::EIN, NP = Cfg::NP;
     Stage<Cfg> s(smem, st);
     const int L = p.seqlen, N = p.dstate;
     const Tin *gx = static_cast<const Tin *>(p.x) + row0;
@@ -141,7 +151,7 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
         constexpr int ROWC = 3 * CH * CPR;
 #pragma unroll
         for (int k = 0; k < (ROWC + NT - 1) / NT; ++k) {
-            const int i = tid_x() + k * NT;
+            const int i = me + k * NT;
             const int a = i / (CH * CPR);
             const int rem = i % (CH * CPR);
             const int cc = rem / CPR, q = rem % CPR;
@@ -155,7 +165,7 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
             constexpr int BCC = T * NP / EIN;        // chunks per array
 #pragma unroll
             for (int k = 0; k < (2 * BCC + NT - 1) / NT; ++k) {
-                const int i = tid_x() + k * NT;
+                const int i = me + k * NT;
                 const int which = i / BCC, q = i % BCC;
                 if (i < 2 * BCC && t0 + (q * EIN) / NP < L)   // first token of the chunk
                     cp_async_16((which ? s.cs : s.bs) + q * EIN, (which ? gc : gb) + q * EIN);
@@ -163,7 +173,7 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
         } else {
             const int valid_t = min(T, L - t0);
             const int bc_chunks = (valid_t * N * int(sizeof(Tin))) / 16;
-            for (int i = tid_x(); i < 2 * bc_chunks; i += NT) {
+            for (int i = me; i < 2 * bc_chunks; i += NT) {
                 const int which = i >= bc_chunks;
                 const int q = i - which * bc_chunks;
                 cp_async_16((which ? s.cs : s.bs) + q * EIN, (which ? gc : gb) + q * EIN);
@@ -173,7 +183,7 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
         constexpr int NEL = 3 * CH * T;
 #pragma unroll 4
         for (int k = 0; k < (NEL + NT - 1) / NT; ++k) {
-            const int i = tid_x() + k * NT;
+            const int i = me + k * NT;
             const int a = i / (CH * T);
             const int rem = i % (CH * T);
             const int cc = rem / T, tt = rem % T;
@@ -184,7 +194,7 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
             }
         }
         const int nbc = min(T, L - t0) * N;
-        for (int i = tid_x(); i < 2 * nbc; i += NT) {
+        for (int i = me; i < 2 * nbc; i += NT) {
             const int which = i >= nbc;
             const int q = i - which * nbc;
             (which ? s.cs : s.bs)[q] = (which ? gc : gb)[q];
@@ -326,8 +336,38 @@ scan_fwd_kernel(const ScanArgs p) {
             for (int u2 = 0; u2 < 4; ++u2)
                 prep[(4 * t8 + u2) * CH + cc] = make_float4(o[4 * u2], o[4 * u2 + 1], o[4 * u2 + 2], o[4 * u2 + 3]);
         }
-        // B, C of the tile widened to fp32, zero past dstate / past L
-        if (N == NP && t0 + T <= L) {                       // dense rows: 8 values at a time
+        // B, C of the tile for the recurrence, zero past dstate / past L: packed bf16 quads
+        // (B quad, C quad) per (token, quad) for bf16 inputs, else fp32 rows
+        if constexpr (Cfg::BCPACK) {
+            uint4 *bcp = reinterpret_cast<uint4 *>(Bf);
+            const unsigned short *rb = reinterpret_cast<const unsigned short *>(sv.bs);
+            const unsigned short *rc = reinterpret_cast<const unsigned short *>(sv.cs);
+#pragma unroll
+            for (int k = 0; k < (T * Q + NT - 1) / NT; ++k) {
+                const int i = tid + k * NT;
+                if (i < T * Q) {
+                    const int tt = i / Q, qq = i % Q;
+                    uint4 v;
+                    if (N == NP && t0 + tt < L) {            // dense rows: two 8-byte reads
+                        const uint2 b2 = *reinterpret_cast<const uint2 *>(rb + tt * NP + 4 * qq);
+                        const uint2 c2 = *reinterpret_cast<const uint2 *>(rc + tt * NP + 4 * qq);
+                        v = make_uint4(b2.x, b2.y, c2.x, c2.y);
+                    } else {
+                        unsigned bw[4], cw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int n = 4 * qq + e;
+                            const bool ok = n < N && t0 + tt < L;
+                            bw[e] = ok ? rb[tt * N + n] : 0u;
+                            cw[e] = ok ? rc[tt * N + n] : 0u;
+                        }
+                        v = make_uint4(bw[0] | (bw[1] << 16), bw[2] | (bw[3] << 16),
+                                       cw[0] | (cw[1] << 16), cw[2] | (cw[3] << 16));
+                    }
+                    bcp[i] = v;
+                }
+            }
+        } else if (N == NP && t0 + T <= L) {                // dense rows: 8 values at a time
             constexpr int NV = T * NP / 8;
 #pragma unroll
             for (int k = 0; k < (2 * NV + NT - 1) / NT; ++k) {
@@ -358,17 +398,43 @@ scan_fwd_kernel(const ScanArgs p) {
         {
             const float4 *pp = prep + c;
             float *ypr = yp + (q * CH + c) * Cfg::YP_ROW;
+            const uint4 *bcp = reinterpret_cast<const uint4 *>(Bf) + q;
+            // the B and C quads of token t as fp32 pairs (0,1), (2,3)
+            auto bquad = [&](int t, float2 (&bb)[2], uint2 &craw) {
+                if constexpr (Cfg::BCPACK) {
+                    const uint4 v = bcp[t * Cfg::Q];
+                    bb[0] = bf16x2_to_f2(v.x);
+                    bb[1] = bf16x2_to_f2(v.y);
+                    craw = make_uint2(v.z, v.w);
+                } else {
+                    const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
+                    bb[0] = f2(bq.x, bq.y);
+                    bb[1] = f2(bq.z, bq.w);
+                    craw = make_uint2(0u, 0u);
+                }
+            };
+            auto cquad = [&](int t, uint2 craw, float2 (&cc)[2]) {
+                if constexpr (Cfg::BCPACK) {
+                    cc[0] = bf16x2_to_f2(craw.x);
+                    cc[1] = bf16x2_to_f2(craw.y);
+                } else {
+                    const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
+                    cc[0] = f2(cq.x, cq.y);
+                    cc[1] = f2(cq.z, cq.w);
+                }
+            };
             // decays a = exp(Delta*A) and writes w = Delta*x*B of the 4 tokens of group g, as
-            // state pairs (0,1), (2,3) for the packed FP32 instructions
-            auto decay_write = [&](int g, float2 (&a)[4][2], float2 (&w)[4][2]) {
+            // state pairs (0,1), (2,3) for the packed FP32 instructions; the C quads (packed
+            // form) are kept for the readout
+            auto decay_write = [&](int g, float2 (&a)[4][2], float2 (&w)[4][2], uint2 (&cr)[4]) {
                 const float4 d01 = pp[(2 * g) * CH];   // (Delta, Delta*x or x) of tokens 4g, 4g+1
                 const float4 d23 = pp[(2 * g + 1) * CH];
                 const float dl[4] = {d01.x, d01.z, d23.x, d23.z};
                 const float dx[4] = {d01.y, d01.w, d23.y, d23.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 bq = *reinterpret_cast<const float4 *>(Bf + (4 * g + u) * NP + 4 * q);
-                    const float2 bb[2] = {f2(bq.x, bq.y), f2(bq.z, bq.w)};
+                    float2 bb[2];
+                    bquad(4 * g + u, bb, cr[u]);
                     const float2 dl2 = f2(dl[u], dl[u]);
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
@@ -391,12 +457,12 @@ scan_fwd_kernel(const ScanArgs p) {
                     }
                 }
             };
-            auto recur_read = [&](int g, const float2 (&a)[4][2], const float2 (&w)[4][2]) {
+            auto recur_read = [&](int g, const float2 (&a)[4][2], const float2 (&w)[4][2], const uint2 (&cr)[4]) {
                 float out[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 cq = *reinterpret_cast<const float4 *>(Cf + (4 * g + u) * NP + 4 * q);
-                    const float2 cc2[2] = {f2(cq.x, cq.y), f2(cq.z, cq.w)};
+                    float2 cc2[2];
+                    cquad(4 * g + u, cr[u], cc2);
                     float2 acc = f2(0.f, 0.f);
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
@@ -410,17 +476,21 @@ scan_fwd_kernel(const ScanArgs p) {
             // decays and writes of the next 4 tokens are computed before the recurrence
             // of the current 4, so the SFU work overlaps the FFMA chain
             float2 a0[4][2], w0[4][2];
-            decay_write(0, a0, w0);
+            uint2 c0[4];
+            decay_write(0, a0, w0, c0);
 #pragma unroll
             for (int g = 0; g < T / 4; ++g) {
                 float2 a1[4][2], w1[4][2];
-                if (g + 1 < T / 4) decay_write(g + 1, a1, w1);
-                recur_read(g, a0, w0);
+                uint2 c1[4];
+                if (g + 1 < T / 4) decay_write(g + 1, a1, w1, c1);
+                recur_read(g, a0, w0, c0);
                 if (g + 1 < T / 4) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
+                    for (int u = 0; u < 4; ++u) {
+                        c0[u] = c1[u];
 #pragma unroll
                         for (int k = 0; k < 2; ++k) { a0[u][k] = a1[u][k]; w0[u][k] = w1[u][k]; }
+                    }
                 }
             }
         }

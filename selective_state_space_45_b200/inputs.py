@@ -17,6 +17,7 @@ tiny           1       64         8        4    fp32
 mamba130m      8       2048       1536     16   bf16 (A, D, bias, state fp32)
 mamba2p8b      4       4096       5120     16   bf16
 long1m         1       1048576    1536     16   bf16
+long1m_slow    1       1048576    1536     16   bf16, A[d, n] = -exp(U[-5, 0]): slow decays
 decode         256     1 x 64     5120     16   bf16 tokens, fp32 state
 decode4        256     4 x 16     5120     16   as decode, 4 tokens per call
 bwd130m        8       2048       1536     16   bf16 inputs, dy and gradients (backward)
@@ -30,7 +31,9 @@ Draw order (one generator seeded once): x, delta_raw, z, B, C, D, dt.
   x, z ~ N(0, 1);  delta_raw = 0.5 * N(0, 1);  B, C ~ N(0, 1) per (b, t, n);
   D ~ N(0, 1);  dt ~ U[1e-3, 1e-1] per channel (log-uniform on that range for the
   2.8b shape);  delta_bias = log(expm1(dt)), evaluated in fp64 and stored fp32, so
-  that softplus(delta_bias) = dt;  A[d, n] = -(n + 1).
+  that softplus(delta_bias) = dt;  A[d, n] = -(n + 1), or for long1m_slow
+  A[d, n] = -exp(U[-5, 0]) drawn last (|A| between 0.0067 and 1: states that remember
+  for up to ~10^5 tokens, the hardest case for cutting a sequence into segments).
 The decode workload draws an N(0, 1) fp32 state and, per token, a positive step
 delta = dt * exp(0.5 * N(0, 1)) (the step is an input of the decode call, already
 positive), with x, z, B, C as above.
@@ -49,6 +52,8 @@ CONFIGS = {
                       dt_dist="loguniform"),
     "long1m": dict(batch=1, seqlen=1 << 20, dim=1536, dstate=16, dtype=torch.bfloat16,
                    dt_dist="uniform"),
+    "long1m_slow": dict(batch=1, seqlen=1 << 20, dim=1536, dstate=16, dtype=torch.bfloat16,
+                        dt_dist="uniform", a_dist="slow"),
     "decode": dict(batch=256, steps=64, dim=5120, dstate=16, dtype=torch.bfloat16,
                    dt_dist="uniform"),
     # the decode workload with 4 tokens per call on the carried state (speculative decoding)
@@ -84,7 +89,7 @@ def _draw_dt(n, dist, g, device):
 
 
 def make_scan_inputs(batch, dim, seqlen, dstate, dtype=torch.float32, device="cpu", seed=0,
-                     dt_dist="uniform"):
+                     dt_dist="uniform", a_dist="index"):
     """Inputs of one selective-scan call, as a dict of tensors on ``device``.
 
     Keys: x, delta, z ([batch, dim, seqlen], ``dtype``); B, C ([batch, seqlen, dstate],
@@ -108,7 +113,13 @@ def make_scan_inputs(batch, dim, seqlen, dstate, dtype=torch.float32, device="cp
     D = torch.randn(dim, generator=g, device=device, dtype=f32)
     dt = _draw_dt(dim, dt_dist, g, device)
     delta_bias = torch.log(torch.expm1(dt)).to(f32)
-    A = -torch.arange(1, dstate + 1, device=device, dtype=f32).repeat(dim, 1).contiguous()
+    if a_dist == "index":
+        A = -torch.arange(1, dstate + 1, device=device, dtype=f32).repeat(dim, 1).contiguous()
+    elif a_dist == "slow":
+        u = torch.rand(dim, dstate, generator=g, device=device, dtype=f32)
+        A = -torch.exp(-5.0 * u)
+    else:
+        raise ValueError("unknown A distribution %r" % (a_dist,))
     return dict(x=x, delta=delta, z=z, B=B, C=C, A=A, D=D, delta_bias=delta_bias)
 
 
@@ -157,7 +168,8 @@ def make_config_inputs(name, device="cpu", seed=0):
         return make_decode_inputs(c["batch"], c["dim"], c["dstate"], c["steps"], c["dtype"],
                                   device=device, seed=seed)
     return make_scan_inputs(c["batch"], c["dim"], c["seqlen"], c["dstate"], c["dtype"],
-                            device=device, seed=seed, dt_dist=c["dt_dist"])
+                            device=device, seed=seed, dt_dist=c["dt_dist"],
+                            a_dist=c.get("a_dist", "index"))
 
 
 def make_decode_inputs(batch, dim, dstate, steps, dtype=torch.bfloat16, device="cpu", seed=0,

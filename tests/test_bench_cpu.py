@@ -148,7 +148,9 @@ def test_ssd_counts():
     c = bench.ssd_counts(8, 2048, 24, 64, 128, 2, 2)
     toks = 8 * 2048 * 24
     assert c["bytes"] == toks * (64 * 2 + 2 * 128 * 2 + 4 + 64 * 2)
-    assert c["flops"] == 8 * 24 * 32 * 2 * (64 * 64 * 128 + 64 * 64 * 64 + 2 * 64 * 128 * 64)
+    # 16 chunks of 128 tokens per (sequence, head): scores Q x Q x N, masked scores times x
+    # Q x Q x P, and the two state products Q x N x P
+    assert c["flops"] == 8 * 24 * 16 * 2 * (128 * 128 * 128 + 128 * 128 * 64 + 2 * 128 * 128 * 64)
     assert c["tokch"] == toks * 64
     r = bench.oracle_rate("ssd130m", threads=2, budget_s=0.1)
     assert r["value"] > 0

@@ -47,5 +47,10 @@ def test_mamba2p8b_shape_sampled(cuda_lib):
 
 
 def test_long_context_sampled(cuda_lib):
-    # one sequence of 2^20 tokens: the kernel splits every tile over stitched sub-chunks
+    # one sequence of 2^20 tokens, cut into segments scanned in parallel from their carries
     _check_sampled(cuda_lib, "long1m", 6, out_dtypes=(torch.bfloat16,))
+
+
+def test_long_context_slow_decays_sampled(cuda_lib):
+    # the same length with |A| down to 0.0067: a segment's carry outlives the segment
+    _check_sampled(cuda_lib, "long1m_slow", 6, out_dtypes=(torch.bfloat16,))

@@ -33,12 +33,14 @@ def assert_ssd_close(gpu, ref, what):
     return rel_l2, norm_max
 
 
-CASES = [  # batch, L, heads, headdim, dstate
-    (1, 150, 3, 64, 128),     # three chunks, the last ragged
-    (2, 256, 4, 64, 64),
-    (1, 100, 2, 32, 128),
-    (2, 64, 3, 32, 64),       # exactly one chunk
+CASES = [  # batch, L, heads, headdim, dstate (chunks of 128 tokens)
+    (1, 150, 3, 64, 128),     # two chunks, the last ragged
+    (2, 256, 4, 64, 64),      # exactly two chunks
+    (1, 100, 2, 32, 128),     # one ragged chunk
+    (2, 128, 3, 32, 64),      # exactly one chunk
     (1, 7, 2, 64, 128),       # shorter than a chunk
+    (2, 421, 2, 64, 128),     # four chunks, more CTAs than one
+    (1, 300, 5, 32, 64),
 ]
 
 
@@ -51,6 +53,7 @@ def test_ssd_parity(cuda_lib, batch, L, heads, P, N, out_dtype):
     yr, hr = oracle.ssd_loop(inp["x"], inp["a"], inp["B"], inp["C"])
     assert_ssd_close(y, yr, "y")
     assert_ssd_close(hN, hr, "final state")
+    assert cuda_lib.ssm_device_timeouts() == 0
 
 
 def test_ssd_from_a_start_state_and_resume(cuda_lib):
@@ -105,3 +108,4 @@ def test_ssd130m_sampled_heads(cuda_lib):
         yr, hr = oracle.ssd_loop(sl["x"], sl["a"], sl["B"], sl["C"])
         assert_ssd_close(y[b:b + 1, :, h:h + 1], yr, "y (b=%d, h=%d)" % (b, h))
         assert_ssd_close(hN[b:b + 1, h:h + 1], hr, "final state (b=%d, h=%d)" % (b, h))
+    assert cuda_lib.ssm_device_timeouts() == 0
