@@ -81,11 +81,14 @@ int plan_scan(ssm::ScanArgs &a, long long &cgroups) {
     a.groups_per_seq = int(groups);
     cgroups = groups * a.batch;
     const size_t smem = Cfg::SMEM_BYTES;
-    if (smem > 48 * 1024) {   // opt in to large shared memory for both kernel variants
-        if (cudaFuncSetAttribute(scan_kernel<Cfg, false, ZOH>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(scan_kernel<Cfg, true, ZOH>(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(smem)) != cudaSuccess)
+    // both kernel variants: large shared memory where needed, and the whole unified L1 /
+    // shared array given to shared memory so that every resident CTA the registers allow fits
+    for (auto k : {scan_kernel<Cfg, false, ZOH>(), scan_kernel<Cfg, true, ZOH>()}) {
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        if (cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
             return SSM_ERR_CUDA;
     }
     const long long slots = resident_slots(scan_kernel<Cfg, true, ZOH>(), Cfg::NTHREADS, smem);
@@ -122,9 +125,12 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
 }
 
 // Tile shape per padded state width: 32-token tiles; 32 channels per CTA (64 at N <= 4).
+// bf16 inputs at N = 16: a 2-stage ring, 42 KB of shared memory and at most 96 registers,
+// so 5 CTAs share an SM (740 on the chip: 4 sequences x 5120 channels run in one wave).
 template <int NP, typename Tin, typename Tout, bool VEC>
 struct ScanConfig {
-    using C16 = ssm::ScanCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>;
+    using C16 = std::conditional_t<sizeof(Tin) == 2, ssm::ScanCfg<16, 1, 32, 2, Tin, Tout, VEC, 5>,
+                                   ssm::ScanCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>>;
     using C8 = ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>;
     using C4 = ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>;
     using type = std::conditional_t<NP == 16, C16, std::conditional_t<NP == 8, C8, C4>>;

@@ -24,8 +24,8 @@
 //   * The decays and writes of the next 4 tokens are computed before the recurrence of
 //     the current 4, so SFU work overlaps the FFMA chain.
 //   * x, delta, z, B, C are staged by a cp.async ring of NSTAGE tiles (16-byte copies)
-//     when every row is 16-byte aligned, else by guarded scalar loads; y is staged in
-//     shared memory and stored as 16-byte rows.
+//     when every row is 16-byte aligned, else by guarded scalar loads; y leaves as 16-byte
+//     stores of 8 tokens straight from the epilogue's registers.
 //
 // Long sequences with few channels are split into segments scanned by different CTAs.
 // The scan is linear in its carry, so a segment's end state from a zero start is
@@ -83,13 +83,20 @@ struct ScanCfg {
     static constexpr int NWARP = Q * CG;
     static constexpr int NTHREADS = 32 * NWARP;
     static constexpr int EIN = 16 / sizeof(Tin);
-    static constexpr int EOUT = 16 / sizeof(Tout);
     static constexpr int T8 = T / 8;                  // 8-token chunks per tile row
     static constexpr int NTASK = CH * T8;             // per-(t, d) tasks per tile
     static constexpr int TASKS_PER_THREAD = (NTASK + NTHREADS - 1) / NTHREADS;
-    static constexpr int RAW_ROW = T + EIN;           // row stride 16 B past a multiple of
-    static constexpr int Y_ROW = T + EOUT;            // 16 B: conflict-free 16 B column reads
-    static constexpr int YP_ROW = T + 4;              // floats
+    // staged x, delta, z rows: CPR 16-byte chunks per channel, RPL rows to a 128-byte line;
+    // chunk j of row cc sits in slot j XOR ((cc / RPL) mod CPR), so 16-byte reads of one
+    // chunk column across 8 consecutive channels hit distinct banks without padding
+    static constexpr int CPR = T / EIN;
+    static constexpr int RPL = CPR >= 8 ? 1 : 8 / CPR;
+    static_assert((CPR & (CPR - 1)) == 0 && T % 8 == 0, "staged rows: a power of two of 16-byte chunks");
+    static constexpr int RAW_ROW = T;
+    __host__ __device__ static constexpr int raw_at(int cc, int t) {
+        return cc * RAW_ROW + (((t / EIN) ^ ((cc / RPL) & (CPR - 1))) * EIN) + t % EIN;
+    }
+    static constexpr int YP_SLOTS = T / 4;            // float4 slots of a partial-sum row
     static_assert(T % 8 == 0, "tile must hold whole 8-token chunks");
     static_assert(NTASK % NTHREADS == 0, "tasks must divide evenly");
 
@@ -111,12 +118,16 @@ struct ScanCfg {
     static constexpr size_t CF_BYTES = BCPACK ? 0 : al(size_t(T) * NP * sizeof(float));
     static constexpr size_t OFF_BF = OFF_PREP + al(size_t(T / 2) * CH * sizeof(float4));
     static constexpr size_t OFF_CF = OFF_BF + BF_BYTES;
+    // quad partial sums of the readout [Q][CH][T], slot g of a row stored at g XOR (channel
+    // mod 8): the recurrence's 16-byte writes (lanes over channels) and the epilogue's reads
+    // are conflict free without padding
     static constexpr size_t OFF_YP = OFF_CF + CF_BYTES;
-    static constexpr size_t OFF_Y = OFF_YP + al(size_t(Q) * CH * YP_ROW * sizeof(float));
-    static constexpr size_t SMEM_BYTES = OFF_Y + al(size_t(CH) * Y_ROW * sizeof(Tout));
+    static constexpr size_t SMEM_BYTES = OFF_YP + al(size_t(Q) * CH * T * sizeof(float));
+    static_assert(YP_SLOTS == 8, "the XOR swizzle of the partial rows assumes 8 slots");
 };
 
-// Views of one ring stage: x, delta, z rows [CH][RAW_ROW]; B, C as [T][N] contiguous.
+// Views of one ring stage: x, delta, z as [CH][T] in swizzled 16-byte chunks (raw_at); B, C
+// as [T][N] contiguous.
 template <class Cfg> struct Stage {
     typename Cfg::Tin *xs, *ds, *zs, *bs, *cs;
     __device__ __forceinline__ Stage(unsigned char *smem, int s) {
@@ -128,6 +139,21 @@ template <class Cfg> struct Stage {
         cs = reinterpret_cast<typename Cfg::Tin *>(base + 3 * Cfg::RAW_ARR + Cfg::RAW_BC);
     }
 };
+
+// Tokens 8 t8 .. 8 t8 + 7 of channel cc of a staged x, delta or z array, as fp32.
+template <class Cfg>
+__device__ __forceinline__ void stage_row8(const typename Cfg::Tin *arr, int cc, int t8, float (&v)[8]) {
+    using Tin = typename Cfg::Tin;
+    if constexpr (Cfg::EIN == 8) {
+        load8<Tin>(arr + Cfg::raw_at(cc, 8 * t8), v);
+    } else {
+        float lo[4], hi[4];
+        loadn<4, Tin>(arr + Cfg::raw_at(cc, 8 * t8), lo);
+        loadn<4, Tin>(arr + Cfg::raw_at(cc, 8 * t8 + 4), hi);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) { v[u] = lo[u]; v[4 + u] = hi[u]; }
+    }
+}
 
 // Stage tile [t0, t0 + T) of x, delta, z (rows of nch channels) and of B, C into ring stage
 // st, with every index split by compile-time divisors; thread `me` of the NT staging
@@ -157,7 +183,7 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
             const int cc = rem / CPR, q = rem % CPR;
             if (i < ROWC && a < narr && cc < nch && t0 + q * EIN < L) {
                 const Tin *src = (a == 0 ? gx : a == 1 ? gd : gz) + size_t(cc) * L + t0 + q * EIN;
-                Tin *dst = (a == 0 ? s.xs : a == 1 ? s.ds : s.zs) + cc * Cfg::RAW_ROW + q * EIN;
+                Tin *dst = (a == 0 ? s.xs : a == 1 ? s.ds : s.zs) + Cfg::raw_at(cc, q * EIN);
                 cp_async_16(dst, src);
             }
         }
@@ -189,7 +215,7 @@ __device__ __forceinline__ void load_tile(const ScanArgs &p, unsigned char *smem
             const int cc = rem / T, tt = rem % T;
             if (i < NEL && a < narr && cc < nch && t0 + tt < L) {
                 const Tin *src = (a == 0 ? gx : a == 1 ? gd : gz) + size_t(cc) * L + t0 + tt;
-                Tin *dst = (a == 0 ? s.xs : a == 1 ? s.ds : s.zs) + cc * Cfg::RAW_ROW + tt;
+                Tin *dst = (a == 0 ? s.xs : a == 1 ? s.ds : s.zs) + Cfg::raw_at(cc, tt);
                 *dst = *src;
             }
         }
@@ -235,7 +261,6 @@ scan_fwd_kernel(const ScanArgs p) {
     float *Bf = reinterpret_cast<float *>(smem + Cfg::OFF_BF);
     float *Cf = reinterpret_cast<float *>(smem + Cfg::OFF_CF);
     float *yp = reinterpret_cast<float *>(smem + Cfg::OFF_YP);
-    Tout *ys = reinterpret_cast<Tout *>(smem + Cfg::OFF_Y);
 
     // this lane's 4 states: A * log2(e)
     float A2[4];
@@ -309,8 +334,8 @@ scan_fwd_kernel(const ScanArgs p) {
             const int task = tid + k * NT;
             const int cc = task % CH, t8 = task / CH;
             float dr[8], xr[8];
-            load8<Tin>(sv.ds + cc * Cfg::RAW_ROW + 8 * t8, dr);
-            load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+            stage_row8<Cfg>(sv.ds, cc, t8, dr);
+            stage_row8<Cfg>(sv.xs, cc, t8, xr);
             const float bias = tbias[k];
             float o[16];
             if (cc < nch && t0 + 8 * t8 + 8 <= L) {          // whole chunk inside the data
@@ -397,7 +422,7 @@ scan_fwd_kernel(const ScanArgs p) {
         // ---- the recurrence: 4 states of one channel per lane, carried across tiles ----
         {
             const float4 *pp = prep + c;
-            float *ypr = yp + (q * CH + c) * Cfg::YP_ROW;
+            float4 *ypr = reinterpret_cast<float4 *>(yp) + (q * CH + c) * Cfg::YP_SLOTS;
             const uint4 *bcp = reinterpret_cast<const uint4 *>(Bf) + q;
             // the B and C quads of token t as fp32 pairs (0,1), (2,3)
             auto bquad = [&](int t, float2 (&bb)[2], uint2 &craw) {
@@ -471,7 +496,7 @@ scan_fwd_kernel(const ScanArgs p) {
                     }
                     out[u] = acc.x + acc.y;
                 }
-                *reinterpret_cast<float4 *>(ypr + 4 * g) = make_float4(out[0], out[1], out[2], out[3]);
+                ypr[g ^ (c & 7)] = make_float4(out[0], out[1], out[2], out[3]);
             };
             // decays and writes of the next 4 tokens are computed before the recurrence
             // of the current 4, so the SFU work overlaps the FFMA chain
@@ -496,61 +521,44 @@ scan_fwd_kernel(const ScanArgs p) {
         }
         __syncthreads();
 
-        // ---- epilogue: sum the quads, skip, gate, convert; stage y rows ----
+        // ---- epilogue: sum the quads, skip, gate, convert; 16-byte stores of y ----
+        Tout *gy = static_cast<Tout *>(p.y) + row0;
 #pragma unroll
         for (int k = 0; k < Cfg::TASKS_PER_THREAD; ++k) {
             const int task = tid + k * NT;
             const int cc = task % CH, t8 = task / CH;
-            float acc[8];
-            {
-                const float *src = yp + cc * Cfg::YP_ROW + 8 * t8;
-                const float4 a0 = *reinterpret_cast<const float4 *>(src);
-                const float4 a1 = *reinterpret_cast<const float4 *>(src + 4);
-                acc[0] = a0.x; acc[1] = a0.y; acc[2] = a0.z; acc[3] = a0.w;
-                acc[4] = a1.x; acc[5] = a1.y; acc[6] = a1.z; acc[7] = a1.w;
-            }
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int qq = 1; qq < Q; ++qq) {
-                const float *src = yp + (qq * CH + cc) * Cfg::YP_ROW + 8 * t8;
-                const float4 a0 = *reinterpret_cast<const float4 *>(src);
-                const float4 a1 = *reinterpret_cast<const float4 *>(src + 4);
+            for (int qq = 0; qq < Q; ++qq) {
+                const float4 *row = reinterpret_cast<const float4 *>(yp) + (qq * CH + cc) * Cfg::YP_SLOTS;
+                const float4 a0 = row[(2 * t8) ^ (cc & 7)];
+                const float4 a1 = row[(2 * t8 + 1) ^ (cc & 7)];
                 acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
                 acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
             }
             float xr[8];
-            load8<Tin>(sv.xs + cc * Cfg::RAW_ROW + 8 * t8, xr);
+            stage_row8<Cfg>(sv.xs, cc, t8, xr);
             const float Dd = tD[k];
 #pragma unroll
             for (int u = 0; u < 8; ++u) acc[u] = fmaf(Dd, xr[u], acc[u]);
             if (p.z != nullptr) {
                 float zr[8];
-                load8<Tin>(sv.zs + cc * Cfg::RAW_ROW + 8 * t8, zr);
+                stage_row8<Cfg>(sv.zs, cc, t8, zr);
 #pragma unroll
                 for (int u = 0; u < 8; ++u) acc[u] *= silu_f(zr[u]);
             }
-            store8<Tout>(ys + cc * Cfg::Y_ROW + 8 * t8, acc);
-        }
-        __syncthreads();
-
-        // ---- write y rows back (coalesced) ----
-        Tout *gy = static_cast<Tout *>(p.y) + row0;
-        if constexpr (Cfg::VEC) {
-            constexpr int CPR = T / Cfg::EOUT;
-#pragma unroll
-            for (int k = 0; k < (CH * CPR + NT - 1) / NT; ++k) {
-                const int i = tid + k * NT;
-                const int cc = i / CPR, qq = i % CPR;
-                const int tg = t0 + qq * Cfg::EOUT;
-                if (i < CH * CPR && cc < nch && tg < L)
-                    *reinterpret_cast<uint4 *>(gy + size_t(cc) * L + tg) =
-                        *reinterpret_cast<const uint4 *>(ys + cc * Cfg::Y_ROW + qq * Cfg::EOUT);
-            }
-        } else {
-            for (int i = tid; i < nch * T; i += NT) {
-                const int cc = i / T, tt = i % T;
-                if (t0 + tt < L) gy[size_t(cc) * L + t0 + tt] = ys[cc * Cfg::Y_ROW + tt];
+            const int tg = t0 + 8 * t8;
+            if (cc < nch) {
+                if (Cfg::VEC && tg + 8 <= L) {
+                    store_run<8>(gy + size_t(cc) * L + tg, acc);
+                } else {
+                    for (int u = 0; u < 8; ++u)
+                        if (tg + u < L) gy[size_t(cc) * L + tg + u] = from_f32<Tout>(acc[u]);
+                }
             }
         }
+        // the next tile's first barrier orders these reads before the partials and the
+        // stage are written again
     }
     cp_async_wait<0>();
     h[0] = hp[0].x; h[1] = hp[0].y; h[2] = hp[1].x; h[3] = hp[1].y;
