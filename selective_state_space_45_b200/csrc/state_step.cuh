@@ -45,6 +45,24 @@ template <> __device__ __forceinline__ void load4_nc<__nv_bfloat16>(const __nv_b
     v[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
+// One token on a quad of 4 states of one channel, as packed FP32 pairs (0,1), (2,3):
+// h_n <- 2^(Delta A2_n) h_n + (Delta x) B_n with A2 = A log2(e), and the quad's share of
+// the readout, (C_0 h_0 + C_2 h_2) + (C_1 h_1 + C_3 h_3).  Both decode kernels update and
+// read out every quad through this one function, so they agree bit for bit.
+__device__ __forceinline__ float quad_step(float (&h)[4], const float (&A2)[4], float dl, float dx,
+                                           const float (&b)[4], const float (&c)[4]) {
+    const float2 dl2 = f2(dl, dl), dx2 = f2(dx, dx);
+    float2 acc = f2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const float2 a = ex2_pair(fmul2(dl2, f2(A2[2 * k], A2[2 * k + 1])));
+        const float2 hk = ffma2(a, f2(h[2 * k], h[2 * k + 1]), fmul2(dx2, f2(b[2 * k], b[2 * k + 1])));
+        h[2 * k] = hk.x; h[2 * k + 1] = hk.y;
+        acc = ffma2(f2(c[2 * k], c[2 * k + 1]), hk, acc);
+    }
+    return acc.x + acc.y;
+}
+
 // One thread = J channel-quads (4 states each).  Quad j of a thread is global quad
 // gq = (blockIdx.x * J + j) * blockDim.x + threadIdx.x, so each of the J accesses of a
 // warp covers 32 consecutive quads (512 contiguous bytes of state at N = 16).  Every load
@@ -59,7 +77,7 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
     long long chs[J];
     int rs[J], ds[J];
     bool act[J];
-    float h[J][4], a4[J][4], bb[J][4], cc[J][4], dl[J], xv[J], zv[J], Dv[J];
+    float h[J][4], a4[J][4], bb[J][4], cc[J][4], dl[J], xv[J], zv[J], Dv[J];   // a4: A log2(e)
 #pragma unroll
     for (int j = 0; j < J; ++j) {
         const long long g = ((long long)blockIdx.x * J + j) * blockDim.x + threadIdx.x;
@@ -80,7 +98,8 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
                 const float4 hv = *reinterpret_cast<const float4 *>(hp);
                 const float4 av = __ldg(reinterpret_cast<const float4 *>(Ap));
                 h[j][0] = hv.x; h[j][1] = hv.y; h[j][2] = hv.z; h[j][3] = hv.w;
-                a4[j][0] = av.x; a4[j][1] = av.y; a4[j][2] = av.z; a4[j][3] = av.w;
+                a4[j][0] = av.x * kLog2e; a4[j][1] = av.y * kLog2e;
+                a4[j][2] = av.z * kLog2e; a4[j][3] = av.w * kLog2e;
                 load4_nc<Tin>(Bb, bb[j]);
                 load4_nc<Tin>(Cb, cc[j]);
             } else {
@@ -92,7 +111,7 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
             for (int s = 0; s < 4; ++s) {
                 const bool ok = act[j] && n0 + s < N;
                 h[j][s] = ok ? hp[s] : 0.f;
-                a4[j][s] = ok ? Ap[s] : 0.f;
+                a4[j][s] = ok ? Ap[s] * kLog2e : 0.f;
                 bb[j][s] = ok ? to_f32(Bb[s]) : 0.f;
                 cc[j][s] = ok ? to_f32(Cb[s]) : 0.f;
             }
@@ -104,13 +123,7 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
     }
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-        const float dx = dl[j] * xv[j];
-        float acc = 0.f;
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            h[j][s] = fmaf(ex2_approx(dl[j] * a4[j][s] * kLog2e), h[j][s], dx * bb[j][s]);
-            acc = fmaf(cc[j][s], h[j][s], acc);
-        }
+        float acc = quad_step(h[j], a4[j], dl[j], dl[j] * xv[j], bb[j], cc[j]);
         const int n0 = 4 * rs[j];
         float *hp = p.state + (size_t)chs[j] * N + n0;
         if constexpr (VEC4) {
@@ -132,19 +145,23 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
 }
 
 // Several decode tokens per call (ssm_state_step_multi: speculative or chunked decoding),
-// one channel per thread with all of its states in registers: the state (and A) is read
-// once, carried through the ntok tokens in registers and written once, so the state
-// traffic is that of one step whatever ntok is.  A block holds kStepThreads consecutive
-// channels of one sequence (blockIdx.x = b * dblocks + channel block).  Per round of up to
-// kStepsRound tokens every thread issues the loads of its (x, Delta, z) for all the
-// round's tokens at once, and the block stages the sequence's B and C rows of the round in
-// shared memory (padded to NP with zeros), read back as 16-byte broadcasts.
+// one channel per thread with all of its states in registers: the state is read once,
+// carried through the ntok tokens in registers and written once, so the state traffic is
+// that of one step whatever ntok is.
+//
+// A block holds kStepThreads consecutive channels and walks the sequences b = slice,
+// slice + slices, ... (blockIdx.x = slice * dblocks + channel block), so A and D stay in
+// registers for all of them, and the next sequence's state and first tokens are loaded
+// into registers while the current one is computed, so loads stay in flight through the
+// whole kernel instead of only at its start.  Per round of up to kStepsRound tokens the
+// block stages the sequence's B and C rows in shared memory (padded to NP with zeros),
+// read back as 16-byte broadcasts.
 //
 // Per token the arithmetic is the one-token kernel's, in the same order: each quad of 4
 // states is updated and read out as one thread of state_step_kernel does, and the quad
 // shares are summed in the order the xor-butterfly over the G lanes of a channel gives
 // lane 0.  ntok chained one-token calls therefore give bit-identical states and outputs.
-constexpr int kStepThreads = 256;
+constexpr int kStepThreads = 128;
 constexpr int kStepsRound = 4;
 
 // The readout of a channel from its G = NP / 4 quad shares, in the xor-butterfly order
@@ -155,104 +172,144 @@ template <int G> __device__ __forceinline__ float quad_sum(const float (&s)[G]) 
     else return (s[0] + s[2]) + (s[1] + s[3]);
 }
 
+#ifndef SSM_STEPS_MINB
+#define SSM_STEPS_MINB 4     // resident blocks per SM the registers target
+#endif
 template <int NP, typename Tin, typename Tout, bool VEC4>
-__global__ void __launch_bounds__(kStepThreads, 3) state_steps_kernel(const StepArgs p, int dblocks) {
-    constexpr int G = NP / 4;
-    static_assert(2 * kStepsRound * NP <= kStepThreads, "one thread per staged B/C value");
-    __shared__ __align__(16) float sbc[2][kStepsRound][NP];
-    const int b = int(blockIdx.x / unsigned(dblocks));
-    const int d = (int(blockIdx.x) - b * dblocks) * kStepThreads + int(threadIdx.x);
+__global__ void __launch_bounds__(kStepThreads, SSM_STEPS_MINB) state_steps_kernel(const StepArgs p, int dblocks) {
+    constexpr int G = NP / 4, R = kStepsRound;
+    static_assert(2 * R * NP <= kStepThreads, "one thread per staged B/C value");
+    __shared__ __align__(16) float sbc[2][R][NP];
+    const int cb = int(blockIdx.x % unsigned(dblocks));
+    const int slice = int(blockIdx.x / unsigned(dblocks));
+    const int slices = int(gridDim.x / unsigned(dblocks));
+    const int d = cb * kStepThreads + int(threadIdx.x);
     const bool act = d < p.dim;
-    const int N = p.dstate;
+    const int N = p.dstate, ntok = p.ntok;
     const size_t chans = size_t(p.batch) * p.dim;
-    const size_t ch = size_t(b) * p.dim + (act ? d : 0);
-
-    float *hs = p.state + ch * N;
-    const float *As = p.A + size_t(act ? d : 0) * N;
-    float h[NP], a[NP];
-    if constexpr (VEC4) {                            // rows of whole 16-byte quads
-#pragma unroll
-        for (int q = 0; q < G; ++q) {
-            float4 hv = make_float4(0.f, 0.f, 0.f, 0.f), av = hv;
-            if (act && 4 * q < N) {
-                hv = *reinterpret_cast<const float4 *>(hs + 4 * q);
-                av = __ldg(reinterpret_cast<const float4 *>(As + 4 * q));
-            }
-            h[4 * q] = hv.x; h[4 * q + 1] = hv.y; h[4 * q + 2] = hv.z; h[4 * q + 3] = hv.w;
-            a[4 * q] = av.x; a[4 * q + 1] = av.y; a[4 * q + 2] = av.z; a[4 * q + 3] = av.w;
-        }
-    } else {
-#pragma unroll
-        for (int n = 0; n < NP; ++n) {
-            const bool ok = act && n < N;
-            h[n] = ok ? hs[n] : 0.f;
-            a[n] = ok ? As[n] : 0.f;
-        }
-    }
-    const float Dv = (p.D != nullptr && act) ? p.D[d] : 0.f;
     const Tin *gx = static_cast<const Tin *>(p.x);
     const Tin *gd = static_cast<const Tin *>(p.delta);
     const Tin *gz = static_cast<const Tin *>(p.z);
     const Tin *gB = static_cast<const Tin *>(p.B);
     const Tin *gC = static_cast<const Tin *>(p.C);
     Tout *gy = static_cast<Tout *>(p.y);
-    for (int t0 = 0; t0 < p.ntok; t0 += kStepsRound) {
-        const int nt = min(kStepsRound, p.ntok - t0);
-        float xr[kStepsRound], dr[kStepsRound], zr[kStepsRound];
-#pragma unroll
-        for (int tt = 0; tt < kStepsRound; ++tt) {
-            const bool ok = act && tt < nt;
-            const size_t idx = size_t(t0 + tt) * chans + ch;
-            xr[tt] = ok ? to_f32(gx[idx]) : 0.f;
-            dr[tt] = ok ? to_f32(gd[idx]) : 0.f;
-            zr[tt] = (ok && gz != nullptr) ? to_f32(gz[idx]) : 0.f;
-        }
-        __syncthreads();                      // the previous round's reads are done
-        {
-            const int i = threadIdx.x;
-            const int which = i / (kStepsRound * NP);
-            const int tt = (i / NP) % kStepsRound, n = i % NP;
-            if (i < 2 * kStepsRound * NP && tt < nt) {
-                const size_t idx = (size_t(t0 + tt) * p.batch + b) * N + n;
-                sbc[which][tt][n] = n < N ? to_f32((which ? gC : gB)[idx]) : 0.f;
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int tt = 0; tt < kStepsRound; ++tt) {
-            if (tt >= nt) break;
-            const float dl = dr[tt], xv = xr[tt];
-            const float dx = dl * xv;
-            float sq[G];
-#pragma unroll
-            for (int q = 0; q < G; ++q) {
-                const float4 bq = *reinterpret_cast<const float4 *>(&sbc[0][tt][4 * q]);
-                const float4 cq = *reinterpret_cast<const float4 *>(&sbc[1][tt][4 * q]);
-                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-                const float cc[4] = {cq.x, cq.y, cq.z, cq.w};
-                float acc = 0.f;
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const int n = 4 * q + s;
-                    h[n] = fmaf(ex2_approx(dl * a[n] * kLog2e), h[n], dx * bb[s]);
-                    acc = fmaf(cc[s], h[n], acc);
-                }
-                sq[q] = acc;
-            }
-            float yv = fmaf(Dv, xv, quad_sum<G>(sq));
-            if (gz != nullptr) yv *= silu_f(zr[tt]);
-            if (act) gy[size_t(t0 + tt) * chans + ch] = from_f32<Tout>(yv);
-        }
-    }
+
+    // A log2(e) (and D) of this channel, for every sequence of the block
+    const float *As = p.A + size_t(act ? d : 0) * N;
+    float a[G][4];
     if constexpr (VEC4) {
 #pragma unroll
-        for (int q = 0; q < G; ++q)
-            if (act && 4 * q < N)
-                *reinterpret_cast<float4 *>(hs + 4 * q) = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+        for (int q = 0; q < G; ++q) {
+            float4 av = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (act && 4 * q < N) av = __ldg(reinterpret_cast<const float4 *>(As + 4 * q));
+            a[q][0] = av.x * kLog2e; a[q][1] = av.y * kLog2e; a[q][2] = av.z * kLog2e; a[q][3] = av.w * kLog2e;
+        }
     } else {
 #pragma unroll
-        for (int n = 0; n < NP; ++n)
-            if (act && n < N) hs[n] = h[n];
+        for (int n = 0; n < NP; ++n) a[n / 4][n % 4] = (act && n < N) ? As[n] * kLog2e : 0.f;
+    }
+    const float Dv = (p.D != nullptr && act) ? p.D[d] : 0.f;
+
+    auto state_row = [&](int b) { return p.state + (size_t(b) * p.dim + (act ? d : 0)) * N; };
+    auto load_state = [&](int b, float (&hv)[G][4]) {
+        const float *hs = state_row(b);
+        if constexpr (VEC4) {
+#pragma unroll
+            for (int q = 0; q < G; ++q) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (act && 4 * q < N) v = *reinterpret_cast<const float4 *>(hs + 4 * q);
+                hv[q][0] = v.x; hv[q][1] = v.y; hv[q][2] = v.z; hv[q][3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int n = 0; n < NP; ++n) hv[n / 4][n % 4] = (act && n < N) ? hs[n] : 0.f;
+        }
+    };
+    // the round's token inputs of sequence b (raw, converted when used)
+    auto load_tokens = [&](int b, int t0, Tin (&xr)[R], Tin (&dr)[R], Tin (&zr)[R]) {
+        const size_t ch = size_t(b) * p.dim + (act ? d : 0);
+#pragma unroll
+        for (int tt = 0; tt < R; ++tt) {
+            const bool ok = act && t0 + tt < ntok;
+            const size_t idx = size_t(t0 + tt) * chans + ch;
+            xr[tt] = ok ? gx[idx] : Tin(0.f);
+            dr[tt] = ok ? gd[idx] : Tin(0.f);
+            zr[tt] = (ok && gz != nullptr) ? gz[idx] : Tin(0.f);
+        }
+    };
+    // this thread's staged B/C value of the round (threads 0 .. 2 R NP - 1)
+    auto load_bc = [&](int b, int t0) {
+        const int i = threadIdx.x;
+        const int which = i / (R * NP);
+        const int tt = (i / NP) % R, n = i % NP;
+        float v = 0.f;
+        if (i < 2 * R * NP && t0 + tt < ntok && n < N)
+            v = to_f32((which ? gC : gB)[(size_t(t0 + tt) * p.batch + b) * N + n]);
+        return v;
+    };
+
+    // the first sequence's state and first round, then one sequence ahead
+    float hn[G][4];
+    Tin xn[R], dn[R], zn[R];
+    float bcn = 0.f;
+    if (slice < p.batch) {
+        load_state(slice, hn);
+        load_tokens(slice, 0, xn, dn, zn);
+        bcn = load_bc(slice, 0);
+    }
+    for (int b = slice; b < p.batch; b += slices) {
+        float h[G][4];
+#pragma unroll
+        for (int n = 0; n < NP; ++n) h[n / 4][n % 4] = hn[n / 4][n % 4];
+        Tin xq[R], dq[R], zq[R];
+#pragma unroll
+        for (int tt = 0; tt < R; ++tt) { xq[tt] = xn[tt]; dq[tt] = dn[tt]; zq[tt] = zn[tt]; }
+        float bcv = bcn;
+        if ((long long)b + slices < p.batch) {
+            load_state(b + slices, hn);
+            load_tokens(b + slices, 0, xn, dn, zn);
+            bcn = load_bc(b + slices, 0);
+        }
+        const size_t ch = size_t(b) * p.dim + (act ? d : 0);
+        for (int t0 = 0; t0 < ntok; t0 += R) {
+            const int nt = min(R, ntok - t0);
+            if (t0 > 0) {
+                load_tokens(b, t0, xq, dq, zq);
+                bcv = load_bc(b, t0);
+            }
+            __syncthreads();                      // the previous round's reads are done
+            if (threadIdx.x < 2 * R * NP) (&sbc[0][0][0])[threadIdx.x] = bcv;
+            __syncthreads();
+#pragma unroll
+            for (int tt = 0; tt < R; ++tt) {
+                if (tt >= nt) break;
+                const float dl = to_f32(dq[tt]), xv = to_f32(xq[tt]);
+                const float dx = dl * xv;
+                float sq[G];
+#pragma unroll
+                for (int q = 0; q < G; ++q) {
+                    const float4 bq = *reinterpret_cast<const float4 *>(&sbc[0][tt][4 * q]);
+                    const float4 cq = *reinterpret_cast<const float4 *>(&sbc[1][tt][4 * q]);
+                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+                    const float cc[4] = {cq.x, cq.y, cq.z, cq.w};
+                    sq[q] = quad_step(h[q], a[q], dl, dx, bb, cc);
+                }
+                float yv = fmaf(Dv, xv, quad_sum<G>(sq));
+                if (gz != nullptr) yv *= silu_f(to_f32(zq[tt]));
+                if (act) gy[size_t(t0 + tt) * chans + ch] = from_f32<Tout>(yv);
+            }
+        }
+        float *hs = state_row(b);
+        if constexpr (VEC4) {
+#pragma unroll
+            for (int q = 0; q < G; ++q)
+                if (act && 4 * q < N)
+                    *reinterpret_cast<float4 *>(hs + 4 * q) = make_float4(h[q][0], h[q][1], h[q][2], h[q][3]);
+        } else {
+#pragma unroll
+            for (int n = 0; n < NP; ++n)
+                if (act && n < N) hs[n] = h[n / 4][n % 4];
+        }
     }
 }
 

@@ -37,19 +37,32 @@ int launch_step(const ssm::StepArgs &a, cudaStream_t s) {
     return launch_step_np<16, Tin, Tout>(a, s);
 }
 
-// Several tokens: one channel per thread, kStepThreads consecutive channels of one
-// sequence per block.
+// Several tokens: one channel per thread, kStepThreads consecutive channels per block; the
+// blocks of a channel range share out the sequences, as many blocks in all as the GPU holds
+// at once (or one per (sequence, channel range) if that is fewer).
+template <int NP, typename Tin, typename Tout, bool VEC4>
+int launch_steps_vec(const ssm::StepArgs &a, long long dblocks, cudaStream_t s) {
+    const auto kernel = ssm::state_steps_kernel<NP, Tin, Tout, VEC4>;
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, ssm::kStepThreads, 0) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    const long long resident = std::max(1LL, (long long)sms * per_sm);
+    const long long slices = std::max(1LL, std::min<long long>(a.batch, resident / dblocks));
+    const long long blocks = dblocks * slices;
+    if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    kernel<<<unsigned(blocks), ssm::kStepThreads, 0, s>>>(a, int(dblocks));
+    return status_of(cudaGetLastError());
+}
+
 template <int NP, typename Tin, typename Tout>
 int launch_steps_np(const ssm::StepArgs &a, cudaStream_t s) {
     const long long dblocks = (a.dim + ssm::kStepThreads - 1) / ssm::kStepThreads;
-    const long long blocks = dblocks * a.batch;
-    if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
-    if (blocks == 0) return SSM_OK;
-    if (a.dstate % 4 == 0)
-        ssm::state_steps_kernel<NP, Tin, Tout, true><<<unsigned(blocks), ssm::kStepThreads, 0, s>>>(a, int(dblocks));
-    else
-        ssm::state_steps_kernel<NP, Tin, Tout, false><<<unsigned(blocks), ssm::kStepThreads, 0, s>>>(a, int(dblocks));
-    return status_of(cudaGetLastError());
+    if (dblocks == 0 || a.batch == 0) return SSM_OK;
+    if (dblocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+    return a.dstate % 4 == 0 ? launch_steps_vec<NP, Tin, Tout, true>(a, dblocks, s)
+                             : launch_steps_vec<NP, Tin, Tout, false>(a, dblocks, s);
 }
 
 template <typename Tin, typename Tout>

@@ -145,7 +145,8 @@ def test_multi_token_step_with_no_tokens_keeps_state(cuda_lib):
 
 @pytest.mark.parametrize("batch,dim,N", [(40, 1, 16), (9, 3, 4), (5, 70, 8)])
 def test_multi_token_step_small_dims_span_many_sequences(cuda_lib, batch, dim, N):
-    # a block's channels then cover several sequences, whose B, C are all staged
+    # channel ranges narrower than a block (most lanes idle), sequences shared out over the
+    # blocks, three rounds of staged B, C per sequence (the last one partial)
     ntok = 11
     inp = inputs.make_decode_inputs(batch, dim, N, ntok, torch.float32, device=DEV, seed=batch + dim)
     st = inp["state"].clone()
@@ -159,3 +160,32 @@ def test_multi_token_step_small_dims_span_many_sequences(cuda_lib, batch, dim, N
                             D=inp["D"], z=inp["z"][t])
         assert_parity(y[t], yr, torch.float32, torch.float32, what="y[%d]" % t)
     assert_parity(st, h, torch.float32, torch.float32, what="state")
+
+
+@pytest.mark.parametrize("ntok,N,din,dout", [(6, 16, torch.bfloat16, torch.bfloat16),
+                                             (9, 8, torch.float32, torch.float32)])
+def test_multi_token_step_blocks_walk_many_sequences(cuda_lib, ntok, N, din, dout):
+    # more sequences than the resident blocks of a channel range: each block walks several,
+    # loading the next one's state and first tokens while it computes the current one; the
+    # last channel range is ragged (3000 = 23 x 128 + 56)
+    batch, dim = 96, 3000
+    inp = inputs.make_decode_inputs(batch, dim, N, ntok, din, device=DEV, seed=ntok + N)
+    st_multi = inp["state"].clone()
+    y_multi = torch.empty(ntok, batch, dim, device=DEV, dtype=dout)
+    cuda_lib.ssm_state_step_multi(st_multi, inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"],
+                                  inp["D"], inp["z"], y_multi)
+    st_chain = inp["state"].clone()
+    for t in range(ntok):
+        y = torch.empty(batch, dim, device=DEV, dtype=dout)
+        cuda_lib.ssm_state_step(st_chain, inp["x"][t].clone(), inp["delta"][t].clone(), inp["A"],
+                                inp["B"][t].clone(), inp["C"][t].clone(), inp["D"],
+                                inp["z"][t].clone(), y)
+        torch.cuda.synchronize()
+        assert torch.equal(y_multi[t], y), t
+    assert torch.equal(st_multi, st_chain)
+    h = to64(inp["state"])
+    for t in range(ntok):
+        yr, h = oracle.step(h, inp["x"][t], inp["delta"][t], inp["A"], inp["B"][t], inp["C"][t],
+                            D=inp["D"], z=inp["z"][t])
+        assert_parity(y_multi[t], yr, din, dout, what="y[%d]" % t)
+    assert_parity(st_multi, h, din, torch.float32, what="state")
