@@ -127,9 +127,16 @@ int run_scan(const ssm::ScanArgs &a0, cudaStream_t stream) {
 // Tile shape per padded state width: 32-token tiles; 32 channels per CTA (64 at N <= 4).
 // bf16 inputs at N = 16: a 2-stage ring, 42 KB of shared memory and at most 96 registers,
 // so 5 CTAs share an SM (740 on the chip: 4 sequences x 5120 channels run in one wave).
+#ifndef SSM_SCAN16_NSTAGE
+#define SSM_SCAN16_NSTAGE 2   // ring depth of the bf16 N = 16 tile
+#endif
+#ifndef SSM_SCAN16_MINB
+#define SSM_SCAN16_MINB 5     // resident CTAs per SM its registers target
+#endif
 template <int NP, typename Tin, typename Tout, bool VEC>
 struct ScanConfig {
-    using C16 = std::conditional_t<sizeof(Tin) == 2, ssm::ScanCfg<16, 1, 32, 2, Tin, Tout, VEC, 5>,
+    using C16 = std::conditional_t<sizeof(Tin) == 2,
+                                   ssm::ScanCfg<16, 1, 32, SSM_SCAN16_NSTAGE, Tin, Tout, VEC, SSM_SCAN16_MINB>,
                                    ssm::ScanCfg<16, 1, 32, 3, Tin, Tout, VEC, 4>>;
     using C8 = ssm::ScanCfg<8, 1, 32, 3, Tin, Tout, VEC, 6>;
     using C4 = ssm::ScanCfg<4, 2, 32, 3, Tin, Tout, VEC, 6>;

@@ -76,6 +76,22 @@ def test_ssd_from_a_start_state_and_resume(cuda_lib):
     assert_ssd_close(h2, hr, "final state (resumed)")
 
 
+@pytest.mark.parametrize("scale", [5.0, 12.0])
+def test_ssd_fast_decays(cuda_lib, scale):
+    # decays scaled so that a chunk's cumulative log-decay passes -64: the in-chunk decay
+    # factors span more than the fp32 range and the carried state all but vanishes between
+    # chunks; the first chunk keeps the unscaled decays
+    inp = inputs.make_ssd_inputs(2, 300, 2, 64, 128, device=DEV, seed=int(scale))
+    a = inp["a"].clone()
+    a[:, 128:] *= scale
+    y, hN = ssm.ssd(inp["x"], a, inp["B"], inp["C"])
+    torch.cuda.synchronize()
+    yr, hr = oracle.ssd_loop(inp["x"], a, inp["B"], inp["C"])
+    assert_ssd_close(y, yr, "y")
+    assert_ssd_close(hN, hr, "final state")
+    assert cuda_lib.ssm_device_timeouts() == 0
+
+
 def test_ssd_empty_sequence_copies_the_state(cuda_lib):
     inp = inputs.make_ssd_inputs(1, 0, 2, 64, 128, device=DEV, seed=5)
     h0 = torch.randn(1, 2, 64, 128, device=DEV)
