@@ -100,10 +100,11 @@ struct ScanCfg {
     static_assert(T % 8 == 0, "tile must hold whole 8-token chunks");
     static_assert(NTASK % NTHREADS == 0, "tasks must divide evenly");
 
-    // bf16 inputs: the recurrence reads B and C of a state quad as one 16-byte word of
-    // bf16 pairs (B quad, then C quad) and widens them in registers.  A shared-memory load
-    // that all lanes of a warp share still costs one wavefront per 4 bytes, so this halves
-    // the shared-memory traffic of the recurrence against fp32 B and C rows.
+    // bf16 inputs: per (token, state quad) the recurrence reads B as 4 fp32 values (16
+    // bytes) and C as 4 bf16 values (8 bytes, widened in registers).  A shared-memory load
+    // that all lanes of a warp share still costs one wavefront per 4 bytes, so this is 6
+    // wavefronts per token and quad against 8 for fp32 B and C rows; widening only C keeps
+    // the issue slots (shared with the SFU-bound decays) for the recurrence.
     static constexpr bool BCPACK = sizeof(Tin) == 2;
 
     static constexpr size_t al(size_t v) { return (v + 15) & ~size_t(15); }
@@ -113,9 +114,10 @@ struct ScanCfg {
     static constexpr size_t OFF_RAW = 0;
     // prep: float4 [T/2][CH] = (Delta_t, Delta_t x_t, Delta_t+1, Delta_t+1 x_t+1)
     static constexpr size_t OFF_PREP = OFF_RAW + NSTAGE * STAGE_BYTES;
-    // B, C of the tile: packed uint4 [T][Q] (bf16 inputs), else fp32 rows [T][NP] each
+    // B, C of the tile: for bf16 inputs B as float4 [T][Q] and C as bf16 quads (uint2)
+    // [T][Q]; else fp32 rows [T][NP] each
     static constexpr size_t BF_BYTES = BCPACK ? al(size_t(T) * Q * 16) : al(size_t(T) * NP * sizeof(float));
-    static constexpr size_t CF_BYTES = BCPACK ? 0 : al(size_t(T) * NP * sizeof(float));
+    static constexpr size_t CF_BYTES = BCPACK ? al(size_t(T) * Q * 8) : al(size_t(T) * NP * sizeof(float));
     static constexpr size_t OFF_BF = OFF_PREP + al(size_t(T / 2) * CH * sizeof(float4));
     static constexpr size_t OFF_CF = OFF_BF + BF_BYTES;
     // quad partial sums of the readout [Q][CH][T], slot g of a row stored at g XOR (channel
@@ -361,10 +363,9 @@ scan_fwd_kernel(const ScanArgs p) {
             for (int u2 = 0; u2 < 4; ++u2)
                 prep[(4 * t8 + u2) * CH + cc] = make_float4(o[4 * u2], o[4 * u2 + 1], o[4 * u2 + 2], o[4 * u2 + 3]);
         }
-        // B, C of the tile for the recurrence, zero past dstate / past L: packed bf16 quads
-        // (B quad, C quad) per (token, quad) for bf16 inputs, else fp32 rows
+        // B, C of the tile for the recurrence, zero past dstate / past L: per (token, quad)
+        // the B quad in fp32 and the C quad as bf16 for bf16 inputs, else fp32 rows
         if constexpr (Cfg::BCPACK) {
-            uint4 *bcp = reinterpret_cast<uint4 *>(Bf);
             const unsigned short *rb = reinterpret_cast<const unsigned short *>(sv.bs);
             const unsigned short *rc = reinterpret_cast<const unsigned short *>(sv.cs);
 #pragma unroll
@@ -389,7 +390,10 @@ scan_fwd_kernel(const ScanArgs p) {
                         v = make_uint4(bw[0] | (bw[1] << 16), bw[2] | (bw[3] << 16),
                                        cw[0] | (cw[1] << 16), cw[2] | (cw[3] << 16));
                     }
-                    bcp[i] = v;
+                    reinterpret_cast<float4 *>(Bf)[i] =
+                        make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                                    __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+                    reinterpret_cast<uint2 *>(Cf)[i] = make_uint2(v.z, v.w);
                 }
             }
         } else if (N == NP && t0 + T <= L) {                // dense rows: 8 values at a time
@@ -423,14 +427,13 @@ scan_fwd_kernel(const ScanArgs p) {
         {
             const float4 *pp = prep + c;
             float4 *ypr = reinterpret_cast<float4 *>(yp) + (q * CH + c) * Cfg::YP_SLOTS;
-            const uint4 *bcp = reinterpret_cast<const uint4 *>(Bf) + q;
             // the B and C quads of token t as fp32 pairs (0,1), (2,3)
             auto bquad = [&](int t, float2 (&bb)[2], uint2 &craw) {
                 if constexpr (Cfg::BCPACK) {
-                    const uint4 v = bcp[t * Cfg::Q];
-                    bb[0] = bf16x2_to_f2(v.x);
-                    bb[1] = bf16x2_to_f2(v.y);
-                    craw = make_uint2(v.z, v.w);
+                    const float4 bq = reinterpret_cast<const float4 *>(Bf)[t * Cfg::Q + q];
+                    bb[0] = f2(bq.x, bq.y);
+                    bb[1] = f2(bq.z, bq.w);
+                    craw = reinterpret_cast<const uint2 *>(Cf)[t * Cfg::Q + q];
                 } else {
                     const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
                     bb[0] = f2(bq.x, bq.y);
