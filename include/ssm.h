@@ -290,8 +290,8 @@ int ssm_state_step_multi(float *state, const void *x, const void *delta, const f
  * operands with fp32 accumulation; the masked scores, the decay-weighted inputs and the
  * state are rounded to bf16 where they enter a product.  The state stays on the chip
  * between chunks (fp32): the call allocates nothing and writes only y and final_state.
- * seqlen = 0 copies the start state through.  Uses up to 227 KB of shared memory and 512
- * tensor-memory columns per CTA (one CTA per SM).
+ * seqlen = 0 copies the start state through.  Uses about 100 KB of shared memory and 256
+ * tensor-memory columns per CTA (two CTAs per SM).
  */
 int ssm_ssd_fwd(const void *x, const float *a, const void *B, const void *C, void *y,
                 const float *initial_state, float *final_state,

@@ -62,7 +62,9 @@ int launch_ssd(const void *x, const void *B, const void *C, ssm::SsdTcArgs a, cu
     if (cudaGetSymbolAddress(&counter, g_wait_timeouts) != cudaSuccess) return SSM_ERR_CUDA;
     a.timeouts = static_cast<unsigned *>(counter);
     if (cudaFuncSetAttribute(ssm::ssd_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(Cfg::SMEM_BYTES)) != cudaSuccess)
+                             int(Cfg::SMEM_BYTES)) != cudaSuccess ||
+        cudaFuncSetAttribute(ssm::ssd_tc_kernel<Cfg>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
         return SSM_ERR_CUDA;
     ssm::ssd_tc_kernel<Cfg><<<unsigned(ctas), Cfg::NT, Cfg::SMEM_BYTES, s>>>(mx, mb, mc, a);
     return status_of(cudaGetLastError());
