@@ -151,9 +151,9 @@ __global__ void __launch_bounds__(256) state_step_kernel(const StepArgs p) {
 //
 // A block holds kStepThreads consecutive channels and walks the sequences b = slice,
 // slice + slices, ... (blockIdx.x = slice * dblocks + channel block), so A and D stay in
-// registers for all of them, and the next sequence's state and first tokens are loaded
-// into registers while the current one is computed, so loads stay in flight through the
-// whole kernel instead of only at its start.  Per round of up to kStepsRound tokens the
+// registers for all of them, and while the current sequence is computed the next one's
+// state row streams into a shared ring (cp.async) and its first tokens into registers, so
+// loads stay in flight through the whole kernel instead of only at its start.  Per round of up to kStepsRound tokens the
 // block stages the sequence's B and C rows in shared memory (padded to NP with zeros),
 // read back as 16-byte broadcasts.
 //
@@ -173,7 +173,7 @@ template <int G> __device__ __forceinline__ float quad_sum(const float (&s)[G]) 
 }
 
 #ifndef SSM_STEPS_MINB
-#define SSM_STEPS_MINB 4     // resident blocks per SM the registers target
+#define SSM_STEPS_MINB 5     // resident blocks per SM the registers target
 #endif
 template <int NP, typename Tin, typename Tout, bool VEC4>
 __global__ void __launch_bounds__(kStepThreads, SSM_STEPS_MINB) state_steps_kernel(const StepArgs p, int dblocks) {
@@ -248,25 +248,59 @@ __global__ void __launch_bounds__(kStepThreads, SSM_STEPS_MINB) state_steps_kern
         return v;
     };
 
+    // whole quads (N % 4 == 0): the next sequence's state row goes into a 2-slot shared
+    // ring with cp.async, each thread copying and reading back only its own row, so the
+    // prefetch holds no registers (5 blocks per SM fit); otherwise into registers
+    constexpr bool RING = VEC4;
+    constexpr int RPL = 8 / G;
+    __shared__ __align__(16) float4 sring[RING ? 2 : 1][kStepThreads * G];
+    const int tid = int(threadIdx.x);
+    auto slot = [&](int q) { return tid * G + (q ^ ((tid / RPL) & (G - 1))); };
+    auto ring_issue = [&](long long bq, int st) {
+        if constexpr (RING) {
+            if (act && bq < p.batch) {
+                const float *hs = state_row(int(bq));
+#pragma unroll
+                for (int q = 0; q < G; ++q)
+                    if (4 * q < N) cp_async_16(&sring[st][slot(q)], hs + 4 * q);
+            }
+            cp_async_commit();
+        }
+    };
+
     // the first sequence's state and first round, then one sequence ahead
-    float hn[G][4];
+    float hn[RING ? 1 : G][4];
     Tin xn[R], dn[R], zn[R];
     float bcn = 0.f;
+    ring_issue(slice, 0);
     if (slice < p.batch) {
-        load_state(slice, hn);
+        if constexpr (!RING) load_state(slice, *reinterpret_cast<float (*)[G][4]>(&hn[0][0]));
         load_tokens(slice, 0, xn, dn, zn);
         bcn = load_bc(slice, 0);
     }
-    for (int b = slice; b < p.batch; b += slices) {
+    int it = 0;
+    for (int b = slice; b < p.batch; b += slices, ++it) {
         float h[G][4];
+        if constexpr (RING) {
+            ring_issue((long long)b + slices, (it + 1) & 1);
+            cp_async_wait<1>();                          // this sequence's row has landed
 #pragma unroll
-        for (int n = 0; n < NP; ++n) h[n / 4][n % 4] = hn[n / 4][n % 4];
+            for (int q = 0; q < G; ++q) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (act && 4 * q < N) v = sring[it & 1][slot(q)];
+                h[q][0] = v.x; h[q][1] = v.y; h[q][2] = v.z; h[q][3] = v.w;
+            }
+        } else {
+            const float (&hp)[G][4] = *reinterpret_cast<const float (*)[G][4]>(&hn[0][0]);
+#pragma unroll
+            for (int n = 0; n < NP; ++n) h[n / 4][n % 4] = hp[n / 4][n % 4];
+        }
         Tin xq[R], dq[R], zq[R];
 #pragma unroll
         for (int tt = 0; tt < R; ++tt) { xq[tt] = xn[tt]; dq[tt] = dn[tt]; zq[tt] = zn[tt]; }
         float bcv = bcn;
         if ((long long)b + slices < p.batch) {
-            load_state(b + slices, hn);
+            if constexpr (!RING) load_state(b + slices, *reinterpret_cast<float (*)[G][4]>(&hn[0][0]));
             load_tokens(b + slices, 0, xn, dn, zn);
             bcn = load_bc(b + slices, 0);
         }
@@ -311,6 +345,7 @@ __global__ void __launch_bounds__(kStepThreads, SSM_STEPS_MINB) state_steps_kern
                 if (act && n < N) hs[n] = h[n / 4][n % 4];
         }
     }
+    if constexpr (RING) cp_async_wait<0>();
 }
 
 }  // namespace ssm
