@@ -573,11 +573,107 @@ def count_kernel_nodes(graph):
         return None
 
 
+def time_e2e_scan(wl, steps):
+    """time_e2e for the whole-sequence scan, pipelined over slices of the batch (or, for
+    one sequence, of the channels): per slice, its inputs go up on one stream, its scan
+    runs on a second and its outputs come back on a third, so that the two copy
+    directions overlap each other and the scans.  Every step still copies all of its
+    inputs from pinned host memory and reads all of its outputs back."""
+    import torch
+    import selective_state_space_45_b200 as ssm
+    dev = wl.sets[0]
+    batch, dim, L = dev["x"].shape
+    names_in = ["x", "delta", "z", "B", "C", "A", "D", "delta_bias"]
+    host = {}
+    for n in names_in:
+        host[n] = torch.empty(dev[n].shape, dtype=dev[n].dtype, pin_memory=True)
+        host[n].copy_(dev[n])
+    outs = {n: torch.empty(dev[n].shape, dtype=dev[n].dtype, pin_memory=True) for n in ("y", "fs")}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    if batch >= 2:                      # one slice per sequence; shared parameters with the first
+        slices = [(b, b + 1, 0, dim) for b in range(batch)]
+        shared = ["A", "D", "delta_bias"]
+    else:                               # one sequence: four channel ranges; B, C with the first
+        k = 4
+        cuts = [dim * i // k for i in range(k + 1)]
+        slices = [(0, 1, cuts[i], cuts[i + 1]) for i in range(k)]
+        shared = ["B", "C"]
+
+    def view(t, n, sl):
+        b0, b1, d0, d1 = sl
+        if n in ("A",):
+            return t[d0:d1]
+        if n in ("D", "delta_bias"):
+            return t[d0:d1]
+        if n in ("B", "C"):
+            return t[b0:b1]
+        return t[b0:b1, d0:d1]
+
+    s_up, s_run, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ns = len(slices)
+    ev_up = [torch.cuda.Event() for _ in range(ns)]
+    ev_run = [torch.cuda.Event() for _ in range(ns)]
+    ev_down = [torch.cuda.Event() for _ in range(ns)]
+    main = torch.cuda.current_stream()
+    for e in ev_up + ev_run + ev_down:
+        e.record(main)
+
+    def one():
+        for i, sl in enumerate(slices):
+            s_up.wait_event(ev_run[i])          # this slice's inputs are free again
+            with torch.cuda.stream(s_up):
+                for n in names_in:
+                    if n in shared and i > 0:
+                        continue
+                    if n in shared:             # every slice's scan reads these: wait for them
+                        s_up.wait_event(ev_run[ns - 1])
+                    view(dev[n], n, sl if n not in shared else (0, batch, 0, dim)).copy_(
+                        view(host[n], n, sl if n not in shared else (0, batch, 0, dim)), non_blocking=True)
+                ev_up[i].record(s_up)
+            s_run.wait_event(ev_up[i])
+            s_run.wait_event(ev_up[0])
+            s_run.wait_event(ev_down[i])        # this slice's outputs have been read back
+            b0, b1, d0, d1 = sl
+            ssm.ssm_selective_scan_fwd(view(dev["x"], "x", sl), view(dev["delta"], "delta", sl),
+                                       view(dev["delta_bias"], "delta_bias", sl), True,
+                                       view(dev["A"], "A", sl), view(dev["B"], "B", sl),
+                                       view(dev["C"], "C", sl), view(dev["D"], "D", sl),
+                                       view(dev["z"], "z", sl), view(dev["y"], "y", sl),
+                                       view(dev["fs"], "fs", sl), stream=s_run)
+            ev_run[i].record(s_run)
+            s_down.wait_event(ev_run[i])
+            with torch.cuda.stream(s_down):
+                for n in ("y", "fs"):
+                    view(outs[n], n, sl).copy_(view(dev[n], n, sl), non_blocking=True)
+                ev_down[i].record(s_down)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for st in (s_up, s_run, s_down):
+        st.wait_event(e0)
+    for _ in range(steps):
+        one()
+    for st in (s_up, s_run, s_down):
+        main.wait_stream(st)
+    e1.record(main)
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) / 1e3
+    return dict(value=wl.counts["tokch"] * steps / sec, unit=UNIT, h2d_bytes_per_step=h2d,
+                d2h_bytes_per_step=d2h, ms_per_step=1e3 * sec / steps,
+                pipeline="%d slices: uploads, scans and read-backs on three streams" % ns)
+
+
 def time_e2e(wl, steps, stream):
     """The same metric through the public API with HOST buffers: every step copies its
     inputs from pinned host memory, runs the call and reads the outputs back."""
     import torch
     import selective_state_space_45_b200 as ssm
+    if wl.kind == "scan":
+        return time_e2e_scan(wl, steps)
     dev = wl.sets[0]
     # per-token inputs of the decode kinds are [steps, ...]: one token's slice travels
     per_token = {"decode": ("x", "delta", "z", "B", "C"), "convstep": ("x",),
