@@ -125,3 +125,17 @@ def test_ssd130m_sampled_heads(cuda_lib):
         assert_ssd_close(y[b:b + 1, :, h:h + 1], yr, "y (b=%d, h=%d)" % (b, h))
         assert_ssd_close(hN[b:b + 1, h:h + 1], hr, "final state (b=%d, h=%d)" % (b, h))
     assert cuda_lib.ssm_device_timeouts() == 0
+
+
+def test_ssd_more_ctas_than_resident_slots(cuda_lib):
+    # 16 x 24 = 384 (sequence, head) CTAs: more than two per SM, so a second wave starts as
+    # CTAs of the first finish; sampled heads from both waves against the oracle
+    inp = inputs.make_ssd_inputs(16, 300, 24, 64, 128, device=DEV, seed=9)
+    y, hN = ssm.ssd(inp["x"], inp["a"], inp["B"], inp["C"])
+    torch.cuda.synchronize()
+    for b, h in [(0, 0), (6, 5), (12, 17), (15, 23)]:
+        sl = {k: v[b:b + 1, :, h:h + 1].contiguous() for k, v in inp.items()}
+        yr, hr = oracle.ssd_loop(sl["x"], sl["a"], sl["B"], sl["C"])
+        assert_ssd_close(y[b:b + 1, :, h:h + 1], yr, "y (b=%d, h=%d)" % (b, h))
+        assert_ssd_close(hN[b:b + 1, h:h + 1], hr, "final state (b=%d, h=%d)" % (b, h))
+    assert cuda_lib.ssm_device_timeouts() == 0

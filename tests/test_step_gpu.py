@@ -163,11 +163,15 @@ def test_multi_token_step_small_dims_span_many_sequences(cuda_lib, batch, dim, N
 
 
 @pytest.mark.parametrize("ntok,N,din,dout", [(6, 16, torch.bfloat16, torch.bfloat16),
-                                             (9, 8, torch.float32, torch.float32)])
+                                             (9, 8, torch.float32, torch.float32),
+                                             (5, 12, torch.bfloat16, torch.float32),
+                                             (7, 5, torch.float32, torch.bfloat16)])
 def test_multi_token_step_blocks_walk_many_sequences(cuda_lib, ntok, N, din, dout):
     # more sequences than the resident blocks of a channel range: each block walks several,
-    # loading the next one's state and first tokens while it computes the current one; the
-    # last channel range is ragged (3000 = 23 x 128 + 56)
+    # loading the next one's state and first tokens while it computes the current one (the
+    # state through the shared ring when N is a multiple of 4, else through registers; N =
+    # 12 leaves the last quad of the padded 16 empty); the last channel range is ragged
+    # (3000 = 23 x 128 + 56)
     batch, dim = 96, 3000
     inp = inputs.make_decode_inputs(batch, dim, N, ntok, din, device=DEV, seed=ntok + N)
     st_multi = inp["state"].clone()
