@@ -68,36 +68,7 @@ __device__ __forceinline__ float silu_f(float z) {
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 ex2_pair(float2 v) { return f2(ex2_approx(v.x), ex2_approx(v.y)); }
-
-// 2^v for a pair of values on the FMA pipe instead of the SFU, so that a share of the
-// decays can be taken off the SFU, the scan's bottleneck.  Range reduction: v is clamped
-// to [-126, 126] (the result stays a normal number: 2^-126 where the SFU's flush-to-zero
-// ex2 gives 0, a difference far below a state's resolution), the nearest integer r of v
-// comes from adding 1.5 * 2^23 (round to nearest in the low mantissa bits), f = v - r is
-// exact and lies in [-1/2, 1/2].  2^f is a degree-5 polynomial fitted here to 2^f on
-// [-1/2, 1/2] by iterated reweighted least squares on relative error (max relative error
-// 2.3e-7 in fp32 Horner form, about the SFU's own), and r is added to the exponent field
-// with an integer add.  The coefficients are pinned by tests/test_poly_exp2.py.
-__device__ __forceinline__ float2 exp2_poly_pair(float2 v) {
-    constexpr float kRound = 12582912.f;   // 1.5 * 2^23
-    v.x = fminf(fmaxf(v.x, -126.f), 126.f);
-    v.y = fminf(fmaxf(v.y, -126.f), 126.f);
-    const float2 t = fadd2(v, f2(kRound, kRound));
-    const float2 r = fadd2(t, f2(-kRound, -kRound));
-    const float2 f = ffma2(r, f2(-1.f, -1.f), v);
-    float2 q = f2(1.327647129073739e-3f, 1.327647129073739e-3f);
-    q = ffma2(q, f, f2(9.675541892647743e-3f, 9.675541892647743e-3f));
-    q = ffma2(q, f, f2(5.550713092088699e-2f, 5.550713092088699e-2f));
-    q = ffma2(q, f, f2(2.4022120237350464e-1f, 2.4022120237350464e-1f));
-    q = ffma2(q, f, f2(6.931469440460205e-1f, 6.931469440460205e-1f));
-    q = ffma2(q, f, f2(1.0000001192092896f, 1.0000001192092896f));
-    // the low bits of t hold r (two's complement); shifted by 23 they add r to the exponent
-    const unsigned ex = __float_as_uint(q.x) + (__float_as_uint(t.x) << 23);
-    const unsigned ey = __float_as_uint(q.y) + (__float_as_uint(t.y) << 23);
-    return f2(__uint_as_float(ex), __uint_as_float(ey));
-}
 
 // A pair of bf16 values packed in 32 bits (first in the low half) as an fp32 pair: bf16 ->
 // fp32 is a 16-bit shift (exact).
