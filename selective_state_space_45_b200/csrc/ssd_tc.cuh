@@ -67,7 +67,8 @@ struct SsdTcCfg {
     static constexpr uint32_t OFF_ZERO = OFF_S + 128 * XROW;  // a zero [Q][64] block (N = 64)
     static constexpr uint32_t OFF_CUM = OFF_ZERO + (N == 64 ? BC_BLOCK : 0);   // cum [Q], totals
     static constexpr uint32_t OFF_EA = OFF_CUM + 4 * (Q + 8);                   // e^{a} [Q]
-    static constexpr uint32_t OFF_BAR = OFF_EA + 4 * Q;
+    static constexpr uint32_t OFF_EAI = OFF_EA + 4 * Q;                         // e^{-a} [Q]
+    static constexpr uint32_t OFF_BAR = OFF_EAI + 4 * Q;
     static constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;   // + alignment slack
     static constexpr uint32_t TX_BYTES = X_BYTES + 2 * NB * BC_BLOCK;
     // tensor memory columns: G (then D), Yc, Yi
@@ -104,6 +105,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *cum = reinterpret_cast<float *>(smem + Cfg::OFF_CUM);           // [Q] + warp totals
     float *ea = reinterpret_cast<float *>(smem + Cfg::OFF_EA);             // e^{a_s} [Q]
+    float *eai = reinterpret_cast<float *>(smem + Cfg::OFF_EAI);           // e^{-a_s} [Q]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *bar_tma = bars + 0, *bar_g = bars + 1, *bar_d = bars + 2, *bar_yi = bars + 3;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4);
@@ -214,6 +216,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         float cs = a_next;
         a_next = load_a(c + 1);
         ea[row] = ex2_approx(cs * kLog2e);
+        eai[row] = ex2_approx(-cs * kLog2e);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float u = __shfl_up_sync(0xffffffffu, cs, o);
@@ -279,8 +282,18 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                     m[e] = __uint_as_float(graw[e]) * dec;
                     dec *= ea[s0b + e];
                 }
+            } else if (fabsf(cum[s0b] - cum[s0b + 31]) <= 80.f) {
+                // the diagonal block, its 32 decays within a factor e^80: one exponential
+                // for the first column, then e^{cum_l - cum_(s+1)} = e^{cum_l - cum_s} e^{-a_(s+1)}
+                // up the columns (0 above the diagonal, whatever the product there)
+                float dec = ex2_approx((cs - cum[s0b]) * kLog2e);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    m[e] = s0b + e <= row ? __uint_as_float(graw[e]) * dec : 0.f;
+                    if (e < 31) dec *= eai[s0b + e + 1];
+                }
             } else {
-                // the diagonal block: one exponential per score, 0 above the diagonal
+                // the diagonal block otherwise: one exponential per score
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int s = s0b + e;
