@@ -88,6 +88,8 @@ struct BwdCfg {
     static constexpr int G_ROW = T + EG;
     static constexpr int P_ROW = T + 4;         // per-quad partial rows (floats)
     static constexpr int X_ROW = 36;            // transpose rows: conflict-free both ways
+    static constexpr bool BCPACK = sizeof(Tin) == 2;   // B, C staged as bf16 quads
+    static_assert(!BCPACK || T * Q <= NT, "one thread per packed (token, quad)");
     static constexpr int TW = 4;                // tokens per (t, d) task
     static constexpr int NTW = T / TW;          // task chunks per row
     static constexpr int NTASK = CH * NTW;      // (channel, token chunk) tasks per tile
@@ -246,21 +248,65 @@ __device__ __forceinline__ void bwd_prep(const BwdArgs &p, const BwdStage<Cfg> &
     }
 }
 
-// B (and C when `both`) of the tile widened to fp32 [T][NP], zero past dstate and past L.
+// B (and C when `both`) of the tile, zero past dstate and past L: for bf16 inputs as bf16
+// quads (8 bytes per (token, state quad): the recurrence reads them as 8-byte broadcasts,
+// half the shared-memory wavefronts of fp32 quads, and widens them in registers), else
+// widened to fp32 [T][NP].
 template <class Cfg>
 __device__ __forceinline__ void bwd_widen_bc(const BwdArgs &p, const BwdStage<Cfg> &sv, float *Bf,
                                              float *Cf, int t0, bool both) {
-    constexpr int T = Cfg::T, NP = Cfg::NP, NT = Cfg::NT;
+    constexpr int T = Cfg::T, NP = Cfg::NP, NT = Cfg::NT, Q = Cfg::Q;
     const int L = p.seqlen, N = p.dstate;
+    if constexpr (Cfg::BCPACK) {
+        const unsigned short *rb = reinterpret_cast<const unsigned short *>(sv.bs);
+        const unsigned short *rc = reinterpret_cast<const unsigned short *>(sv.cs);
+        const int i = tid_x();
+        if (i < T * Q) {
+            const int tt = i / Q, qq = i % Q;
+            uint2 b2 = make_uint2(0u, 0u), c2 = make_uint2(0u, 0u);
+            if (N == NP && t0 + tt < L) {            // dense rows: 8-byte reads
+                b2 = *reinterpret_cast<const uint2 *>(rb + tt * NP + 4 * qq);
+                if (both) c2 = *reinterpret_cast<const uint2 *>(rc + tt * NP + 4 * qq);
+            } else {
+                unsigned bw[4], cw[4];
 #pragma unroll
-    for (int k = 0; k < (T * NP + NT - 1) / NT; ++k) {
-        const int i = tid_x() + k * NT;
-        if (i < T * NP) {
-            const int tt = i / NP, n = i % NP;
-            const bool ok = n < N && t0 + tt < L;
-            Bf[i] = ok ? to_f32(sv.bs[tt * N + n]) : 0.f;
-            if (both) Cf[i] = ok ? to_f32(sv.cs[tt * N + n]) : 0.f;
+                for (int e = 0; e < 4; ++e) {
+                    const int n = 4 * qq + e;
+                    const bool ok = n < N && t0 + tt < L;
+                    bw[e] = ok ? rb[tt * N + n] : 0u;
+                    cw[e] = (ok && both) ? rc[tt * N + n] : 0u;
+                }
+                b2 = make_uint2(bw[0] | (bw[1] << 16), bw[2] | (bw[3] << 16));
+                c2 = make_uint2(cw[0] | (cw[1] << 16), cw[2] | (cw[3] << 16));
+            }
+            reinterpret_cast<uint2 *>(Bf)[i] = b2;
+            if (both) reinterpret_cast<uint2 *>(Cf)[i] = c2;
         }
+    } else {
+#pragma unroll
+        for (int k = 0; k < (T * NP + NT - 1) / NT; ++k) {
+            const int i = tid_x() + k * NT;
+            if (i < T * NP) {
+                const int tt = i / NP, n = i % NP;
+                const bool ok = n < N && t0 + tt < L;
+                Bf[i] = ok ? to_f32(sv.bs[tt * N + n]) : 0.f;
+                if (both) Cf[i] = ok ? to_f32(sv.cs[tt * N + n]) : 0.f;
+            }
+        }
+    }
+}
+
+// The B (or C) quad q of token t from the tile's staging as fp32 pairs (0,1), (2,3).
+template <class Cfg>
+__device__ __forceinline__ void bwd_quad(const float *Xf, int t, int q, float2 (&v)[2]) {
+    if constexpr (Cfg::BCPACK) {
+        const uint2 w = reinterpret_cast<const uint2 *>(Xf)[t * Cfg::Q + q];
+        v[0] = bf16x2_to_f2(w.x);
+        v[1] = bf16x2_to_f2(w.y);
+    } else {
+        const float4 x4 = *reinterpret_cast<const float4 *>(Xf + t * Cfg::NP + 4 * q);
+        v[0] = f2(x4.x, x4.y);
+        v[1] = f2(x4.z, x4.w);
     }
 }
 
@@ -343,8 +389,8 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
         for (int t = 0; t < T; ++t) {
             if (t % 4 == 0) *ck(tile * (T / 4) + t / 4) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
             const float4 pv = prep[t * CH + c];
-            const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
-            const float2 bb[2] = {f2(bq.x, bq.y), f2(bq.z, bq.w)};
+            float2 bb[2];
+            bwd_quad<Cfg>(Bf, t, q, bb);
             const float2 dl2 = f2(pv.x, pv.x);
             const float dx = pv.x * pv.y;
             const float2 dx2 = f2(dx, dx);
@@ -412,10 +458,9 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
                 const int t = 4 * j + u;
                 const float4 pv = prep[t * CH + c];
                 dl[u] = pv.x; xv[u] = pv.y; dyp[u] = pv.z;
-                const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
-                const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
-                const float2 bb[2] = {f2(bq.x, bq.y), f2(bq.z, bq.w)};
-                const float2 cb[2] = {f2(cq.x, cq.y), f2(cq.z, cq.w)};
+                float2 bb[2], cb[2];
+                bwd_quad<Cfg>(Bf, t, q, bb);
+                bwd_quad<Cfg>(Cf, t, q, cb);
                 const float2 dl2 = f2(dl[u], dl[u]);
                 const float dx = dl[u] * xv[u];
                 const float2 dx2 = f2(dx, dx);
@@ -433,10 +478,9 @@ __global__ void __launch_bounds__(Cfg::NT, 3) scan_bwd_kernel(const BwdArgs p) {
 #pragma unroll
             for (int u = 3; u >= 0; --u) {
                 const int t = 4 * j + u;
-                const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
-                const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
-                const float2 bb[2] = {f2(bq.x, bq.y), f2(bq.z, bq.w)};
-                const float2 cb[2] = {f2(cq.x, cq.y), f2(cq.z, cq.w)};
+                float2 bb[2], cb[2];
+                bwd_quad<Cfg>(Bf, t, q, bb);
+                bwd_quad<Cfg>(Cf, t, q, cb);
                 const float dlx = dl[u] * xv[u];
                 const float2 dyp2 = f2(dyp[u], dyp[u]), dlx2 = f2(dlx, dlx), dl2 = f2(dl[u], dl[u]);
                 // sum_n lambda B_n gives both dx (times Delta) and, times x, the B part of
