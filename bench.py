@@ -52,7 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2p8b",
-                    choices=["mamba130m", "mamba2p8b", "long1m", "long1m_slow", "decode", "tiny",
+                    choices=["mamba130m", "mamba2p8b", "mamba2p8b_d4736", "mamba2p8b_d5920",
+                             "long1m", "long1m_slow", "decode", "tiny",
                              "conv130m", "conv2p8b", "convstep", "bwd130m", "decode4", "ssd130m"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")

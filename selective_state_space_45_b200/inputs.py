@@ -50,6 +50,13 @@ CONFIGS = {
                       dt_dist="uniform"),
     "mamba2p8b": dict(batch=4, seqlen=4096, dim=5120, dstate=16, dtype=torch.bfloat16,
                       dt_dist="loguniform"),
+    # the 2.8b shape with d_inner set so that the grid of 32-channel CTAs fills the 148 SMs
+    # evenly: 592 CTAs (4 per SM) and 740 CTAs (5 per SM); the 2.8b shape's own 640 CTAs
+    # leave 48 SMs with a fifth CTA
+    "mamba2p8b_d4736": dict(batch=4, seqlen=4096, dim=4736, dstate=16, dtype=torch.bfloat16,
+                            dt_dist="loguniform"),
+    "mamba2p8b_d5920": dict(batch=4, seqlen=4096, dim=5920, dstate=16, dtype=torch.bfloat16,
+                            dt_dist="loguniform"),
     "long1m": dict(batch=1, seqlen=1 << 20, dim=1536, dstate=16, dtype=torch.bfloat16,
                    dt_dist="uniform"),
     "long1m_slow": dict(batch=1, seqlen=1 << 20, dim=1536, dstate=16, dtype=torch.bfloat16,
