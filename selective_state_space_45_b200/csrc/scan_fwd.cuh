@@ -101,10 +101,10 @@ struct ScanCfg {
     static_assert(NTASK % NTHREADS == 0, "tasks must divide evenly");
 
     // bf16 inputs: per (token, state quad) the recurrence reads B as 4 fp32 values (16
-    // bytes) and C as 4 bf16 values (8 bytes, widened in registers).  A shared-memory load
-    // that all lanes of a warp share still costs one wavefront per 4 bytes, so this is 6
-    // wavefronts per token and quad against 8 for fp32 B and C rows; widening only C keeps
-    // the issue slots (shared with the SFU-bound decays) for the recurrence.
+    // bytes) and C as 4 bf16 values (8 bytes, widened in registers).  A 16-byte shared load
+    // that all lanes of a warp share still takes two wavefronts (an 8-byte one takes one),
+    // so this is 3 wavefronts per token and quad against 4 for fp32 B and C rows; widening
+    // only C keeps the issue slots (shared with the SFU-bound decays) for the recurrence.
     static constexpr bool BCPACK = sizeof(Tin) == 2;
 
     static constexpr size_t al(size_t v) { return (v + 15) & ~size_t(15); }
