@@ -59,6 +59,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0,
                     help="CPU seconds the oracle baseline may spend")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="scan workloads: force this many time segments per sequence "
+                         "(ssm_scan_force_segments; 0 = the library's own choice)")
     return ap.parse_args(argv)
 
 
@@ -755,6 +758,10 @@ def run_ours(args):
     dist = init_dist(world, "nccl")
     import selective_state_space_45_b200 as ssm
     ssm.load_library()
+    if args.segments:
+        if workload_kind(args.workload) != "scan":
+            raise SystemExit("bench.py: --segments applies to the scan workloads only")
+        ssm.ssm_scan_force_segments(args.segments)
 
     wl = Workload(args.workload, device, seed=rank)
     stream = torch.cuda.Stream(device)
@@ -807,7 +814,7 @@ def run_ours(args):
         achieved = wl.counts["exps"] / kern_s / 1e9
         roof = dict(bound="alu", achieved=achieved, peak=peak_gexp, unit="Gexp/s",
                     frac=achieved / peak_gexp,
-                    traffic=recorded_traffic(kernel_name(wl.kind), wl.name),
+                    traffic=None if args.segments else recorded_traffic(kernel_name(wl.kind), wl.name),
                     kernel=kernel_name(wl.kind), kernel_ms=kern_ms,
                     peak_basis=("148 SMs x 16 ex2/clk/SM x %.0f MHz max SM clock; the 16 ex2/clk/SM "
                                 "is the SFU rate of the CUDA programming guide's throughput table "
@@ -851,6 +858,8 @@ def run_ours(args):
             config.update(heads=c["heads"], headdim=c["headdim"], chunk=128)
         if "seqlen" in c:
             config.update(seqlen=c["seqlen"], global_batch=c["batch"] * world)
+        if wl.kind == "scan":
+            config.update(segments=args.segments if args.segments else "auto")
         line = dict(metric=METRIC, value=total_units / sec, unit=UNIT, n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=1e3 * sec / args.steps, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype="f32",
