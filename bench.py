@@ -748,6 +748,27 @@ def time_e2e(wl, steps, stream):
                 d2h_bytes_per_step=d2h, ms_per_step=1e3 * sec / steps)
 
 
+def sfu_probe_rate(ssm, device, stream, sm_mhz):
+    """The SFU ex2 rate measured on this GPU by the library's probe (ssm_sfu_probe: 8
+    independent ex2 chains per thread, 2048 threads per SM), timed with CUDA events on the
+    launching stream.  Reported beside the derived peak, not used as the denominator."""
+    import torch
+    blocks, iters = N_SM * 8, 4096
+    out = torch.empty(blocks * 256, device=device, dtype=torch.float32)
+    ssm.ssm_sfu_probe(out, blocks, 64, stream)             # load and warm up
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        ssm.ssm_sfu_probe(out, blocks, iters, stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) / 1e3
+    n = blocks * 256 * 8 * iters
+    return dict(gexp_s=n / sec / 1e9, ex2_per_clk_per_sm=n / sec / (N_SM * sm_mhz * 1e6),
+                at_sm_mhz=sm_mhz, ex2=n, ms=1e3 * sec)
+
+
 def run_ours(args):
     import torch
     rank, world, local = dist_env()
@@ -818,10 +839,12 @@ def run_ours(args):
                     kernel=kernel_name(wl.kind), kernel_ms=kern_ms,
                     peak_basis=("148 SMs x 16 ex2/clk/SM x %.0f MHz max SM clock; the 16 ex2/clk/SM "
                                 "is the SFU rate of the CUDA programming guide's throughput table "
-                                "for compute capability 10.x, not measured by this script"
+                                "for compute capability 10.x; sfu_probe measures it on this GPU"
                                 % peaks["sm_max_mhz"]),
                     hbm=dict(achieved_gbs=gbs, peak_gbs=peaks["hbm_gbs"], frac=gbs / peaks["hbm_gbs"],
-                             peak_source=peaks["source"]))
+                             peak_source=peaks["source"]),
+                    sfu_probe=sfu_probe_rate(ssm, device, stream,
+                                             clocks.get("sm_mhz") or peaks["sm_max_mhz"]))
     elif wl.kind == "ssd":
         tfl = wl.counts["flops"] / kern_s / 1e12
         roof = dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",

@@ -307,6 +307,17 @@ int ssm_ssd_fwd(const void *x, const float *a, const void *B, const void *C, voi
  */
 unsigned ssm_device_timeouts(void);
 
+/*
+ * Diagnostic, not part of the path: the SFU exponential rate that the scan's roofline
+ * counts against (decays are SFU ex2 operations).  Launches `blocks` CTAs of 256 threads;
+ * each thread runs 8 independent chains v <- 2^(-v) for `iters` steps (one ex2 each, the
+ * values staying in [0.5, 1]) and writes the sum of its chains to out[thread] (`out`:
+ * device, blocks * 256 floats, 16-byte aligned, owned by the caller).  blocks * 256 * 8 *
+ * iters ex2 in all; time the call with events on `cuda_stream`.  SSM_ERR_INVALID_ARG for a
+ * NULL `out`, blocks < 1 or iters < 0; asynchronous like every call.
+ */
+int ssm_sfu_probe(float *out, int blocks, int iters, void *cuda_stream);
+
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char *ssm_status_string(int status);
 

@@ -28,6 +28,7 @@ from ._lib import (  # noqa: F401
     ssm_selective_scan_fwd_ex,
     ssm_selective_scan_fwd_noalloc,
     ssm_scan_force_segments,
+    ssm_sfu_probe,
     ssm_ssd_fwd,
     ssm_state_step,
     ssm_state_step_multi,

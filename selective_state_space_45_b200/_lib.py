@@ -73,6 +73,8 @@ def load_library(path: str | None = None):
         lib.ssm_device_timeouts.argtypes = []
         lib.ssm_scan_force_segments.restype = i
         lib.ssm_scan_force_segments.argtypes = [i]
+        lib.ssm_sfu_probe.restype = i
+        lib.ssm_sfu_probe.argtypes = [vp, i, i, vp]
         _lib = lib
         return lib
 
@@ -89,6 +91,15 @@ def ssm_device_timeouts() -> int:
     """How many bounded waits inside the library's kernels gave up on this device (0 in
     normal operation; see include/ssm.h).  Synchronises with the device."""
     return int(load_library().ssm_device_timeouts())
+
+
+def ssm_sfu_probe(out, blocks, iters, stream=None):
+    """Diagnostic SFU throughput probe (see include/ssm.h): ``blocks`` CTAs of 256 threads,
+    8 ex2 chains of ``iters`` steps per thread; ``out`` is a CUDA fp32 tensor of at least
+    blocks * 256 elements.  Asynchronous on ``stream``."""
+    if out.dtype.itemsize != 4 or out.numel() < int(blocks) * 256:
+        raise ValueError("out must hold blocks * 256 fp32 values")
+    _check(load_library().ssm_sfu_probe(_ptr(out), int(blocks), int(iters), _stream(stream, out)))
 
 
 def ssm_scan_force_segments(segments: int) -> int:

@@ -235,6 +235,18 @@ def test_step_multi_argument_checks(lib, kw, status):
                                     args["dout"], None) == status
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(out=None), ssm.SSM_ERR_INVALID_ARG),
+    (dict(blocks=0), ssm.SSM_ERR_INVALID_ARG),
+    (dict(iters=-1), ssm.SSM_ERR_INVALID_ARG),
+    (dict(out=MIS), ssm.SSM_ERR_ALIGNMENT),
+])
+def test_sfu_probe_argument_checks(lib, kw, status):
+    args = dict(out=P, blocks=1, iters=1)
+    args.update(kw)
+    assert lib.ssm_sfu_probe(args["out"], args["blocks"], args["iters"], None) == status
+
+
 def test_python_binding_raises_on_error(lib):
     with pytest.raises(ssm.SsmError) as e:
         ssm._lib._check(ssm.SSM_ERR_UNSUPPORTED)
