@@ -18,15 +18,17 @@
 //   TMA      x [Q][P], B and C [Q][N] (64-state column blocks) into one buffer set
 //   MMA 1    G  = C B^T                (tensor-memory columns 0 .. Q-1)
 //   MMA 2    Yc = C S^T                (columns Q .. Q+P-1)
-//   CUDA     cumulative decays (computed before the tiles are waited for); masked scores
-//            M = G o e^{cum_l - cum_s} (s <= l) written as bf16 over C, whose products are
-//            done -- below the diagonal block as a running product of e^{a_s} from one
-//            exponential per 32 columns; B's rows scaled in place by w_s = e^{cum_end - cum_s}
+//   CUDA     masked scores M = G o e^{cum_l - cum_s} (s <= l) written as bf16 over C, whose
+//            products are done -- below the diagonal block as a running product of e^{a_s}
+//            from one exponential per 32 columns; B's rows scaled in place by
+//            w_s = e^{cum_end - cum_s}
 //   MMA 3    D  = (w o B)^T x          (columns 0 .. P-1: G has been read)
 //   MMA 4    Yi = M x                  (columns Q+P .. Q+2P-1)
 //   CUDA     the next chunk's loads go out once MMA 4 is done (its tiles were sent
-//            towards L2 when this chunk's MMA 1 was issued); S' = e^{cum_end} S + D;
-//            y = Yi + e^{cum_l} Yc
+//            towards L2 when this chunk's MMA 1 was issued); S' = e^{cum_end} S + D; the
+//            next chunk's cumulative decays; once its tiles land, its MMA 1 (D has been
+//            read, so G's columns are free) runs while this chunk's y = Yi + e^{cum_l} Yc
+//            is written; its MMA 2 follows once Yc has been read
 // So a CTA holds one buffer set (~98 KB of shared memory at P = 64, N = 128) and 256
 // tensor-memory columns: two CTAs fit on an SM, and one CTA's loads and barriers overlap
 // the other's products and row-wise work.  Every mbarrier wait is bounded; a CTA whose
@@ -207,14 +209,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
     };
     int w_tma = 0, w_g = 0, w_d = 0, w_yi = 0;
     float a_next = load_a(0);
-    bool ok = true;
-    int c = 0;
-    for (; c < nchunk; ++c) {
-        const int t = c * Q + row;
-        // the chunk's decays: inclusive cumulative sum over the chunk (zero past L), before
-        // its tiles are needed
-        float cs = a_next;
-        a_next = load_a(c + 1);
+    // the decays of chunk cc: inclusive cumulative sum over the chunk (zero past L) into
+    // cum[], e^{a} and e^{-a} into ea[], eai[]; this row's cum (cs), e^{cum} (el) and the
+    // chunk's total (tot).  One barrier inside; cum[] is read after the next one.
+    float cs = 0.f, el = 1.f, tot = 0.f;
+    auto chunk_decays = [&](int cc) {
+        cs = a_next;
+        a_next = load_a(cc + 1);
         ea[row] = ex2_approx(cs * kLog2e);
         eai[row] = ex2_approx(-cs * kLog2e);
 #pragma unroll
@@ -225,33 +226,49 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         if (lane == 31) cum[Q + warp] = cs;
         __syncthreads();
         for (int w = 0; w < warp; ++w) cs += cum[Q + w];
-        const float tot = cum[Q] + cum[Q + 1] + cum[Q + 2] + cum[Q + 3];
+        tot = cum[Q] + cum[Q + 1] + cum[Q + 2] + cum[Q + 3];
         cum[row] = cs;
-        const float el = ex2_approx(cs * kLog2e);
-        // cum[] and ea[] are read after the next barrier (the wait for the tiles)
-        // chunk c's tiles have landed: G = C B^T, Yc = C S^T (S: the state entering chunk c)
-        if (!(ok = wait_all(bar_tma, w_tma))) break;
-        if (tid == 0) {
-            tc_fence_after_sync();
+        el = ex2_approx(cs * kLog2e);
+    };
+    // MMA 1 (G = C B^T) of chunk cc, whose tiles have landed; and the L2 prefetch of the
+    // chunk after it
+    auto issue_g = [&](int cc) {
+        tc_fence_after_sync();
 #pragma unroll
-            for (int k = 0; k < N / 16; ++k) {
-                const uint32_t koff = (k >> 2) * Cfg::BC_BLOCK + (k & 3) * 32;
-                umma_bf16(tmem + Cfg::TM_G, at(dsc_cm, koff), at(dsc_b, koff), ID_G, k > 0);
-                umma_bf16(tmem + Cfg::TM_YC, at(dsc_cm, koff), at(dsc_s, k * MN_KSTEP), ID_YC, k > 0);
-            }
-            umma_commit(bar_g);
-            ++n_g;
-            // the next chunk's tiles start towards L2 now, so that their loads (issued
-            // once this chunk's products are done) find them there
-            if (c + 1 < nchunk) {
-                tma_prefetch_l2_4d(&tm_x, 0, h, (c + 1) * Q, b);
+        for (int k = 0; k < N / 16; ++k) {
+            const uint32_t koff = (k >> 2) * Cfg::BC_BLOCK + (k & 3) * 32;
+            umma_bf16(tmem + Cfg::TM_G, at(dsc_cm, koff), at(dsc_b, koff), ID_G, k > 0);
+        }
+        if (cc + 1 < nchunk) {
+            tma_prefetch_l2_4d(&tm_x, 0, h, (cc + 1) * Q, b);
 #pragma unroll
-                for (int k = 0; k < NB; ++k) {
-                    tma_prefetch_l2_4d(&tm_b, 64 * k, h, (c + 1) * Q, b);
-                    tma_prefetch_l2_4d(&tm_c, 64 * k, h, (c + 1) * Q, b);
-                }
+            for (int k = 0; k < NB; ++k) {
+                tma_prefetch_l2_4d(&tm_b, 64 * k, h, (cc + 1) * Q, b);
+                tma_prefetch_l2_4d(&tm_c, 64 * k, h, (cc + 1) * Q, b);
             }
         }
+    };
+    // MMA 2 (Yc = C S^T, S the state entering the chunk), then one commit for MMAs 1 and 2:
+    // the masking waits for both, since it overwrites C
+    auto issue_yc = [&]() {
+        tc_fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < N / 16; ++k) {
+            const uint32_t koff = (k >> 2) * Cfg::BC_BLOCK + (k & 3) * 32;
+            umma_bf16(tmem + Cfg::TM_YC, at(dsc_cm, koff), at(dsc_s, k * MN_KSTEP), ID_YC, k > 0);
+        }
+        umma_commit(bar_g);
+        ++n_g;
+    };
+    chunk_decays(0);
+    bool ok = wait_all(bar_tma, w_tma);
+    if (ok && tid == 0) {
+        issue_g(0);
+        issue_yc();
+    }
+    int c = 0;
+    for (; ok && c < nchunk; ++c) {
+        const int t = c * Q + row;
 
         // masked scores from G (row l): e^{cum_l - cum_s} for s <= l, 0 above, as bf16 over
         // C (its products are complete); then B's row s times w_s = e^{tot - cum_s}
@@ -364,6 +381,17 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
             for (int e = 0; e < P; ++e) S[e] = fmaf(dtot, S[e], __uint_as_float(d[e]));
             write_state();
         }
+        // the next chunk's decays, and its MMA 1 once its tiles land (G's columns are free:
+        // D has been read), so that the product runs while this chunk's y is written
+        const float el_c = el;
+        const bool more = c + 1 < nchunk;
+        if (more) {
+            chunk_decays(c + 1);
+            fence_async_smem();
+            tc_fence_before_sync();
+            if (!(ok = wait_all(bar_tma, w_tma))) break;
+            if (tid == 0) issue_g(c + 1);
+        }
         // y = Yi + e^{cum_l} Yc, row l
         {
             Tout *yrow = static_cast<Tout *>(p.y) + ((size_t(b) * L + t) * H + h) * P;
@@ -375,18 +403,19 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
                 tmem_wait_ld();
                 float yv[PW];
 #pragma unroll
-                for (int e = 0; e < PW; ++e) yv[e] = fmaf(el, __uint_as_float(ycr[e]), __uint_as_float(yir[e]));
+                for (int e = 0; e < PW; ++e) yv[e] = fmaf(el_c, __uint_as_float(ycr[e]), __uint_as_float(yir[e]));
                 if (t < L) {
 #pragma unroll
                     for (int e = 0; e < PW; e += 8) store_run<8>(yrow + j + e, yv + e);
                 }
             }
         }
-        // the new S copy reaches the next chunk's MMA 2; every tensor-memory read of this
-        // chunk is done before the next chunk's products overwrite G, Yc and Yi
+        // every tensor-memory read of Yc and Yi is done before the next chunk's MMA 2 and
+        // MMA 4 overwrite them; the new S copy reaches MMA 2
         fence_async_smem();
         tc_fence_before_sync();
         __syncthreads();
+        if (more && tid == 0) issue_yc();
     }
     if (ok) {
         if (p.hN != nullptr && row < N) {
