@@ -26,10 +26,10 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
-// log1p(u) for u in [0, 1], as u * p(u) with p a degree-7 polynomial fitted to log1p(u)/u
-// (least squares at Chebyshev nodes, relative weighting).  Evaluated in fp32 Horner form
-// its relative error is below 3.3e-7 on the whole interval.
-__device__ __forceinline__ float log1p_unit(float u) {
+// log1p(u) for u in [0, 1] is u * p(u), p a degree-7 polynomial fitted to log1p(u)/u (least
+// squares at Chebyshev nodes, relative weighting).  Evaluated in fp32 Horner form u * p(u)
+// has a relative error below 3.3e-7 on the whole interval.  log1p_poly gives p(u).
+__device__ __forceinline__ float log1p_poly(float u) {
     float p = -0.008336497470736504f;
     p = fmaf(p, u, 0.04337085038423538f);
     p = fmaf(p, u, -0.10667790472507477f);
@@ -38,13 +38,14 @@ __device__ __forceinline__ float log1p_unit(float u) {
     p = fmaf(p, u, 0.3327118754386902f);
     p = fmaf(p, u, -0.49997127056121826f);
     p = fmaf(p, u, 0.9999997615814209f);
-    return u * p;
+    return p;
 }
 
-// softplus(v) = log(1 + e^v), in the overflow-free form max(v, 0) + log1p(e^-|v|):
-// one SFU exponential, the logarithm on the FMA pipe.
+// softplus(v) = log(1 + e^v), in the overflow-free form max(v, 0) + log1p(e^-|v|): one SFU
+// exponential, the logarithm on the FMA pipe, its last product fused with the sum.
 __device__ __forceinline__ float softplus_f(float v) {
-    return fmaxf(v, 0.f) + log1p_unit(ex2_approx(-fabsf(v) * kLog2e));
+    const float u = ex2_approx(-fabsf(v) * kLog2e);
+    return fmaf(u, log1p_poly(u), fmaxf(v, 0.f));
 }
 
 // expm1(v) for |v| < 0.1 from its Taylor series through v^5 (truncation below 1.4e-8
@@ -69,6 +70,28 @@ __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 ex2_pair(float2 v) { return f2(ex2_approx(v.x), ex2_approx(v.y)); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// softplus_f and silu_f on two values at once: the same operations in the same order on
+// each half, the FP32 ones as packed pairs (each half rounded as its scalar counterpart),
+// so the results are bit-identical to the scalar functions'.
+__device__ __forceinline__ float2 softplus_pair(float2 v) {
+    const float2 u = f2(ex2_approx(-fabsf(v.x) * kLog2e), ex2_approx(-fabsf(v.y) * kLog2e));
+    float2 p = f2(-0.008336497470736504f, -0.008336497470736504f);
+    p = ffma2(p, u, f2(0.04337085038423538f, 0.04337085038423538f));
+    p = ffma2(p, u, f2(-0.10667790472507477f, -0.10667790472507477f));
+    p = ffma2(p, u, f2(0.1767549365758896f, 0.1767549365758896f));
+    p = ffma2(p, u, f2(-0.2447046935558319f, -0.2447046935558319f));
+    p = ffma2(p, u, f2(0.3327118754386902f, 0.3327118754386902f));
+    p = ffma2(p, u, f2(-0.49997127056121826f, -0.49997127056121826f));
+    p = ffma2(p, u, f2(0.9999997615814209f, 0.9999997615814209f));
+    return ffma2(u, p, f2(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f)));
+}
+__device__ __forceinline__ float2 silu_pair(float2 z) {
+    const float2 e = ex2_pair(fmul2(z, f2(-kLog2e, -kLog2e)));
+    const float2 d = fadd2(f2(1.f, 1.f), e);
+    return fmul2(z, f2(rcp_approx(d.x), rcp_approx(d.y)));
+}
 
 // A pair of bf16 values packed in 32 bits (first in the low half) as an fp32 pair: bf16 ->
 // fp32 is a 16-bit shift (exact).

@@ -342,11 +342,13 @@ scan_fwd_kernel(const ScanArgs p) {
             float o[16];
             if (cc < nch && t0 + 8 * t8 + 8 <= L) {          // whole chunk inside the data
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    float dl = dr[u] + bias;
-                    if (p.softplus) dl = softplus_f(dl);
-                    o[2 * u] = dl;
-                    o[2 * u + 1] = ZOH ? xr[u] : dl * xr[u];
+                for (int u = 0; u < 8; u += 2) {                // tokens in pairs, packed FP32
+                    float2 dl = fadd2(f2(dr[u], dr[u + 1]), f2(bias, bias));
+                    if (p.softplus) dl = softplus_pair(dl);
+                    const float2 xv = f2(xr[u], xr[u + 1]);
+                    const float2 dx = ZOH ? xv : fmul2(dl, xv);
+                    o[2 * u] = dl.x; o[2 * u + 1] = dx.x;
+                    o[2 * u + 2] = dl.y; o[2 * u + 3] = dx.y;
                 }
             } else {
                 const bool cok = cc < nch;
@@ -530,26 +532,31 @@ scan_fwd_kernel(const ScanArgs p) {
         for (int k = 0; k < Cfg::TASKS_PER_THREAD; ++k) {
             const int task = tid + k * NT;
             const int cc = task % CH, t8 = task / CH;
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            // tokens in pairs, packed FP32: the quads' partials summed in order, the skip,
+            // the gate
+            float2 acc2[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
             for (int qq = 0; qq < Q; ++qq) {
                 const float4 *row = reinterpret_cast<const float4 *>(yp) + (qq * CH + cc) * Cfg::YP_SLOTS;
                 const float4 a0 = row[(2 * t8) ^ (cc & 7)];
                 const float4 a1 = row[(2 * t8 + 1) ^ (cc & 7)];
-                acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
-                acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
+                acc2[0] = fadd2(acc2[0], f2(a0.x, a0.y)); acc2[1] = fadd2(acc2[1], f2(a0.z, a0.w));
+                acc2[2] = fadd2(acc2[2], f2(a1.x, a1.y)); acc2[3] = fadd2(acc2[3], f2(a1.z, a1.w));
             }
             float xr[8];
             stage_row8<Cfg>(sv.xs, cc, t8, xr);
             const float Dd = tD[k];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) acc[u] = fmaf(Dd, xr[u], acc[u]);
+            for (int j = 0; j < 4; ++j) acc2[j] = ffma2(f2(Dd, Dd), f2(xr[2 * j], xr[2 * j + 1]), acc2[j]);
             if (p.z != nullptr) {
                 float zr[8];
                 stage_row8<Cfg>(sv.zs, cc, t8, zr);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) acc[u] *= silu_f(zr[u]);
+                for (int j = 0; j < 4; ++j) acc2[j] = fmul2(acc2[j], silu_pair(f2(zr[2 * j], zr[2 * j + 1])));
             }
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) { acc[2 * j] = acc2[j].x; acc[2 * j + 1] = acc2[j].y; }
             const int tg = t0 + 8 * t8;
             if (cc < nch) {
                 if (Cfg::VEC && tg + 8 <= L) {
