@@ -26,18 +26,34 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
+// Packed FP32 pairs (sm_100: one instruction does two FP32 FMAs / sums / products, each
+// rounded as fmaf / a plain sum or product would be).  Used where independent values pair up.
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 ex2_pair(float2 v) { return f2(ex2_approx(v.x), ex2_approx(v.y)); }
+
+// A constant shaped like v, and one Horner step p * u + c, on a value or on a pair of
+// values (c the same for both halves).
+__device__ __forceinline__ float splat(float, float c) { return c; }
+__device__ __forceinline__ float2 splat(float2, float c) { return f2(c, c); }
+__device__ __forceinline__ float horner(float p, float u, float c) { return fmaf(p, u, c); }
+__device__ __forceinline__ float2 horner(float2 p, float2 u, float c) { return ffma2(p, u, f2(c, c)); }
+
 // log1p(u) for u in [0, 1] is u * p(u), p a degree-7 polynomial fitted to log1p(u)/u (least
 // squares at Chebyshev nodes, relative weighting).  Evaluated in fp32 Horner form u * p(u)
-// has a relative error below 3.3e-7 on the whole interval.  log1p_poly gives p(u).
-__device__ __forceinline__ float log1p_poly(float u) {
-    float p = -0.008336497470736504f;
-    p = fmaf(p, u, 0.04337085038423538f);
-    p = fmaf(p, u, -0.10667790472507477f);
-    p = fmaf(p, u, 0.1767549365758896f);
-    p = fmaf(p, u, -0.2447046935558319f);
-    p = fmaf(p, u, 0.3327118754386902f);
-    p = fmaf(p, u, -0.49997127056121826f);
-    p = fmaf(p, u, 0.9999997615814209f);
+// has a relative error below 3.3e-7 on the whole interval.  log1p_poly gives p(u), for one
+// value or a pair (each half rounded exactly as the single value is).
+template <typename V> __device__ __forceinline__ V log1p_poly(V u) {
+    V p = splat(u, -0.008336497470736504f);
+    p = horner(p, u, 0.04337085038423538f);
+    p = horner(p, u, -0.10667790472507477f);
+    p = horner(p, u, 0.1767549365758896f);
+    p = horner(p, u, -0.2447046935558319f);
+    p = horner(p, u, 0.3327118754386902f);
+    p = horner(p, u, -0.49997127056121826f);
+    p = horner(p, u, 0.9999997615814209f);
     return p;
 }
 
@@ -64,28 +80,12 @@ __device__ __forceinline__ float silu_f(float z) {
     return z * rcp_approx(1.f + ex2_approx(-z * kLog2e));
 }
 
-// Packed FP32 pairs (sm_100: one instruction does two FP32 FMAs / products, each rounded
-// as fmaf / a plain product would be).  Used where independent states pair up.
-__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 ex2_pair(float2 v) { return f2(ex2_approx(v.x), ex2_approx(v.y)); }
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-
 // softplus_f and silu_f on two values at once: the same operations in the same order on
-// each half, the FP32 ones as packed pairs (each half rounded as its scalar counterpart),
-// so the results are bit-identical to the scalar functions'.
+// each half, the FP32 ones as packed pairs, so the results are bit-identical to the scalar
+// functions'.
 __device__ __forceinline__ float2 softplus_pair(float2 v) {
     const float2 u = f2(ex2_approx(-fabsf(v.x) * kLog2e), ex2_approx(-fabsf(v.y) * kLog2e));
-    float2 p = f2(-0.008336497470736504f, -0.008336497470736504f);
-    p = ffma2(p, u, f2(0.04337085038423538f, 0.04337085038423538f));
-    p = ffma2(p, u, f2(-0.10667790472507477f, -0.10667790472507477f));
-    p = ffma2(p, u, f2(0.1767549365758896f, 0.1767549365758896f));
-    p = ffma2(p, u, f2(-0.2447046935558319f, -0.2447046935558319f));
-    p = ffma2(p, u, f2(0.3327118754386902f, 0.3327118754386902f));
-    p = ffma2(p, u, f2(-0.49997127056121826f, -0.49997127056121826f));
-    p = ffma2(p, u, f2(0.9999997615814209f, 0.9999997615814209f));
-    return ffma2(u, p, f2(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f)));
+    return ffma2(u, log1p_poly(u), f2(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f)));
 }
 __device__ __forceinline__ float2 silu_pair(float2 z) {
     const float2 e = ex2_pair(fmul2(z, f2(-kLog2e, -kLog2e)));
