@@ -100,13 +100,6 @@ struct ScanCfg {
     static_assert(T % 8 == 0, "tile must hold whole 8-token chunks");
     static_assert(NTASK % NTHREADS == 0, "tasks must divide evenly");
 
-    // bf16 inputs: per (token, state quad) the recurrence reads B as 4 fp32 values (16
-    // bytes) and C as 4 bf16 values (8 bytes, widened in registers).  A 16-byte shared load
-    // that all lanes of a warp share still takes two wavefronts (an 8-byte one takes one),
-    // so this is 3 wavefronts per token and quad against 4 for fp32 B and C rows; widening
-    // only C keeps the issue slots (shared with the SFU-bound decays) for the recurrence.
-    static constexpr bool BCPACK = sizeof(Tin) == 2;
-
     static constexpr size_t al(size_t v) { return (v + 15) & ~size_t(15); }
     static constexpr size_t RAW_ARR = al(size_t(CH) * RAW_ROW * sizeof(Tin));
     static constexpr size_t RAW_BC = al(size_t(T) * NP * sizeof(Tin));
@@ -114,10 +107,11 @@ struct ScanCfg {
     static constexpr size_t OFF_RAW = 0;
     // prep: float4 [T/2][CH] = (Delta_t, Delta_t x_t, Delta_t+1, Delta_t+1 x_t+1)
     static constexpr size_t OFF_PREP = OFF_RAW + NSTAGE * STAGE_BYTES;
-    // B, C of the tile: for bf16 inputs B as float4 [T][Q] and C as bf16 quads (uint2)
-    // [T][Q]; else fp32 rows [T][NP] each
-    static constexpr size_t BF_BYTES = BCPACK ? al(size_t(T) * Q * 16) : al(size_t(T) * NP * sizeof(float));
-    static constexpr size_t CF_BYTES = BCPACK ? al(size_t(T) * Q * 8) : al(size_t(T) * NP * sizeof(float));
+    // B, C of the tile widened to fp32 rows [T][NP] once per tile, so that the recurrence
+    // reads each state quad as one 16-byte broadcast (two shared-memory wavefronts for a
+    // warp) and spends no instruction on widening
+    static constexpr size_t BF_BYTES = al(size_t(T) * NP * sizeof(float));
+    static constexpr size_t CF_BYTES = al(size_t(T) * NP * sizeof(float));
     static constexpr size_t OFF_BF = OFF_PREP + al(size_t(T / 2) * CH * sizeof(float4));
     static constexpr size_t OFF_CF = OFF_BF + BF_BYTES;
     // quad partial sums of the readout [Q][CH][T], slot g of a row stored at g XOR (channel
@@ -365,16 +359,18 @@ scan_fwd_kernel(const ScanArgs p) {
             for (int u2 = 0; u2 < 4; ++u2)
                 prep[(4 * t8 + u2) * CH + cc] = make_float4(o[4 * u2], o[4 * u2 + 1], o[4 * u2 + 2], o[4 * u2 + 3]);
         }
-        // B, C of the tile for the recurrence, zero past dstate / past L: per (token, quad)
-        // the B quad in fp32 and the C quad as bf16 for bf16 inputs, else fp32 rows
-        if constexpr (Cfg::BCPACK) {
+        // B, C of the tile for the recurrence as fp32 rows, zero past dstate / past L
+        if constexpr (sizeof(Tin) == 2) {
+            // bf16: one (token, state quad) per item, both quads read as 8-byte words and
+            // stored as 16-byte fp32 quads by consecutive lanes (conflict free)
+            constexpr int QD = NP / 4;
             const unsigned short *rb = reinterpret_cast<const unsigned short *>(sv.bs);
             const unsigned short *rc = reinterpret_cast<const unsigned short *>(sv.cs);
 #pragma unroll
-            for (int k = 0; k < (T * Q + NT - 1) / NT; ++k) {
+            for (int k = 0; k < (T * QD + NT - 1) / NT; ++k) {
                 const int i = tid + k * NT;
-                if (i < T * Q) {
-                    const int tt = i / Q, qq = i % Q;
+                if (i < T * QD) {
+                    const int tt = i / QD, qq = i % QD;
                     uint4 v;
                     if (N == NP && t0 + tt < L) {            // dense rows: two 8-byte reads
                         const uint2 b2 = *reinterpret_cast<const uint2 *>(rb + tt * NP + 4 * qq);
@@ -395,7 +391,9 @@ scan_fwd_kernel(const ScanArgs p) {
                     reinterpret_cast<float4 *>(Bf)[i] =
                         make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
                                     __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
-                    reinterpret_cast<uint2 *>(Cf)[i] = make_uint2(v.z, v.w);
+                    reinterpret_cast<float4 *>(Cf)[i] =
+                        make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u),
+                                    __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
                 }
             }
         } else if (N == NP && t0 + T <= L) {                // dense rows: 8 values at a time
@@ -429,34 +427,15 @@ scan_fwd_kernel(const ScanArgs p) {
         {
             const float4 *pp = prep + c;
             float4 *ypr = reinterpret_cast<float4 *>(yp) + (q * CH + c) * Cfg::YP_SLOTS;
-            // the B and C quads of token t as fp32 pairs (0,1), (2,3)
-            auto bquad = [&](int t, float2 (&bb)[2], uint2 &craw) {
-                if constexpr (Cfg::BCPACK) {
-                    const float4 bq = reinterpret_cast<const float4 *>(Bf)[t * Cfg::Q + q];
-                    bb[0] = f2(bq.x, bq.y);
-                    bb[1] = f2(bq.z, bq.w);
-                    craw = reinterpret_cast<const uint2 *>(Cf)[t * Cfg::Q + q];
-                } else {
-                    const float4 bq = *reinterpret_cast<const float4 *>(Bf + t * NP + 4 * q);
-                    bb[0] = f2(bq.x, bq.y);
-                    bb[1] = f2(bq.z, bq.w);
-                    craw = make_uint2(0u, 0u);
-                }
-            };
-            auto cquad = [&](int t, uint2 craw, float2 (&cc)[2]) {
-                if constexpr (Cfg::BCPACK) {
-                    cc[0] = bf16x2_to_f2(craw.x);
-                    cc[1] = bf16x2_to_f2(craw.y);
-                } else {
-                    const float4 cq = *reinterpret_cast<const float4 *>(Cf + t * NP + 4 * q);
-                    cc[0] = f2(cq.x, cq.y);
-                    cc[1] = f2(cq.z, cq.w);
-                }
+            // the B or C quad of token t (fp32 rows) as pairs (0,1), (2,3)
+            auto quad = [&](const float *X, int t, float2 (&v)[2]) {
+                const float4 x4 = *reinterpret_cast<const float4 *>(X + t * NP + 4 * q);
+                v[0] = f2(x4.x, x4.y);
+                v[1] = f2(x4.z, x4.w);
             };
             // decays a = exp(Delta*A) and writes w = Delta*x*B of the 4 tokens of group g, as
-            // state pairs (0,1), (2,3) for the packed FP32 instructions; the C quads (packed
-            // form) are kept for the readout
-            auto decay_write = [&](int g, float2 (&a)[4][2], float2 (&w)[4][2], uint2 (&cr)[4]) {
+            // state pairs (0,1), (2,3) for the packed FP32 instructions
+            auto decay_write = [&](int g, float2 (&a)[4][2], float2 (&w)[4][2]) {
                 const float4 d01 = pp[(2 * g) * CH];   // (Delta, Delta*x or x) of tokens 4g, 4g+1
                 const float4 d23 = pp[(2 * g + 1) * CH];
                 const float dl[4] = {d01.x, d01.z, d23.x, d23.z};
@@ -464,7 +443,7 @@ scan_fwd_kernel(const ScanArgs p) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     float2 bb[2];
-                    bquad(4 * g + u, bb, cr[u]);
+                    quad(Bf, 4 * g + u, bb);
                     const float2 dl2 = f2(dl[u], dl[u]);
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
@@ -487,12 +466,12 @@ scan_fwd_kernel(const ScanArgs p) {
                     }
                 }
             };
-            auto recur_read = [&](int g, const float2 (&a)[4][2], const float2 (&w)[4][2], const uint2 (&cr)[4]) {
+            auto recur_read = [&](int g, const float2 (&a)[4][2], const float2 (&w)[4][2]) {
                 float out[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     float2 cc2[2];
-                    cquad(4 * g + u, cr[u], cc2);
+                    quad(Cf, 4 * g + u, cc2);
                     float2 acc = f2(0.f, 0.f);
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
@@ -506,18 +485,15 @@ scan_fwd_kernel(const ScanArgs p) {
             // decays and writes of the next 4 tokens are computed before the recurrence
             // of the current 4, so the SFU work overlaps the FFMA chain
             float2 a0[4][2], w0[4][2];
-            uint2 c0[4];
-            decay_write(0, a0, w0, c0);
+            decay_write(0, a0, w0);
 #pragma unroll
             for (int g = 0; g < T / 4; ++g) {
                 float2 a1[4][2], w1[4][2];
-                uint2 c1[4];
-                if (g + 1 < T / 4) decay_write(g + 1, a1, w1, c1);
-                recur_read(g, a0, w0, c0);
+                if (g + 1 < T / 4) decay_write(g + 1, a1, w1);
+                recur_read(g, a0, w0);
                 if (g + 1 < T / 4) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        c0[u] = c1[u];
 #pragma unroll
                         for (int k = 0; k < 2; ++k) { a0[u][k] = a1[u][k]; w0[u][k] = w1[u][k]; }
                     }
