@@ -105,14 +105,15 @@ struct ScanCfg {
     static constexpr size_t RAW_BC = al(size_t(T) * NP * sizeof(Tin));
     static constexpr size_t STAGE_BYTES = 3 * RAW_ARR + 2 * RAW_BC;
     static constexpr size_t OFF_RAW = 0;
-    // prep: float4 [T/2][CH] = (Delta_t, Delta_t x_t, Delta_t+1, Delta_t+1 x_t+1)
+    // prep: Delta as fp32 rows [CH][T], 4-token slot g of channel c's row stored at
+    // g XOR (c mod 8) as the partial rows are; the recurrence takes x from the staged rows
     static constexpr size_t OFF_PREP = OFF_RAW + NSTAGE * STAGE_BYTES;
     // B, C of the tile widened to fp32 rows [T][NP] once per tile, so that the recurrence
     // reads each state quad as one 16-byte broadcast (two shared-memory wavefronts for a
     // warp) and spends no instruction on widening
     static constexpr size_t BF_BYTES = al(size_t(T) * NP * sizeof(float));
     static constexpr size_t CF_BYTES = al(size_t(T) * NP * sizeof(float));
-    static constexpr size_t OFF_BF = OFF_PREP + al(size_t(T / 2) * CH * sizeof(float4));
+    static constexpr size_t OFF_BF = OFF_PREP + al(size_t(CH) * T * sizeof(float));
     static constexpr size_t OFF_CF = OFF_BF + BF_BYTES;
     // quad partial sums of the readout [Q][CH][T], slot g of a row stored at g XOR (channel
     // mod 8): the recurrence's 16-byte writes (lanes over channels) and the epilogue's reads
@@ -323,26 +324,25 @@ scan_fwd_kernel(const ScanArgs p) {
         }
         Stage<Cfg> sv(smem, st);
 
-        // ---- prep: Delta and Delta*x once per (t, d); task = (channel, 8-token chunk),
-        //      lanes run over channels so the 16-byte row reads and writes are conflict free
+        // ---- prep: Delta once per (t, d); task = (channel, 8-token chunk), lanes run over
+        //      channels so the 16-byte row reads and writes are conflict free.  No-op tokens
+        //      (past L or past dim) get Delta = 0 and a staged x of 0, so that they leave the
+        //      state as it is.
 #pragma unroll
         for (int k = 0; k < Cfg::TASKS_PER_THREAD; ++k) {
             const int task = tid + k * NT;
             const int cc = task % CH, t8 = task / CH;
-            float dr[8], xr[8];
+            float dr[8];
             stage_row8<Cfg>(sv.ds, cc, t8, dr);
-            stage_row8<Cfg>(sv.xs, cc, t8, xr);
             const float bias = tbias[k];
-            float o[16];
+            float o[8];
             if (cc < nch && t0 + 8 * t8 + 8 <= L) {          // whole chunk inside the data
 #pragma unroll
                 for (int u = 0; u < 8; u += 2) {                // tokens in pairs, packed FP32
                     float2 dl = fadd2(f2(dr[u], dr[u + 1]), f2(bias, bias));
                     if (p.softplus) dl = softplus_pair(dl);
-                    const float2 xv = f2(xr[u], xr[u + 1]);
-                    const float2 dx = ZOH ? xv : fmul2(dl, xv);
-                    o[2 * u] = dl.x; o[2 * u + 1] = dx.x;
-                    o[2 * u + 2] = dl.y; o[2 * u + 3] = dx.y;
+                    o[u] = dl.x;
+                    o[u + 1] = dl.y;
                 }
             } else {
                 const bool cok = cc < nch;
@@ -350,14 +350,14 @@ scan_fwd_kernel(const ScanArgs p) {
                 for (int u = 0; u < 8; ++u) {
                     float dl = dr[u] + bias;
                     if (p.softplus) dl = softplus_f(dl);
-                    const bool ok = cok && (t0 + 8 * t8 + u < L);   // past L / dim: no-op token
-                    o[2 * u] = ok ? dl : 0.f;
-                    o[2 * u + 1] = ok ? (ZOH ? xr[u] : dl * xr[u]) : 0.f;
+                    const bool ok = cok && (t0 + 8 * t8 + u < L);
+                    o[u] = ok ? dl : 0.f;
+                    if (!ok) sv.xs[Cfg::raw_at(cc, 8 * t8 + u)] = Tin(0.f);
                 }
             }
-#pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2)
-                prep[(4 * t8 + u2) * CH + cc] = make_float4(o[4 * u2], o[4 * u2 + 1], o[4 * u2 + 2], o[4 * u2 + 3]);
+            float4 *prow = prep + cc * Cfg::YP_SLOTS;
+            prow[(2 * t8) ^ (cc & 7)] = make_float4(o[0], o[1], o[2], o[3]);
+            prow[(2 * t8 + 1) ^ (cc & 7)] = make_float4(o[4], o[5], o[6], o[7]);
         }
         // B, C of the tile for the recurrence as fp32 rows, zero past dstate / past L
         if constexpr (sizeof(Tin) == 2) {
@@ -425,7 +425,8 @@ scan_fwd_kernel(const ScanArgs p) {
 
         // ---- the recurrence: 4 states of one channel per lane, carried across tiles ----
         {
-            const float4 *pp = prep + c;
+            const float4 *pp = prep + c * Cfg::YP_SLOTS;
+            uint4 xq = make_uint4(0u, 0u, 0u, 0u);     // staged x chunk of the current token pair
             float4 *ypr = reinterpret_cast<float4 *>(yp) + (q * CH + c) * Cfg::YP_SLOTS;
             // the B or C quad of token t (fp32 rows) as pairs (0,1), (2,3)
             auto quad = [&](const float *X, int t, float2 (&v)[2]) {
@@ -436,10 +437,20 @@ scan_fwd_kernel(const ScanArgs p) {
             // decays a = exp(Delta*A) and writes w = Delta*x*B of the 4 tokens of group g, as
             // state pairs (0,1), (2,3) for the packed FP32 instructions
             auto decay_write = [&](int g, float2 (&a)[4][2], float2 (&w)[4][2]) {
-                const float4 d01 = pp[(2 * g) * CH];   // (Delta, Delta*x or x) of tokens 4g, 4g+1
-                const float4 d23 = pp[(2 * g + 1) * CH];
-                const float dl[4] = {d01.x, d01.z, d23.x, d23.z};
-                const float dx[4] = {d01.y, d01.w, d23.y, d23.w};
+                const float4 d4 = pp[g ^ (c & 7)];     // Delta of tokens 4g .. 4g+3
+                const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
+                float xv[4];                           // x of the same tokens (staged rows)
+                if constexpr (Cfg::EIN == 8) {         // a 16-byte chunk serves two groups
+                    if ((g & 1) == 0) xq = *reinterpret_cast<const uint4 *>(sv.xs + Cfg::raw_at(c, 4 * g));
+                    const unsigned lo = (g & 1) ? xq.z : xq.x, hi = (g & 1) ? xq.w : xq.y;
+                    xv[0] = __uint_as_float(lo << 16); xv[1] = __uint_as_float(lo & 0xffff0000u);
+                    xv[2] = __uint_as_float(hi << 16); xv[3] = __uint_as_float(hi & 0xffff0000u);
+                } else {
+                    loadn<4, Tin>(sv.xs + Cfg::raw_at(c, 4 * g), xv);
+                }
+                float dx[4];                           // Delta*x (or x for the exact gain)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) dx[u] = ZOH ? xv[u] : dl[u] * xv[u];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     float2 bb[2];
