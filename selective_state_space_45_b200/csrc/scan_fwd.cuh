@@ -18,9 +18,11 @@
 //     are the same for every lane: one broadcast shared load each per token.  The quads
 //     of a channel live in different warps; their readouts are summed once per (t, d)
 //     after the tile through a shared buffer, not by shuffles inside the recurrence.
-//   * Per (t, d) work -- the softplus step and Delta*x before the scan (prep), the skip,
-//     gate and output conversion after it (epilogue) -- is done once per (t, d) by tasks
-//     of 8 tokens of one channel with 16-byte, bank-conflict-free shared accesses.
+//   * Per (t, d) work -- the softplus step before the scan (prep), the skip, gate and
+//     output conversion after it (epilogue) -- is done once per (t, d) by tasks of 8
+//     tokens of one channel with 16-byte, bank-conflict-free shared accesses, on packed
+//     FP32 pairs.  Each warp forms Delta*x itself from the staged x, and reads B_t and
+//     C_t as fp32 quads widened once per tile.
 //   * The decays and writes of the next 4 tokens are computed before the recurrence of
 //     the current 4, so SFU work overlaps the FFMA chain.
 //   * x, delta, z, B, C are staged by a cp.async ring of NSTAGE tiles (16-byte copies)
