@@ -163,3 +163,20 @@ def test_oracle_sample_and_call_for_every_workload_kind(name):
     assert kind == bench.workload_kind(name) or (kind == "scan" and name == "mamba130m")
     assert units > 0 and what
     bench._oracle_call(kind, inp, 2)
+
+
+def test_grid_fill_workloads_and_segment_option():
+    """The 2.8b shape at d_inner 4736 / 5920 (592 and 740 CTAs of 32 channels, an even 4 or
+    5 per SM on 148 SMs) are scan workloads that differ from mamba2p8b in d_inner only,
+    and --segments parses for the scan sweeps (0, the default, leaves the plan automatic)."""
+    from selective_state_space_45_b200 import inputs
+    base = inputs.CONFIGS["mamba2p8b"]
+    for name, dim in (("mamba2p8b_d4736", 4736), ("mamba2p8b_d5920", 5920)):
+        c = inputs.CONFIGS[name]
+        assert bench.workload_kind(name) == "scan"
+        assert c["dim"] == dim and 4 * (dim // 32) in (592, 740)
+        assert {k: v for k, v in c.items() if k != "dim"} == {k: v for k, v in base.items() if k != "dim"}
+        assert "d_inner %d" % dim in bench.describe_workload(name)
+        assert bench.parse_args(["--workload", name]).workload == name
+    assert bench.parse_args([]).segments == 0
+    assert bench.parse_args(["--workload", "long1m", "--segments", "8"]).segments == 8
