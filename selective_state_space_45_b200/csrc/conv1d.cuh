@@ -117,11 +117,16 @@ causal_conv1d_vec_kernel(ConvArgs a, long long nvr, long long spans_per_row, lon
         if (p < nvr) {
             float o[V];
 #pragma unroll
-            for (int t = 0; t < V; ++t) {
-                float acc = b0;
+            for (int t = 0; t < V; t += 2) {  // outputs in pairs, the gate on packed FP32
+                float2 acc = f2(b0, b0);
 #pragma unroll
-                for (int i = 0; i < K; ++i) acc = fmaf(w[i], xe[t + i], acc);
-                o[t] = a.silu ? silu_f(acc) : acc;
+                for (int i = 0; i < K; ++i) {
+                    acc.x = fmaf(w[i], xe[t + i], acc.x);
+                    acc.y = fmaf(w[i], xe[t + 1 + i], acc.y);
+                }
+                if (a.silu) acc = silu_pair(acc);
+                o[t] = acc.x;
+                o[t + 1] = acc.y;
             }
             store_run<V>(ur + p * V, o);
             if (a.hist_out && p == nvr - 1) {   // the row's last vector: the window to continue from
